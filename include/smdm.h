@@ -1,0 +1,207 @@
+/*
+ * smdm.h — C ABI of the sparse masked-diffusion sampling library (B200, sm_100a).
+ *
+ * Method: Sparse-LaViDa (arXiv 2512.14008).  At sampling step k a masked discrete diffusion
+ * model runs only a sparse row set through the transformer: the prompt and earlier decoded
+ * tokens live in an incrementally appended KV cache; the tokens decoded at step k-1 are
+ * computed once more and appended; the masked positions of the step-k decode set C get logits;
+ * n_reg register tokens with position ids L+1..L+n_reg close the sequence.  A step-causal
+ * attention mask ties the rows together.  (papernotes.org CVPR-2026 notes, "Key design 1-3"
+ * and the Figure-3 example; paperlayer.ai Sec. 3.1-3.3 and Appendix 7.2-7.3.)
+ *
+ * Conventions shared by every entry point
+ *  - All pointers named d_* are DEVICE pointers, h_* are HOST pointers.  The caller owns every
+ *    buffer (weights, workspace, inputs, outputs); the library never allocates device memory.
+ *    The handle borrows the weights and the workspace: both must outlive it.
+ *  - Every call that takes a cudaStream_t is asynchronous on that stream.  Calls on one handle
+ *    must be ordered by the caller (use one stream).  The handle's host-side bookkeeping
+ *    (cache lengths, step counters) advances when the call is made, so a sequence of calls
+ *    can be captured into a CUDA graph and replayed as a whole.
+ *  - Argument errors are detected on the host before anything is launched: the call returns a
+ *    non-zero smdm_status, leaves the state unchanged and smdm_last_error() explains why.
+ *    Device-side problems (a bounded wait that timed out, a failed bounds check) are OR-ed
+ *    into a status word that smdm_device_status() reads (it synchronises the stream).
+ *  - Positions are 1-based: prompt 1..P, generated tokens P+1..P+Lgen, registers
+ *    L+1..L+n_reg with L = P + Lgen.
+ *  - Token ids: content ids 0..vocab-1, [MASK] = vocab, [LEN] = vocab+1, register j =
+ *    vocab+2+j.  The embedding table has vocab+2+n_reg rows; the LM head covers content ids
+ *    only.  A grid (the generated part of a sequence) is int32 [Lgen], -1 = still masked.
+ *  - Weight layout: every linear weight is [out_features][in_features], input features
+ *    contiguous; dtype per smdm_config.dtype (float32 or bfloat16).
+ */
+#ifndef SMDM_H_
+#define SMDM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SMDM_OK = 0,
+  SMDM_EINVAL = 1,   /* bad argument (null pointer, out-of-range value, bad plan) */
+  SMDM_ESHAPE = 2,   /* shape not supported or beyond the configured maxima */
+  SMDM_ENOMEM = 3,   /* workspace too small */
+  SMDM_ECUDA = 4,    /* a CUDA runtime/driver call failed */
+  SMDM_ESTATE = 5,   /* call out of order (e.g. step before prefill) */
+  SMDM_ETIMEOUT = 6, /* a device-side bounded wait gave up (see smdm_device_status) */
+  SMDM_EDEVICE = 7   /* a device-side bounds check failed */
+} smdm_status;
+
+enum { SMDM_F32 = 0, SMDM_BF16 = 1 };
+enum { SMDM_POLICY_ALL = 0, SMDM_POLICY_TOPN = 1 };
+enum { SMDM_MODE_SPARSE = 0, SMDM_MODE_DENSE = 1 };
+/* Row types of a step-labelled sequence.  PROMPT/CLEAN rows are clean tokens; MASK and REG
+ * rows belong to a masked block (registers share their block's number). */
+enum { SMDM_TYPE_PROMPT = 0, SMDM_TYPE_CLEAN = 1, SMDM_TYPE_MASK = 2, SMDM_TYPE_REG = 3 };
+enum { SMDM_PLAN_ORDER = 0, SMDM_PLAN_SEMIAR = 1 };
+#define SMDM_MAX_BATCH 8
+
+/* Model and capacity.  The pages do not describe the base network; the library implements a
+ * pre-RMSNorm transformer (multi-head attention with 1-D rotate-half RoPE on the original
+ * position ids, SwiGLU MLP, untied LM head).
+ * bf16 models need d_model % 128 == 0, d_head in {64, 128}, d_ffn % 64 == 0. */
+typedef struct {
+  int n_layers, d_model, n_heads, d_head, d_ffn;
+  int vocab;         /* content vocabulary V */
+  int n_reg;         /* register tokens per step (64 in the method) */
+  int dtype;         /* SMDM_F32 or SMDM_BF16 (weights and activations) */
+  float rope_theta;  /* e.g. 10000 */
+  float rms_eps;     /* e.g. 1e-6 */
+  int max_batch;     /* sequences held at once, <= SMDM_MAX_BATCH */
+  int max_len;       /* max P + Lgen of one sequence */
+  int max_step_rows; /* max rows of one sequence in one sampling step: n_new + n_query + n_reg */
+  int max_rows;      /* max rows of any single forward: a batched step (sum over sequences),
+                        a prefill (P), a dense step (P + Lgen, per sequence) or a
+                        training-form forward (n) */
+} smdm_config;
+
+/* Device pointers to the weights (borrowed).  Per-layer fields are HOST arrays of n_layers
+ * device pointers; the library copies the pointer arrays at create. */
+typedef struct {
+  const void* emb;        /* [vocab + 2 + n_reg][d] */
+  const void* final_norm; /* [d] */
+  const void* lm_head;    /* [vocab][d] */
+  const void* const* attn_norm; /* [d] */
+  const void* const* w_qkv;     /* [3d][d]: rows 0..d-1 -> q, d..2d-1 -> k, 2d..3d-1 -> v;
+                                   head h owns rows h*d_head .. h*d_head + d_head - 1 of each */
+  const void* const* w_o;       /* [d][d] */
+  const void* const* mlp_norm;  /* [d] */
+  const void* const* w_gate;    /* [d_ffn][d] */
+  const void* const* w_up;      /* [d_ffn][d] */
+  const void* const* w_down;    /* [d][d_ffn] */
+} smdm_weights;
+
+typedef struct smdm_handle smdm_handle;
+
+/* Bytes of device workspace the handle needs (KV caches for max_batch sequences, activations,
+ * RoPE table, reduction scratch).  Returns 0 for an invalid config. */
+size_t smdm_workspace_bytes(const smdm_config* cfg);
+
+/* Create a handle.  d_workspace: caller-allocated device memory of >= smdm_workspace_bytes,
+ * 256-byte aligned; it is initialised here (synchronously, on the legacy default stream).
+ * Fails with SMDM_ENOMEM if `bytes` is too small, SMDM_ESHAPE for unsupported shapes. */
+smdm_status smdm_create(const smdm_config* cfg, const smdm_weights* w, void* d_workspace,
+                        size_t bytes, smdm_handle** out);
+void smdm_destroy(smdm_handle* h);
+const char* smdm_last_error(const smdm_handle* h);
+
+/* Prefill (Sec. 3.2: the prompt is prefetched into the KV cache).  Starts sequence slot `seq`:
+ * runs the P prompt rows (block 0, bidirectional among themselves) through every layer and
+ * stores their K/V; no logits.  d_grid: caller-owned int32 [Lgen] that the library fills with
+ * -1 and then updates at every step; it must stay valid while the sequence is in use.
+ * P may be 0. */
+smdm_status smdm_prefill(smdm_handle* h, int seq, const int32_t* d_prompt, int P, int Lgen,
+                         int32_t* d_grid, cudaStream_t stream);
+
+/* One sampling step for one sequence (Figure-3 example; Sec. 3.2; Appendix 7.2).
+ * Rows, in this order: the tokens decoded at the previous step of this sequence (new cache:
+ * their ids from the grid, label k-1), the decode set C (id [MASK], label k), n_reg registers.
+ *  - d_query_pos != NULL: C is this explicit list of n_query 1-based positions (each still
+ *    masked, no duplicates — validated on the device only in checked builds).
+ *  - d_query_pos == NULL: C is every still-masked position in [block_lo, block_hi) in
+ *    position order (semi-autoregressive block decoding); n_query must equal their number.
+ * After the forward: tok = argmax of the row's logits (ties -> lowest id), conf = max softmax
+ * probability.  policy SMDM_POLICY_ALL commits every row of C; SMDM_POLICY_TOPN commits the
+ * n_commit most confident rows (ties -> lowest position).  Committed tokens are written into
+ * the grid and become the next step's new-cache rows (in row order). */
+typedef struct {
+  int seq;                  /* sequence slot */
+  const int32_t* d_query_pos;
+  int n_query;
+  int block_lo, block_hi;
+  int policy;
+  int n_commit;
+} smdm_step_desc;
+
+/* Advance n_seq sequences by one step in ONE batched forward (the weights are streamed once
+ * for all of them).  h_desc: host array [n_seq].  d_logits: optional fp32
+ * [sum of n_query][vocab] (descriptor order), written when non-NULL.  d_tok / d_conf:
+ * optional int32 / fp32 [sum of n_query] argmax and confidence per query row. */
+smdm_status smdm_step(smdm_handle* h, int n_seq, const smdm_step_desc* h_desc, float* d_logits,
+                      int32_t* d_tok, float* d_conf, cudaStream_t stream);
+
+/* The dense comparator (the standard MDM step the pages argue against, papernotes
+ * "Key design 1"): all P+Lgen rows of sequence `seq`, [MASK] ids at undecoded positions, no
+ * registers, no cache, full bidirectional attention, logits for every generated position
+ * (Lgen x V).  The decode set / commit policy are as in smdm_step; the grid is updated the
+ * same way.  d_logits (optional) receives fp32 logits for every generated position,
+ * [Lgen][vocab]; d_tok / d_conf (optional) are per decode-set row as in smdm_step. */
+smdm_status smdm_dense_step(smdm_handle* h, const smdm_step_desc* h_desc, float* d_logits,
+                            int32_t* d_tok, float* d_conf, cudaStream_t stream);
+
+/* A whole sampling plan. */
+typedef struct {
+  int kind;                   /* SMDM_PLAN_ORDER or SMDM_PLAN_SEMIAR */
+  int n_steps;                /* K */
+  const int32_t* h_n_per_step;/* ORDER: host [K], tokens decoded per step (sum = Lgen) */
+  const int32_t* d_order;     /* ORDER: device [Lgen], 1-based positions in decode order */
+  int block;                  /* SEMIAR: block length (Lgen % block == 0) */
+  int steps_per_block;        /* SEMIAR */
+  int commit;                 /* SEMIAR: tokens committed per step (block == steps * commit) */
+} smdm_plan;
+
+/* Full generation of `batch` sequences (slots 0..batch-1) with the same P, Lgen and step
+ * count: prefill, then K steps.  d_prompts: int32 [batch][P]; plans: host [batch];
+ * d_grids: int32 [batch][Lgen] (output).  mode SMDM_MODE_SPARSE batches the sequences into
+ * one forward per step; SMDM_MODE_DENSE runs the dense comparator step per sequence. */
+smdm_status smdm_generate(smdm_handle* h, int batch, const int32_t* d_prompts, int P, int Lgen,
+                          const smdm_plan* plans, int mode, int32_t* d_grids,
+                          cudaStream_t stream);
+
+/* Training (parallel) form (Sec. 3.3, Appendix 7.3): one forward over an arbitrary
+ * step-labelled sequence of n rows under the step-causal mask — clean rows (PROMPT label 0,
+ * CLEAN label = the step they were decoded at) see clean rows with label <= theirs; MASK and
+ * REG rows of label s see clean rows with label < s and the MASK/REG rows of label s.
+ * Writes fp32 logits [n_rows][vocab] for the rows listed in d_logit_rows.  Does not touch any
+ * sequence's generation state. */
+smdm_status smdm_forward_stepcausal(smdm_handle* h, const int32_t* d_ids, const int32_t* d_pos,
+                                    const int32_t* d_type, const int32_t* d_label, int n,
+                                    const int32_t* d_logit_rows, int n_rows, float* d_logits,
+                                    cudaStream_t stream);
+
+/* Test hook: evaluate the device's step-causal predicate for n rows into a bitmap
+ * uint32 [n][(n+31)/32] (bit j of row i = row i may attend to row j). */
+smdm_status smdm_debug_mask(smdm_handle* h, const int32_t* d_type, const int32_t* d_label, int n,
+                            uint32_t* d_bitmap, cudaStream_t stream);
+
+/* Test hook: copy the row arrays of the most recent forward (pack output) into caller
+ * buffers of >= *h_n int32 each (any may be NULL).  *h_n receives the row count. */
+smdm_status smdm_debug_rows(smdm_handle* h, int32_t* d_ids, int32_t* d_pos, int32_t* d_type,
+                            int32_t* d_label, int* h_n, cudaStream_t stream);
+
+/* Cache length (prompt + cached clean tokens) of a sequence slot, host bookkeeping. */
+int smdm_context_length(const smdm_handle* h, int seq);
+
+/* Synchronise `stream` and return the device status word (0 = no device-side error) and clear
+ * it.  Returns SMDM_ETIMEOUT / SMDM_EDEVICE when a bit is set. */
+smdm_status smdm_device_status(smdm_handle* h, unsigned* h_bits, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SMDM_H_ */

@@ -1,0 +1,919 @@
+// C ABI of the sparse sampling library: handle, workspace carving, TMA descriptors and the
+// forward driver that chains the kernels of one step (pack -> [QKV+RoPE+KV append ->
+// step-causal attention -> O-proj+residual -> RMSNorm -> gate/up+SwiGLU -> down+residual ->
+// RMSNorm] x layers -> LM head over the decode set -> unmask).
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "attn.h"
+#include "gemm.h"
+#include "misc.h"
+#include "smdm.h"
+
+using namespace smdm;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows, 128-byte swizzle.
+bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Layout {
+  size_t kc, vc, kscr, vscr, x, h, q, ao, act, hq, pmax, psum, parg, rows, rope, partial,
+      counters, status, newpos, prompts, aux, total;
+  int cap, max_pos, n_vt, rt_max, max_tiles, n_sms;
+  size_t partial_bytes;
+};
+
+bool config_ok(const smdm_config* c, std::string* why) {
+  auto fail = [&](const char* s) {
+    if (why) *why = s;
+    return false;
+  };
+  if (!c) return fail("null config");
+  if (c->n_layers < 1 || c->d_model < 1 || c->n_heads < 1 || c->d_head < 1 || c->d_ffn < 1 ||
+      c->vocab < 1 || c->n_reg < 0)
+    return fail("non-positive model dimension");
+  if (c->n_heads * c->d_head != c->d_model) return fail("n_heads * d_head != d_model");
+  if (c->d_head % 2) return fail("d_head must be even (rotary pairs)");
+  if (c->max_batch < 1 || c->max_batch > SMDM_MAX_BATCH) return fail("max_batch out of range");
+  if (c->max_len < 1 || c->max_step_rows < 1 || c->max_rows < 1) return fail("bad capacity");
+  if (c->dtype == SMDM_BF16) {
+    if (c->d_model % 128) return fail("bf16 models need d_model % 128 == 0");
+    if (c->d_head != 64 && c->d_head != 128) return fail("bf16 models need d_head 64 or 128");
+    if (c->d_ffn % 64) return fail("bf16 models need d_ffn % 64 == 0");
+  } else if (c->dtype == SMDM_F32) {
+    if (c->d_head % 32 || c->d_head > 128) return fail("fp32 models need d_head % 32 == 0, <= 128");
+  } else {
+    return fail("unknown dtype");
+  }
+  return true;
+}
+
+int query_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+Layout make_layout(const smdm_config* c, int n_sms) {
+  Layout L{};
+  const size_t es = c->dtype == SMDM_BF16 ? 2 : 4;
+  const size_t d = c->d_model, H = c->n_heads, dh = c->d_head;
+  L.cap = (int)align_up((size_t)c->max_len + c->max_step_rows, 8);
+  L.max_pos = c->max_len + c->n_reg + 2;
+  L.n_vt = (c->vocab + 127) / 128;
+  L.n_sms = n_sms;
+  const size_t MR = align_up((size_t)c->max_rows, 256);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 1024);
+    return o;
+  };
+  const size_t cache_elems = (size_t)c->max_batch * c->n_layers * H * L.cap * dh;
+  L.kc = take(cache_elems * es);
+  L.vc = take(cache_elems * es);
+  L.kscr = take(H * MR * dh * es);
+  L.vscr = take(H * MR * dh * es);
+  L.x = take(MR * d * 4);
+  L.h = take(MR * d * es);
+  L.q = take(MR * d * es);
+  L.ao = take(MR * d * es);
+  L.act = take(MR * c->d_ffn * es);
+  L.hq = take(MR * d * es);
+  L.pmax = take(MR * L.n_vt * 4);
+  L.psum = take(MR * L.n_vt * 4);
+  L.parg = take(MR * L.n_vt * 4);
+  L.rows = take(9 * MR * 4);
+  L.aux = take(9 * MR * 4);
+  L.rope = take((size_t)L.max_pos * (dh / 2) * 8);
+  L.rt_max = c->max_rows > 256 ? 512 : (int)align_up(c->max_rows, 16);
+  L.partial_bytes = (size_t)n_sms * 2 * L.rt_max * 128 * 4;
+  L.partial = take(L.partial_bytes);
+  int max_nt = 3 * c->d_model / 128 + 1;
+  max_nt = std::max(max_nt, c->d_ffn / 64 + 1);
+  max_nt = std::max(max_nt, (c->vocab + 127) / 128);
+  const int rb = c->max_rows > 512 ? (c->max_rows + 255) / 256 : 1;
+  L.max_tiles = max_nt * rb;
+  L.counters = take((size_t)L.max_tiles * 4);
+  L.status = take(256);
+  L.newpos = take((size_t)c->max_batch * c->max_step_rows * 4);
+  L.prompts = take((size_t)c->max_batch * c->max_len * 4);
+  L.total = off + 1024;
+  return L;
+}
+
+struct SeqState {
+  bool active = false;
+  bool dense = false;
+  int P = 0, Lg = 0;
+  int ctx = 0;     // KV cache length (prompt + cached clean tokens)
+  int n_new = 0;   // tokens committed at the previous step
+  int k = 0;       // steps taken
+  int32_t* grid = nullptr;
+};
+
+}  // namespace
+
+struct smdm_handle {
+  smdm_config cfg;
+  Layout L;
+  bool bf16;
+  const void* emb;
+  const void* final_norm;
+  const void* lm_head;
+  std::vector<const void*> attn_norm, w_qkv, w_o, mlp_norm, w_gate, w_up, w_down;
+  uint8_t* ws;
+  Rows rows, aux;
+  std::vector<CUtensorMap> tm_qkv, tm_o, tm_gate, tm_up, tm_down;
+  CUtensorMap tm_lm, tm_kc, tm_vc, tm_kscr, tm_vscr, tm_q;
+  std::string err;
+  SeqState seq[SMDM_MAX_BATCH];
+  int last_rows = 0;
+
+  template <typename P> P* at(size_t off) { return reinterpret_cast<P*>(ws + off); }
+  uint32_t* status() { return at<uint32_t>(L.status); }
+  int* newpos(int s) { return at<int>(L.newpos) + (size_t)s * cfg.max_step_rows; }
+  int* prompt(int s) { return at<int>(L.prompts) + (size_t)s * cfg.max_len; }
+  size_t es() const { return bf16 ? 2 : 4; }
+};
+
+namespace {
+
+smdm_status fail(smdm_handle* h, smdm_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  if (h) h->err = buf;
+  return st;
+}
+
+#define CK(call)                                                                    \
+  do {                                                                              \
+    cudaError_t e_ = (call);                                                        \
+    if (e_ != cudaSuccess)                                                          \
+      return fail(h, SMDM_ECUDA, "%s failed: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+Rows rows_at(smdm_handle* h, size_t off) {
+  const size_t MR = align_up((size_t)h->cfg.max_rows, 256);
+  int* b = h->at<int>(off);
+  Rows r;
+  r.ids = b;
+  r.pos = b + MR;
+  r.type = b + 2 * MR;
+  r.label = b + 3 * MR;
+  r.seq = b + 4 * MR;
+  r.slot = b + 5 * MR;
+  r.kvlen = b + 6 * MR;
+  r.qrow = b + 7 * MR;
+  r.qpos = b + 8 * MR;
+  return r;
+}
+
+KVAddr cache_addr(smdm_handle* h) {
+  const smdm_config& c = h->cfg;
+  KVAddr kv;
+  kv.k = h->at<uint8_t>(h->L.kc);
+  kv.v = h->at<uint8_t>(h->L.vc);
+  kv.cap = h->L.cap;
+  kv.head_stride = (long long)h->L.cap * c.d_head;
+  kv.layer_stride = kv.head_stride * c.n_heads;
+  kv.seq_stride = kv.layer_stride * c.n_layers;
+  return kv;
+}
+
+KVAddr scratch_addr(smdm_handle* h) {
+  const smdm_config& c = h->cfg;
+  const long long MR = (long long)align_up((size_t)c.max_rows, 256);
+  KVAddr kv;
+  kv.k = h->at<uint8_t>(h->L.kscr);
+  kv.v = h->at<uint8_t>(h->L.vscr);
+  kv.cap = (int)MR;
+  kv.head_stride = MR * c.d_head;
+  kv.layer_stride = 0;
+  kv.seq_stride = 0;
+  return kv;
+}
+
+// What one forward needs beyond the row arrays.
+struct FwdSpec {
+  int R;                      // rows
+  int attn_mode;              // 0 prefix, 1 label
+  bool scratch_kv;            // training form: K/V into the scratch, not a sequence cache
+  int n_seg;
+  AttnSeg seg[SMDM_MAX_BATCH];
+  int n_logit;                // decode-set rows (0 = no LM head)
+  float* logits;              // optional [n_logit][V]
+};
+
+smdm_status gemm(smdm_handle* h, const CUtensorMap* tmA, const CUtensorMap* tmA2, const void* W,
+                 const void* W2, void* X, int K, int n_out, int rows, int swiglu,
+                 const EpiParams& ep, cudaStream_t st) {
+  if (rows <= 0) return SMDM_OK;
+  if (h->bf16) {
+    CUtensorMap tmB;
+    const size_t MR = align_up((size_t)h->cfg.max_rows, 256);
+    if (!encode_2d(&tmB, X, K, MR, (uint64_t)K * 2, 64, gemm_tc_box_rows(rows)))
+      return fail(h, SMDM_ECUDA, "cuTensorMapEncodeTiled failed for an activation operand");
+    GemmCall c{};
+    c.tmA = tmA;
+    c.tmA2 = tmA2;
+    c.tmB = &tmB;
+    c.K = K;
+    c.n_out = n_out;
+    c.rows = rows;
+    c.row0 = 0;
+    c.swiglu = swiglu;
+    c.num_ctas = h->L.n_sms;
+    c.partial = h->at<float>(h->L.partial);
+    c.partial_bytes = h->L.partial_bytes;
+    c.counters = h->at<unsigned>(h->L.counters);
+    c.max_tiles = h->L.max_tiles;
+    c.status = h->status();
+    c.epi = ep;
+    CK(launch_gemm_tc(c, st));
+  } else {
+    CK(launch_gemm_simt(static_cast<const float*>(W), static_cast<const float*>(W2),
+                        static_cast<const float*>(X), K, K, n_out, rows, swiglu, ep, st));
+  }
+  return SMDM_OK;
+}
+
+smdm_status norm(smdm_handle* h, float* x, const void* gain, void* out, const int* gather,
+                 const void* emb, const int* ids, int rows, cudaStream_t st) {
+  NormArgs a;
+  a.x = x;
+  a.gain = gain;
+  a.out = out;
+  a.gather = gather;
+  a.emb = emb;
+  a.ids = ids;
+  a.d = h->cfg.d_model;
+  a.eps = h->cfg.rms_eps;
+  if (h->bf16) CK(launch_rmsnorm<__nv_bfloat16>(a, rows, st));
+  else CK(launch_rmsnorm<float>(a, rows, st));
+  return SMDM_OK;
+}
+
+smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
+  const smdm_config& c = h->cfg;
+  const int d = c.d_model, R = f.R;
+  smdm_status s;
+  float* x = h->at<float>(h->L.x);
+  void* hb = h->at<uint8_t>(h->L.h);
+  void* q = h->at<uint8_t>(h->L.q);
+  void* ao = h->at<uint8_t>(h->L.ao);
+  void* act = h->at<uint8_t>(h->L.act);
+  void* hq = h->at<uint8_t>(h->L.hq);
+  const KVAddr kv = f.scratch_kv ? scratch_addr(h) : cache_addr(h);
+  const Rows& rw = h->rows;
+  h->last_rows = R;
+
+  if ((s = norm(h, x, h->attn_norm[0], hb, nullptr, h->emb, rw.ids, R, st))) return s;
+  for (int l = 0; l < c.n_layers; ++l) {
+    EpiParams ep{};
+    ep.rows = R;
+    // QKV + RoPE + KV append
+    ep.kind = kEpiQKV;
+    ep.n_valid = 3 * d;
+    ep.q_out = q;
+    ep.d_model = d;
+    ep.d_head = c.d_head;
+    ep.layer = f.scratch_kv ? 0 : l;
+    ep.kv = kv;
+    ep.row_seq = rw.seq;
+    ep.row_slot = rw.slot;
+    ep.row_pos = rw.pos;
+    ep.rope = h->at<float2>(h->L.rope);
+    if ((s = gemm(h, h->bf16 ? &h->tm_qkv[l] : nullptr, nullptr, h->w_qkv[l], nullptr, hb, d,
+                  3 * d, R, 0, ep, st)))
+      return s;
+    // step-causal attention
+    if (h->bf16) {
+      AttnCall a{};
+      a.mode = f.attn_mode;
+      a.H = c.n_heads;
+      a.dh = c.d_head;
+      a.d_model = d;
+      a.layer = f.scratch_kv ? 0 : l;
+      a.n_seg = f.n_seg;
+      for (int i = 0; i < f.n_seg; ++i) a.seg[i] = f.seg[i];
+      a.kvlen = rw.kvlen;
+      a.type = rw.type;
+      a.label = rw.label;
+      a.tmQ = &h->tm_q;
+      a.tmK = f.scratch_kv ? &h->tm_kscr : &h->tm_kc;
+      a.tmV = f.scratch_kv ? &h->tm_vscr : &h->tm_vc;
+      a.cache_rows_per_seq = f.scratch_kv ? 0 : (long long)c.n_layers * c.n_heads * h->L.cap;
+      a.cap = kv.cap;
+      a.out = ao;
+      a.status = h->status();
+      CK(launch_attn_tc(a, st));
+    } else {
+      AttnSimtArgs a{};
+      a.mode = f.attn_mode;
+      a.rows = R;
+      a.H = c.n_heads;
+      a.dh = c.d_head;
+      a.d_model = d;
+      a.layer = f.scratch_kv ? 0 : l;
+      a.nkeys = R;
+      a.row_seq = rw.seq;
+      a.kvlen = rw.kvlen;
+      a.type = rw.type;
+      a.label = rw.label;
+      a.scale = 1.0f / sqrtf((float)c.d_head);
+      CK(launch_attn_simt<float>(static_cast<const float*>(q), static_cast<float*>(ao), kv, a, st));
+    }
+    // O-projection + residual
+    EpiParams eo{};
+    eo.kind = kEpiResid;
+    eo.rows = R;
+    eo.n_valid = d;
+    eo.x = x;
+    eo.ld_x = d;
+    if ((s = gemm(h, h->bf16 ? &h->tm_o[l] : nullptr, nullptr, h->w_o[l], nullptr, ao, d, d, R,
+                  0, eo, st)))
+      return s;
+    if ((s = norm(h, x, h->mlp_norm[l], hb, nullptr, nullptr, nullptr, R, st))) return s;
+    // gate/up + SwiGLU
+    EpiParams eg{};
+    eg.kind = kEpiSwiGLU;
+    eg.rows = R;
+    eg.n_valid = c.d_ffn;
+    eg.act = act;
+    eg.ld_act = c.d_ffn;
+    if ((s = gemm(h, h->bf16 ? &h->tm_gate[l] : nullptr, h->bf16 ? &h->tm_up[l] : nullptr,
+                  h->w_gate[l], h->w_up[l], hb, d, c.d_ffn, R, 1, eg, st)))
+      return s;
+    // down + residual
+    EpiParams ed = eo;
+    if ((s = gemm(h, h->bf16 ? &h->tm_down[l] : nullptr, nullptr, h->w_down[l], nullptr, act,
+                  c.d_ffn, d, R, 0, ed, st)))
+      return s;
+    if (l + 1 < c.n_layers)
+      if ((s = norm(h, x, h->attn_norm[l + 1], hb, nullptr, nullptr, nullptr, R, st))) return s;
+  }
+  if (f.n_logit > 0) {
+    if ((s = norm(h, x, h->final_norm, hq, rw.qrow, nullptr, nullptr, f.n_logit, st))) return s;
+    EpiParams el{};
+    el.kind = kEpiLMHead;
+    el.rows = f.n_logit;
+    el.n_valid = c.vocab;
+    el.logits = f.logits;
+    el.ld_logits = c.vocab;
+    el.pmax = h->at<float>(h->L.pmax);
+    el.psum = h->at<float>(h->L.psum);
+    el.parg = h->at<int>(h->L.parg);
+    el.n_vt = h->L.n_vt;
+    if ((s = gemm(h, h->bf16 ? &h->tm_lm : nullptr, nullptr, h->lm_head, nullptr, hq, d, c.vocab,
+                  f.n_logit, 0, el, st)))
+      return s;
+  }
+  return SMDM_OK;
+}
+
+smdm_status check_seq(smdm_handle* h, int seq) {
+  if (seq < 0 || seq >= h->cfg.max_batch)
+    return fail(h, SMDM_EINVAL, "sequence slot %d out of range [0, %d)", seq, h->cfg.max_batch);
+  return SMDM_OK;
+}
+
+// Validate a step descriptor against the sequence state; returns n_query and R.
+smdm_status check_desc(smdm_handle* h, const smdm_step_desc& d, bool dense) {
+  smdm_status s;
+  if ((s = check_seq(h, d.seq))) return s;
+  const SeqState& q = h->seq[d.seq];
+  if (!q.active) return fail(h, SMDM_ESTATE, "sequence %d has not been prefilled", d.seq);
+  if (q.dense != dense)
+    return fail(h, SMDM_ESTATE, "sequence %d mixes sparse and dense steps", d.seq);
+  if (d.n_query < 1) return fail(h, SMDM_EINVAL, "empty decode set");
+  if (d.policy != SMDM_POLICY_ALL && d.policy != SMDM_POLICY_TOPN)
+    return fail(h, SMDM_EINVAL, "unknown policy %d", d.policy);
+  if (d.policy == SMDM_POLICY_TOPN && d.n_commit < 1)
+    return fail(h, SMDM_EINVAL, "TOPN needs n_commit >= 1");
+  if (!d.d_query_pos) {
+    const int lo = q.P + 1, hi = q.P + q.Lg + 1;
+    if (d.block_lo < lo || d.block_hi > hi || d.block_lo >= d.block_hi)
+      return fail(h, SMDM_EINVAL, "block [%d, %d) outside the generated span [%d, %d)",
+                  d.block_lo, d.block_hi, lo, hi);
+    if (d.n_query > d.block_hi - d.block_lo)
+      return fail(h, SMDM_EINVAL, "n_query larger than the block");
+  }
+  if (d.n_query > q.Lg) return fail(h, SMDM_EINVAL, "n_query larger than Lgen");
+  if (!dense) {
+    const int R = q.n_new + d.n_query + h->cfg.n_reg;
+    if (R > h->cfg.max_step_rows)
+      return fail(h, SMDM_ESHAPE, "step rows %d exceed max_step_rows %d", R, h->cfg.max_step_rows);
+    if (q.ctx + R > h->L.cap) return fail(h, SMDM_ESHAPE, "KV cache capacity exceeded");
+  }
+  return SMDM_OK;
+}
+
+int committed(const smdm_step_desc& d) {
+  return d.policy == SMDM_POLICY_ALL ? d.n_query : std::min(d.n_commit, d.n_query);
+}
+
+}  // namespace
+
+// ==============================================================================================
+// C ABI
+// ==============================================================================================
+extern "C" {
+
+size_t smdm_workspace_bytes(const smdm_config* cfg) {
+  if (!config_ok(cfg, nullptr)) return 0;
+  return make_layout(cfg, query_sms()).total;
+}
+
+smdm_status smdm_create(const smdm_config* cfg, const smdm_weights* w, void* d_workspace,
+                        size_t bytes, smdm_handle** out) {
+  if (!out) return SMDM_EINVAL;
+  *out = nullptr;
+  std::string why;
+  if (!config_ok(cfg, &why)) return SMDM_ESHAPE;
+  if (!w || !d_workspace || !w->emb || !w->final_norm || !w->lm_head || !w->attn_norm ||
+      !w->w_qkv || !w->w_o || !w->mlp_norm || !w->w_gate || !w->w_up || !w->w_down)
+    return SMDM_EINVAL;
+  if (reinterpret_cast<uintptr_t>(d_workspace) % 256) return SMDM_EINVAL;
+  smdm_handle* h = new smdm_handle();
+  h->cfg = *cfg;
+  h->bf16 = cfg->dtype == SMDM_BF16;
+  h->L = make_layout(cfg, query_sms());
+  if (bytes < h->L.total) {
+    delete h;
+    return SMDM_ENOMEM;
+  }
+  h->ws = static_cast<uint8_t*>(d_workspace);
+  h->emb = w->emb;
+  h->final_norm = w->final_norm;
+  h->lm_head = w->lm_head;
+  const int nl = cfg->n_layers;
+  for (int l = 0; l < nl; ++l) {
+    if (!w->attn_norm[l] || !w->w_qkv[l] || !w->w_o[l] || !w->mlp_norm[l] || !w->w_gate[l] ||
+        !w->w_up[l] || !w->w_down[l]) {
+      delete h;
+      return SMDM_EINVAL;
+    }
+    h->attn_norm.push_back(w->attn_norm[l]);
+    h->w_qkv.push_back(w->w_qkv[l]);
+    h->w_o.push_back(w->w_o[l]);
+    h->mlp_norm.push_back(w->mlp_norm[l]);
+    h->w_gate.push_back(w->w_gate[l]);
+    h->w_up.push_back(w->w_up[l]);
+    h->w_down.push_back(w->w_down[l]);
+  }
+  h->rows = rows_at(h, h->L.rows);
+  h->aux = rows_at(h, h->L.aux);
+  auto cuda_fail = [&](cudaError_t e) {
+    delete h;
+    (void)e;
+    return SMDM_ECUDA;
+  };
+  cudaError_t e = cudaMemset(d_workspace, 0, h->L.total);
+  if (e != cudaSuccess) return cuda_fail(e);
+  // RoPE table: angle = pos * theta^(-2i/d_head), computed in double, stored (cos, sin) fp32.
+  {
+    const int half = cfg->d_head / 2;
+    std::vector<float2> tab((size_t)h->L.max_pos * half);
+    for (int p = 0; p < h->L.max_pos; ++p)
+      for (int i = 0; i < half; ++i) {
+        const double inv = std::pow((double)cfg->rope_theta, -2.0 * i / cfg->d_head);
+        const double ang = (double)p * inv;
+        tab[(size_t)p * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+      }
+    e = cudaMemcpy(h->at<float2>(h->L.rope), tab.data(), tab.size() * sizeof(float2),
+                   cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  if (h->bf16) {
+    const int d = cfg->d_model, f = cfg->d_ffn, H = cfg->n_heads, dh = cfg->d_head;
+    bool ok = true;
+    h->tm_qkv.resize(nl);
+    h->tm_o.resize(nl);
+    h->tm_gate.resize(nl);
+    h->tm_up.resize(nl);
+    h->tm_down.resize(nl);
+    for (int l = 0; l < nl; ++l) {
+      ok &= encode_2d(&h->tm_qkv[l], w->w_qkv[l], d, 3 * d, (uint64_t)d * 2, 64, 128);
+      ok &= encode_2d(&h->tm_o[l], w->w_o[l], d, d, (uint64_t)d * 2, 64, 128);
+      ok &= encode_2d(&h->tm_gate[l], w->w_gate[l], d, f, (uint64_t)d * 2, 64, 64);
+      ok &= encode_2d(&h->tm_up[l], w->w_up[l], d, f, (uint64_t)d * 2, 64, 64);
+      ok &= encode_2d(&h->tm_down[l], w->w_down[l], f, d, (uint64_t)f * 2, 64, 128);
+    }
+    ok &= encode_2d(&h->tm_lm, w->lm_head, d, cfg->vocab, (uint64_t)d * 2, 64, 128);
+    const size_t MR = align_up((size_t)cfg->max_rows, 256);
+    const uint64_t cache_rows = (uint64_t)cfg->max_batch * nl * H * h->L.cap;
+    ok &= encode_2d(&h->tm_kc, h->at<uint8_t>(h->L.kc), dh, cache_rows, (uint64_t)dh * 2, 64, 128);
+    ok &= encode_2d(&h->tm_vc, h->at<uint8_t>(h->L.vc), dh, cache_rows, (uint64_t)dh * 2, 64, 128);
+    ok &= encode_2d(&h->tm_kscr, h->at<uint8_t>(h->L.kscr), dh, (uint64_t)H * MR, (uint64_t)dh * 2,
+                    64, 128);
+    ok &= encode_2d(&h->tm_vscr, h->at<uint8_t>(h->L.vscr), dh, (uint64_t)H * MR, (uint64_t)dh * 2,
+                    64, 128);
+    ok &= encode_2d(&h->tm_q, h->at<uint8_t>(h->L.q), d, MR, (uint64_t)d * 2, 64, 128);
+    if (!ok) {
+      delete h;
+      return SMDM_ECUDA;
+    }
+    if (gemm_tc_set_smem_attr() != cudaSuccess || attn_tc_set_smem_attr() != cudaSuccess) {
+      delete h;
+      return SMDM_ECUDA;
+    }
+  }
+  e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e);
+  *out = h;
+  return SMDM_OK;
+}
+
+void smdm_destroy(smdm_handle* h) { delete h; }
+
+const char* smdm_last_error(const smdm_handle* h) { return h ? h->err.c_str() : "null handle"; }
+
+int smdm_context_length(const smdm_handle* h, int seq) {
+  if (!h || seq < 0 || seq >= h->cfg.max_batch) return -1;
+  return h->seq[seq].ctx;
+}
+
+smdm_status smdm_prefill(smdm_handle* h, int seq, const int32_t* d_prompt, int P, int Lgen,
+                         int32_t* d_grid, cudaStream_t st) {
+  if (!h) return SMDM_EINVAL;
+  smdm_status s;
+  if ((s = check_seq(h, seq))) return s;
+  if (P < 0 || Lgen < 1 || P + Lgen > h->cfg.max_len)
+    return fail(h, SMDM_ESHAPE, "P=%d, Lgen=%d outside max_len %d", P, Lgen, h->cfg.max_len);
+  if (P > h->cfg.max_rows) return fail(h, SMDM_ESHAPE, "prompt longer than max_rows");
+  if (!d_grid || (P > 0 && !d_prompt)) return fail(h, SMDM_EINVAL, "null prompt or grid");
+  CK(launch_fill_i32(d_grid, Lgen, -1, st));
+  if (P > 0)
+    CK(cudaMemcpyAsync(h->prompt(seq), d_prompt, (size_t)P * 4, cudaMemcpyDeviceToDevice, st));
+  SeqState& q = h->seq[seq];
+  q = SeqState();
+  q.P = P;
+  q.Lg = Lgen;
+  q.grid = d_grid;
+  if (P > 0) {
+    LinearPackArgs a{};
+    a.mode = kPackPrefill;
+    a.n = P;
+    a.seq = seq;
+    a.P = P;
+    a.vocab = h->cfg.vocab;
+    a.emb_rows = h->cfg.vocab + 2 + h->cfg.n_reg;
+    a.max_pos = h->L.max_pos;
+    a.prompt = h->prompt(seq);
+    a.rows = h->rows;
+    a.status = h->status();
+    CK(launch_pack_linear(a, st));
+    FwdSpec f{};
+    f.R = P;
+    f.attn_mode = 0;
+    f.n_seg = 1;
+    f.seg[0] = AttnSeg{seq, 0, P, P, 0};
+    if ((s = forward(h, f, st))) return s;
+  }
+  q.active = true;
+  q.ctx = P;
+  return SMDM_OK;
+}
+
+smdm_status smdm_step(smdm_handle* h, int n_seq, const smdm_step_desc* hd, float* d_logits,
+                      int32_t* d_tok, float* d_conf, cudaStream_t st) {
+  if (!h) return SMDM_EINVAL;
+  if (n_seq < 1 || n_seq > h->cfg.max_batch || !hd) return fail(h, SMDM_EINVAL, "bad batch");
+  smdm_status s;
+  int R = 0, NQ = 0;
+  for (int i = 0; i < n_seq; ++i) {
+    if ((s = check_desc(h, hd[i], false))) return s;
+    for (int j = 0; j < i; ++j)
+      if (hd[j].seq == hd[i].seq) return fail(h, SMDM_EINVAL, "sequence %d twice in a batch", hd[i].seq);
+    R += h->seq[hd[i].seq].n_new + hd[i].n_query + h->cfg.n_reg;
+    NQ += hd[i].n_query;
+  }
+  if (R > h->cfg.max_rows) return fail(h, SMDM_ESHAPE, "batched rows %d exceed max_rows", R);
+  PackArgs pa{};
+  pa.n_seq = n_seq;
+  pa.vocab = h->cfg.vocab;
+  pa.rows = h->rows;
+  pa.status = h->status();
+  FwdSpec f{};
+  f.R = R;
+  f.attn_mode = 0;
+  f.n_seg = n_seq;
+  f.n_logit = NQ;
+  f.logits = d_logits;
+  UnmaskArgs ua{};
+  ua.n_seq = n_seq;
+  int row0 = 0, qbase = 0, max_nq = 0;
+  for (int i = 0; i < n_seq; ++i) {
+    const smdm_step_desc& d = hd[i];
+    SeqState& q = h->seq[d.seq];
+    const int Rs = q.n_new + d.n_query + h->cfg.n_reg;
+    PackSeq& p = pa.s[i];
+    p.seq = d.seq;
+    p.row0 = row0;
+    p.n_new = q.n_new;
+    p.n_q = d.n_query;
+    p.n_reg = h->cfg.n_reg;
+    p.ctx = q.ctx;
+    p.P = q.P;
+    p.Lg = q.Lg;
+    p.label = q.k + 1;
+    p.qbase = qbase;
+    p.block_lo = d.block_lo;
+    p.block_hi = d.block_hi;
+    p.qpos = d.d_query_pos;
+    p.grid = q.grid;
+    p.newpos = h->newpos(d.seq);
+    f.seg[i] = AttnSeg{d.seq, row0, Rs, q.ctx + Rs, 0};
+    UnmaskSeq& u = ua.s[i];
+    u.qbase = qbase;
+    u.n_q = d.n_query;
+    u.lbase = 0;
+    u.dense = 0;
+    u.policy = d.policy;
+    u.n_commit = d.policy == SMDM_POLICY_ALL ? d.n_query : d.n_commit;
+    u.P = q.P;
+    u.Lg = q.Lg;
+    u.grid = q.grid;
+    u.newpos = h->newpos(d.seq);
+    row0 += Rs;
+    qbase += d.n_query;
+    max_nq = std::max(max_nq, d.n_query);
+  }
+  CK(launch_pack_step(pa, st));
+  if ((s = forward(h, f, st))) return s;
+  ua.n_vt = h->L.n_vt;
+  ua.pmax = h->at<float>(h->L.pmax);
+  ua.psum = h->at<float>(h->L.psum);
+  ua.parg = h->at<int>(h->L.parg);
+  ua.qpos_of = h->rows.qpos;
+  ua.tok_out = d_tok;
+  ua.conf_out = d_conf;
+  ua.status = h->status();
+  CK(launch_unmask(ua, max_nq, st));
+  for (int i = 0; i < n_seq; ++i) {
+    SeqState& q = h->seq[hd[i].seq];
+    q.ctx += q.n_new;
+    q.n_new = committed(hd[i]);
+    q.k += 1;
+  }
+  return SMDM_OK;
+}
+
+smdm_status smdm_dense_step(smdm_handle* h, const smdm_step_desc* d, float* d_logits,
+                            int32_t* d_tok, float* d_conf, cudaStream_t st) {
+  if (!h || !d) return SMDM_EINVAL;
+  smdm_status s;
+  if ((s = check_seq(h, d->seq))) return s;
+  SeqState& q = h->seq[d->seq];
+  if (q.active && q.k == 0) q.dense = true;   // a freshly prefilled sequence may go dense
+  if ((s = check_desc(h, *d, true))) return s;
+  const int L = q.P + q.Lg;
+  if (L > h->cfg.max_rows) return fail(h, SMDM_ESHAPE, "P + Lgen exceeds max_rows");
+  // decode set -> aux.qpos
+  PackArgs pa{};
+  pa.n_seq = 1;
+  pa.vocab = h->cfg.vocab;
+  pa.rows = h->aux;
+  pa.status = h->status();
+  PackSeq& p = pa.s[0];
+  p.seq = d->seq;
+  p.row0 = 0;
+  p.n_new = 0;
+  p.n_q = d->n_query;
+  p.n_reg = 0;
+  p.ctx = 0;
+  p.P = q.P;
+  p.Lg = q.Lg;
+  p.label = q.k + 1;
+  p.qbase = 0;
+  p.block_lo = d->block_lo;
+  p.block_hi = d->block_hi;
+  p.qpos = d->d_query_pos;
+  p.grid = q.grid;
+  p.newpos = h->newpos(d->seq);
+  CK(launch_pack_step(pa, st));
+  LinearPackArgs a{};
+  a.mode = kPackDense;
+  a.n = L;
+  a.seq = d->seq;
+  a.P = q.P;
+  a.vocab = h->cfg.vocab;
+  a.emb_rows = h->cfg.vocab + 2 + h->cfg.n_reg;
+  a.max_pos = h->L.max_pos;
+  a.prompt = h->prompt(d->seq);
+  a.grid = q.grid;
+  a.rows = h->rows;
+  a.status = h->status();
+  CK(launch_pack_linear(a, st));
+  FwdSpec f{};
+  f.R = L;
+  f.attn_mode = 0;
+  f.n_seg = 1;
+  f.seg[0] = AttnSeg{d->seq, 0, L, L, 0};
+  f.n_logit = q.Lg;
+  f.logits = d_logits;
+  if ((s = forward(h, f, st))) return s;
+  UnmaskArgs ua{};
+  ua.n_seq = 1;
+  UnmaskSeq& u = ua.s[0];
+  u.qbase = 0;
+  u.n_q = d->n_query;
+  u.lbase = 0;
+  u.dense = 1;
+  u.policy = d->policy;
+  u.n_commit = d->policy == SMDM_POLICY_ALL ? d->n_query : d->n_commit;
+  u.P = q.P;
+  u.Lg = q.Lg;
+  u.grid = q.grid;
+  u.newpos = nullptr;
+  ua.n_vt = h->L.n_vt;
+  ua.pmax = h->at<float>(h->L.pmax);
+  ua.psum = h->at<float>(h->L.psum);
+  ua.parg = h->at<int>(h->L.parg);
+  ua.qpos_of = h->aux.qpos;
+  ua.tok_out = d_tok;
+  ua.conf_out = d_conf;
+  ua.status = h->status();
+  CK(launch_unmask(ua, d->n_query, st));
+  q.k += 1;
+  return SMDM_OK;
+}
+
+smdm_status smdm_generate(smdm_handle* h, int batch, const int32_t* d_prompts, int P, int Lgen,
+                          const smdm_plan* plans, int mode, int32_t* d_grids, cudaStream_t st) {
+  if (!h) return SMDM_EINVAL;
+  if (batch < 1 || batch > h->cfg.max_batch || !plans || !d_grids || (P > 0 && !d_prompts))
+    return fail(h, SMDM_EINVAL, "bad generate arguments");
+  if (mode != SMDM_MODE_SPARSE && mode != SMDM_MODE_DENSE)
+    return fail(h, SMDM_EINVAL, "unknown mode %d", mode);
+  const int K = plans[0].n_steps;
+  for (int b = 0; b < batch; ++b) {
+    const smdm_plan& p = plans[b];
+    if (p.n_steps != K || K < 1) return fail(h, SMDM_EINVAL, "plans need the same step count");
+    if (p.kind == SMDM_PLAN_ORDER) {
+      if (!p.h_n_per_step || !p.d_order) return fail(h, SMDM_EINVAL, "ORDER plan needs order + sizes");
+      long long tot = 0;
+      for (int k = 0; k < K; ++k) {
+        if (p.h_n_per_step[k] < 1) return fail(h, SMDM_EINVAL, "empty step in plan");
+        tot += p.h_n_per_step[k];
+      }
+      if (tot != Lgen) return fail(h, SMDM_EINVAL, "plan sizes sum to %lld, not Lgen %d", tot, Lgen);
+    } else if (p.kind == SMDM_PLAN_SEMIAR) {
+      if (p.block < 1 || p.commit < 1 || p.steps_per_block < 1 || Lgen % p.block ||
+          p.block != p.steps_per_block * p.commit || K != (Lgen / p.block) * p.steps_per_block)
+        return fail(h, SMDM_EINVAL, "inconsistent SEMIAR plan");
+    } else {
+      return fail(h, SMDM_EINVAL, "unknown plan kind");
+    }
+  }
+  smdm_status s;
+  for (int b = 0; b < batch; ++b)
+    if ((s = smdm_prefill(h, b, d_prompts + (size_t)b * P, P, Lgen, d_grids + (size_t)b * Lgen, st)))
+      return s;
+  std::vector<long long> off(batch, 0);
+  for (int k = 1; k <= K; ++k) {
+    smdm_step_desc desc[SMDM_MAX_BATCH];
+    for (int b = 0; b < batch; ++b) {
+      const smdm_plan& p = plans[b];
+      smdm_step_desc& d = desc[b];
+      d = smdm_step_desc{};
+      d.seq = b;
+      if (p.kind == SMDM_PLAN_ORDER) {
+        d.d_query_pos = p.d_order + off[b];
+        d.n_query = p.h_n_per_step[k - 1];
+        d.policy = SMDM_POLICY_ALL;
+        d.n_commit = d.n_query;
+        off[b] += d.n_query;
+      } else {
+        const int blk = (k - 1) / p.steps_per_block, j = (k - 1) % p.steps_per_block;
+        d.d_query_pos = nullptr;
+        d.block_lo = P + 1 + blk * p.block;
+        d.block_hi = d.block_lo + p.block;
+        d.n_query = p.block - j * p.commit;
+        d.policy = SMDM_POLICY_TOPN;
+        d.n_commit = p.commit;
+      }
+    }
+    if (mode == SMDM_MODE_SPARSE) {
+      if ((s = smdm_step(h, batch, desc, nullptr, nullptr, nullptr, st))) return s;
+    } else {
+      for (int b = 0; b < batch; ++b)
+        if ((s = smdm_dense_step(h, &desc[b], nullptr, nullptr, nullptr, st))) return s;
+    }
+  }
+  return SMDM_OK;
+}
+
+smdm_status smdm_forward_stepcausal(smdm_handle* h, const int32_t* d_ids, const int32_t* d_pos,
+                                    const int32_t* d_type, const int32_t* d_label, int n,
+                                    const int32_t* d_logit_rows, int n_rows, float* d_logits,
+                                    cudaStream_t st) {
+  if (!h) return SMDM_EINVAL;
+  if (!d_ids || !d_pos || !d_type || !d_label || !d_logit_rows || !d_logits)
+    return fail(h, SMDM_EINVAL, "null argument");
+  if (n < 1 || n > h->cfg.max_rows || n_rows < 1 || n_rows > h->cfg.max_rows)
+    return fail(h, SMDM_ESHAPE, "n=%d / n_rows=%d outside [1, max_rows]", n, n_rows);
+  LinearPackArgs a{};
+  a.mode = kPackTrain;
+  a.n = n;
+  a.seq = 0;
+  a.vocab = h->cfg.vocab;
+  a.emb_rows = h->cfg.vocab + 2 + h->cfg.n_reg;
+  a.max_pos = h->L.max_pos;
+  a.ids = d_ids;
+  a.pos = d_pos;
+  a.type = d_type;
+  a.label = d_label;
+  a.rows = h->rows;
+  a.status = h->status();
+  CK(launch_pack_linear(a, st));
+  CK(launch_gather_rows(d_logit_rows, n_rows, h->rows.qrow, st));
+  FwdSpec f{};
+  f.R = n;
+  f.attn_mode = 1;
+  f.scratch_kv = true;
+  f.n_seg = 1;
+  f.seg[0] = AttnSeg{0, 0, n, n, 0};
+  f.n_logit = n_rows;
+  f.logits = d_logits;
+  return forward(h, f, st);
+}
+
+smdm_status smdm_debug_mask(smdm_handle* h, const int32_t* d_type, const int32_t* d_label, int n,
+                            uint32_t* d_bitmap, cudaStream_t st) {
+  if (!h) return SMDM_EINVAL;
+  if (!d_type || !d_label || !d_bitmap || n < 1) return fail(h, SMDM_EINVAL, "bad arguments");
+  CK(launch_debug_mask(d_type, d_label, n, d_bitmap, st));
+  return SMDM_OK;
+}
+
+smdm_status smdm_debug_rows(smdm_handle* h, int32_t* d_ids, int32_t* d_pos, int32_t* d_type,
+                            int32_t* d_label, int* h_n, cudaStream_t st) {
+  if (!h || !h_n) return SMDM_EINVAL;
+  const int n = h->last_rows;
+  *h_n = n;
+  const size_t b = (size_t)n * 4;
+  if (n > 0) {
+    if (d_ids) CK(cudaMemcpyAsync(d_ids, h->rows.ids, b, cudaMemcpyDeviceToDevice, st));
+    if (d_pos) CK(cudaMemcpyAsync(d_pos, h->rows.pos, b, cudaMemcpyDeviceToDevice, st));
+    if (d_type) CK(cudaMemcpyAsync(d_type, h->rows.type, b, cudaMemcpyDeviceToDevice, st));
+    if (d_label) CK(cudaMemcpyAsync(d_label, h->rows.label, b, cudaMemcpyDeviceToDevice, st));
+  }
+  return SMDM_OK;
+}
+
+smdm_status smdm_device_status(smdm_handle* h, unsigned* h_bits, cudaStream_t st) {
+  if (!h) return SMDM_EINVAL;
+  uint32_t bits = 0;
+  CK(cudaMemcpyAsync(&bits, h->status(), 4, cudaMemcpyDeviceToHost, st));
+  CK(cudaStreamSynchronize(st));
+  CK(cudaMemsetAsync(h->status(), 0, 4, st));
+  CK(cudaStreamSynchronize(st));
+  if (h_bits) *h_bits = bits;
+  if (bits & kStatusTimeout) return fail(h, SMDM_ETIMEOUT, "a device-side wait timed out");
+  if (bits & kStatusBounds) return fail(h, SMDM_EDEVICE, "a device-side bounds check failed");
+  return SMDM_OK;
+}
+
+}  // extern "C"

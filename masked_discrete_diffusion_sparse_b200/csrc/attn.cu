@@ -1,0 +1,400 @@
+// Step-causal attention of the sparse sampling step (Sparse-LaViDa Figure-3 example and
+// Sec. 3.3).  Two ways of stating which keys a query row sees:
+//   prefix mode — the row sees keys [0, kvlen[row]) of its sequence's KV cache.  At a sampling
+//     step the cache holds [prompt + clean tokens | new-cache rows | masks | registers], so the
+//     step-causal rule is exactly a per-row prefix: new-cache rows stop after the new-cache
+//     rows, mask and register rows see everything.  Prefill and the dense comparator use a
+//     common prefix for all rows.
+//   label mode — the training-form rule evaluated per (query, key) from row types and step
+//     labels; keys are the rows of the same forward.
+//
+// bf16 path: one CTA per (sequence, 128-row query tile, head).  Warp 0 streams Q and K/V tiles
+// with TMA, warp 1 issues tcgen05.mma (S = Q K^T into one of two TMEM buffers, O += P V into a
+// TMEM accumulator), warps 2-5 own one query row per thread: masking, online softmax in the
+// exp2 domain, P (bf16) into swizzled shared memory, final 1/l scaling.  The running maximum is
+// only moved (and O rescaled) when it grows by more than 2^8, so most tiles skip the rescale;
+// the result is exact because numerator and denominator share the reference maximum.
+// fp32 path: one warp per (row, head), SIMT.
+#include "attn.h"
+
+namespace smdm {
+
+constexpr int kAttnThreads = 192;
+
+struct AttnDev {
+  int mode;        // 0 prefix, 1 label
+  int H, dh, d_model, layer;
+  int n_seg;
+  AttnSeg seg[kMaxBatch];         // seg[s].tile0 = first grid block of segment s
+  const int* kvlen;
+  const int* type;
+  const int* label;
+  long long cache_rows_per_seq;   // rows of the 2-D cache map per sequence (n_layers*H*cap)
+  int cap;
+  float scale_log2;               // log2(e) / sqrt(dh)
+  int nstages;
+  int q_off, k_off, v_off, p_off, bar_off, stage_bytes;
+  void* out;                      // [rows][d_model] bf16
+  uint32_t* status;
+};
+
+SMDM_DEV void p_store_swizzled(uint8_t* P, int row, int key8, uint4 val) {
+  // P: [2 sub-tiles][128 rows][64 keys] bf16, 128-byte swizzle; key8 = 16-byte chunk 0..15
+  const int sub = key8 >> 3, cc = key8 & 7;
+  uint8_t* dst = P + sub * 16384 + row * 128 + ((cc ^ (row & 7)) << 4);
+  *reinterpret_cast<uint4*>(dst) = val;
+}
+
+SMDM_DEV uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const AttnDev a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* Qs = smem + a.q_off;
+  uint8_t* Ps = smem + a.p_off;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.bar_off);
+  const int NS = a.nstages;
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* v_full = k_full + NS;
+  uint64_t* kv_empty = v_full + NS;
+  uint64_t* s_full = kv_empty + NS;   // [2]
+  uint64_t* s_free = s_full + 2;      // [2]
+  uint64_t* p_full = s_free + 2;
+  uint64_t* pv_done = p_full + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pv_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int blk = blockIdx.x, h = blockIdx.y;
+  int si = 0;
+  while (si + 1 < a.n_seg && a.seg[si + 1].tile0 <= blk) ++si;
+  const AttnSeg sg = a.seg[si];
+  const int tile = blk - sg.tile0;
+  const int qrow0 = sg.row0 + tile * 128;            // first forward row of this tile
+  const int nq = min(128, sg.rows - tile * 128);     // valid query rows
+  const int nkeys = sg.nkeys;
+  const int nkv = (nkeys + 127) / 128;
+  const int dh = a.dh;
+  const int nsub = dh / 64;                          // 64-wide chunks of the head dim
+  const long long cache_base = (long long)sg.seq * a.cache_rows_per_seq +
+                               ((long long)a.layer * a.H + h) * a.cap;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], 4);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+  const uint32_t t_o = tbase + 256;   // O accumulator columns [256, 256 + dh)
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_q = policy_evict_normal();
+      const uint64_t pol_kv = policy_evict_last();
+      mbar_arrive_expect_tx(q_full, 128 * dh * 2);
+      for (int c = 0; c < nsub; ++c) tma_load_2d(Qs + c * 16384, &tmQ, q_full, h * dh + c * 64, qrow0, pol_q);
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int j = 0; j < nkv; ++j) {
+        if (!mbar_wait(&kv_empty[stage], phase ^ 1, abort_flag, a.status)) break;
+        uint8_t* Ks = smem + a.k_off + stage * a.stage_bytes;
+        uint8_t* Vs = smem + a.v_off + stage * a.stage_bytes;
+        const int y = (int)(cache_base + (long long)j * 128);
+        mbar_arrive_expect_tx(&k_full[stage], 128 * dh * 2);
+        for (int c = 0; c < nsub; ++c) tma_load_2d(Ks + c * 16384, &tmK, &k_full[stage], c * 64, y, pol_kv);
+        mbar_arrive_expect_tx(&v_full[stage], 128 * dh * 2);
+        for (int c = 0; c < nsub; ++c) tma_load_2d(Vs + c * 16384, &tmV, &v_full[stage], c * 64, y, pol_kv);
+        if (++stage == NS) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16(128, 128, 0, 0);
+      const uint32_t idesc_o = idesc_bf16(128, dh, 0, 1);   // V is MN-major (dh contiguous)
+      const uint32_t q_addr = smem_u32(Qs), p_addr = smem_u32(Ps);
+      bool ok = mbar_wait(q_full, 0, abort_flag, a.status);
+      int stage = 0;
+      uint32_t phase = 0;
+      int pstage = 0;
+      uint32_t pphase = 0;
+      for (int j = 0; ok && j <= nkv; ++j) {
+        if (j < nkv) {
+          const int b = j & 1;
+          if (!mbar_wait(&k_full[stage], phase, abort_flag, a.status)) break;
+          if (!mbar_wait(&s_free[b], ((j >> 1) & 1) ^ 1, abort_flag, a.status)) break;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(smem + a.k_off + stage * a.stage_bytes);
+          for (int kk = 0; kk < dh / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            umma_f16(tbase + b * 128, sdesc_sw128(q_addr + off, 16, 1024),
+                     sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[b]);
+          if (++stage == NS) { stage = 0; phase ^= 1; }
+        }
+        if (j >= 1) {
+          // O += P_{j-1} V_{j-1}
+          const int jj = j - 1;
+          if (!mbar_wait(p_full, jj & 1, abort_flag, a.status)) break;
+          if (!mbar_wait(&v_full[pstage], pphase, abort_flag, a.status)) break;
+          tc_fence_after();
+          const uint32_t v_addr = smem_u32(smem + a.v_off + pstage * a.stage_bytes);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+            umma_f16(t_o, sdesc_sw128(p_addr + aoff, 16, 1024),
+                     sdesc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
+                     (jj > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&kv_empty[pstage]);
+          umma_commit(pv_done);
+          if (++pstage == NS) { pstage = 0; pphase ^= 1; }
+        }
+      }
+    }
+  } else {
+    // Softmax warps: thread owns query row em of the tile.
+    const int q4 = warp & 3;
+    const int em = q4 * 32 + lane;
+    const int row = qrow0 + em;
+    const bool valid = em < nq;
+    const uint32_t lane_off = uint32_t(q4 * 32) << 16;
+    int kv_lim = 0, tq = 0, lq = 0;
+    if (valid) {
+      if (a.mode == 0) kv_lim = a.kvlen[row];
+      else { tq = a.type[row]; lq = a.label[row]; kv_lim = nkeys; }
+    }
+    float m_ref = -INFINITY, l = 0.f;
+    for (int j = 0; j < nkv; ++j) {
+      const int b = j & 1;
+      if (!mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag, a.status)) break;
+      tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) tmem_ld16(tbase + lane_off + b * 128 + c * 16, s + c * 16);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[b]);
+      const int key0 = j * 128;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        const int key = key0 + c;
+        bool ok = valid && key < kv_lim;
+        if (ok && a.mode == 1) ok = step_causal_allowed(tq, lq, a.type[key], a.label[key]);
+        s[c] = ok ? s[c] * a.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, s[c]);
+      }
+      float alpha = 1.f;
+      if (mx > m_ref + 8.f) {          // move the reference maximum (also the first time)
+        alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
+        m_ref = mx;
+      }
+      float rs = 0.f;
+      // O and P are still in use by the previous P V product.
+      if (j >= 1 && !mbar_wait(pv_done, (j - 1) & 1, abort_flag, a.status)) break;
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, alpha != 1.f) && j >= 1) {
+        for (int c = 0; c < dh / 16; ++c) {
+          float o[16];
+          tmem_ld16(t_o + lane_off + c * 16, o);
+#pragma unroll
+          for (int t = 0; t < 16; ++t) o[t] *= alpha;
+          tmem_st16(t_o + lane_off + c * 16, o);
+        }
+      }
+#pragma unroll
+      for (int c8 = 0; c8 < 16; ++c8) {
+        float p[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const float sv = s[c8 * 8 + t];
+          p[t] = (sv == -INFINITY) ? 0.f : exp2f(sv - m_ref);
+          rs += p[t];
+        }
+        uint4 pk;
+        pk.x = pack_bf16x2(p[0], p[1]);
+        pk.y = pack_bf16x2(p[2], p[3]);
+        pk.z = pack_bf16x2(p[4], p[5]);
+        pk.w = pack_bf16x2(p[6], p[7]);
+        p_store_swizzled(Ps, em, c8, pk);
+      }
+      l = l * alpha + rs;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    // Final: O / l
+    if (nkv > 0 && mbar_wait(pv_done, (nkv - 1) & 1, abort_flag, a.status)) {
+      tc_fence_after();
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (size_t)row * a.d_model + h * dh;
+      for (int c = 0; c < dh / 16; ++c) {
+        float o[16];
+        tmem_ld16(t_o + lane_off + c * 16, o);
+        if (valid) {
+          uint4 w0, w1;
+          w0.x = pack_bf16x2(o[0] * inv, o[1] * inv);
+          w0.y = pack_bf16x2(o[2] * inv, o[3] * inv);
+          w0.z = pack_bf16x2(o[4] * inv, o[5] * inv);
+          w0.w = pack_bf16x2(o[6] * inv, o[7] * inv);
+          w1.x = pack_bf16x2(o[8] * inv, o[9] * inv);
+          w1.y = pack_bf16x2(o[10] * inv, o[11] * inv);
+          w1.z = pack_bf16x2(o[12] * inv, o[13] * inv);
+          w1.w = pack_bf16x2(o[14] * inv, o[15] * inv);
+          reinterpret_cast<uint4*>(out + c * 16)[0] = w0;
+          reinterpret_cast<uint4*>(out + c * 16)[1] = w1;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// SIMT attention (fp32 models): one warp per (row, head); lanes split the head dimension.
+// ------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void attn_simt_kernel(const T* __restrict__ q, T* __restrict__ out, KVAddr kv,
+                                 AttnSimtArgs a) {
+  const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int row = warp_global / a.H, h = warp_global % a.H;
+  if (row >= a.rows) return;
+  const int dh = a.dh;
+  const int per = dh / 32;   // dims per lane (1..4)
+  float qv[4], acc[4];
+  for (int t = 0; t < per; ++t) {
+    qv[t] = to_f(q[(size_t)row * a.d_model + h * dh + lane * per + t]) * a.scale;
+    acc[t] = 0.f;
+  }
+  const int seq = a.row_seq[row];
+  const T* K = reinterpret_cast<const T*>(kv.k) + seq * kv.seq_stride + a.layer * kv.layer_stride +
+               h * kv.head_stride;
+  const T* V = reinterpret_cast<const T*>(kv.v) + seq * kv.seq_stride + a.layer * kv.layer_stride +
+               h * kv.head_stride;
+  int nk;
+  int tq = 0, lq = 0;
+  if (a.mode == 0) nk = a.kvlen[row];
+  else { nk = a.nkeys; tq = a.type[row]; lq = a.label[row]; }
+  float m = -INFINITY, l = 0.f;
+  for (int key = 0; key < nk; ++key) {
+    if (a.mode == 1 && !step_causal_allowed(tq, lq, a.type[key], a.label[key])) continue;
+    float d = 0.f;
+    for (int t = 0; t < per; ++t) d += qv[t] * to_f(K[(size_t)key * dh + lane * per + t]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+    const float mn = fmaxf(m, d);
+    const float corr = (m == -INFINITY) ? 0.f : expf(m - mn);
+    const float p = expf(d - mn);
+    l = l * corr + p;
+    for (int t = 0; t < per; ++t) acc[t] = acc[t] * corr + p * to_f(V[(size_t)key * dh + lane * per + t]);
+    m = mn;
+  }
+  for (int t = 0; t < per; ++t)
+    out[(size_t)row * a.d_model + h * dh + lane * per + t] = from_f<T>(acc[t] / l);
+}
+
+// ------------------------------------------------------------------------------------------
+// Host side
+// ------------------------------------------------------------------------------------------
+static int attn_layout(int dh, AttnDev& d) {
+  const int q_bytes = 128 * dh * 2;
+  const int kv_bytes = 128 * dh * 2;
+  const int p_bytes = 128 * 128 * 2;
+  d.q_off = 0;
+  d.p_off = q_bytes;
+  d.stage_bytes = kv_bytes;
+  const int budget = 227 * 1024 - 1024 - 256;
+  int ns = (budget - q_bytes - p_bytes) / (2 * kv_bytes);
+  if (ns > 4) ns = 4;
+  d.nstages = ns;
+  d.k_off = q_bytes + p_bytes;
+  d.v_off = d.k_off + ns * kv_bytes;
+  d.bar_off = d.v_off + ns * kv_bytes;
+  return d.bar_off + 256 + 1024;
+}
+
+cudaError_t attn_tc_set_smem_attr() {
+  return cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              227 * 1024);
+}
+
+cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t stream) {
+  AttnDev d{};
+  d.mode = c.mode;
+  d.H = c.H;
+  d.dh = c.dh;
+  d.d_model = c.d_model;
+  d.layer = c.layer;
+  d.kvlen = c.kvlen;
+  d.type = c.type;
+  d.label = c.label;
+  d.cache_rows_per_seq = c.cache_rows_per_seq;
+  d.cap = c.cap;
+  d.scale_log2 = 1.4426950408889634f / sqrtf((float)c.dh);
+  d.out = c.out;
+  d.status = c.status;
+  if (c.n_seg < 1 || c.n_seg > kMaxBatch) return cudaErrorInvalidValue;
+  int nb = 0;
+  d.n_seg = c.n_seg;
+  for (int s = 0; s < c.n_seg; ++s) {
+    d.seg[s] = c.seg[s];
+    d.seg[s].tile0 = nb;
+    nb += (c.seg[s].rows + 127) / 128;
+  }
+  if (nb == 0) return cudaSuccess;
+  const int smem = attn_layout(c.dh, d);
+  dim3 grid(nb, c.H);
+  attn_tc_kernel<<<grid, kAttnThreads, smem, stream>>>(*c.tmQ, *c.tmK, *c.tmV, d);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_attn_simt(const T* q, T* out, const KVAddr& kv, const AttnSimtArgs& a,
+                             cudaStream_t stream) {
+  if (a.rows <= 0) return cudaSuccess;
+  const long long warps = (long long)a.rows * a.H;
+  const int threads = 128;
+  const long long blocks = (warps * 32 + threads - 1) / threads;
+  attn_simt_kernel<T><<<(unsigned)blocks, threads, 0, stream>>>(q, out, kv, a);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_attn_simt<float>(const float*, float*, const KVAddr&,
+                                             const AttnSimtArgs&, cudaStream_t);
+template cudaError_t launch_attn_simt<__nv_bfloat16>(const __nv_bfloat16*, __nv_bfloat16*,
+                                                     const KVAddr&, const AttnSimtArgs&,
+                                                     cudaStream_t);
+
+}  // namespace smdm

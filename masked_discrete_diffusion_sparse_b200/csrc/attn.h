@@ -1,0 +1,50 @@
+// Host-side interface of the attention kernels (see attn.cu).
+#pragma once
+#include "kernels.cuh"
+
+namespace smdm {
+
+// A contiguous run of query rows that belong to one sequence.
+struct AttnSeg {
+  int seq;      // sequence slot (selects the KV cache)
+  int row0;     // first forward row
+  int rows;     // number of rows
+  int nkeys;    // keys to scan: max kvlen over the rows (prefix mode) or n (label mode)
+  int tile0;    // filled in by the launcher
+};
+
+struct AttnCall {
+  int mode;                 // 0 = prefix (kvlen per row), 1 = label (step-causal predicate)
+  int H, dh, d_model, layer;
+  int n_seg;
+  AttnSeg seg[kMaxBatch];
+  const int* kvlen;
+  const int* type;
+  const int* label;
+  const CUtensorMap* tmQ;   // q [rows][d_model] bf16, box {64, 128}
+  const CUtensorMap* tmK;   // K cache as 2-D [cache rows][d_head] bf16, box {64, 128}
+  const CUtensorMap* tmV;   // V cache, same layout
+  long long cache_rows_per_seq;
+  int cap;
+  void* out;                // [rows][d_model] bf16
+  uint32_t* status;
+};
+
+struct AttnSimtArgs {
+  int mode;
+  int rows, H, dh, d_model, layer;
+  int nkeys;                // label mode
+  const int* row_seq;
+  const int* kvlen;
+  const int* type;
+  const int* label;
+  float scale;              // 1/sqrt(dh)
+};
+
+cudaError_t attn_tc_set_smem_attr();
+cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t stream);
+template <typename T>
+cudaError_t launch_attn_simt(const T* q, T* out, const KVAddr& kv, const AttnSimtArgs& a,
+                             cudaStream_t stream);
+
+}  // namespace smdm

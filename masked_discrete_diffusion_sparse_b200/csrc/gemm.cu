@@ -1,0 +1,404 @@
+// Weight-streaming GEMMs of the transformer step: Y[r][n] = sum_k X[r][k] * W[n][k].
+//
+// bf16 path (tcgen05): "swap-AB" tiles — the weight tile (128 output features x 64 of K) is
+// the MMA's A operand and the activation rows (up to 512 of them) are its N dimension, so the
+// per-step row count of a sparse step (|A| + |C| + registers, usually < 300) never pads the
+// 128-row MMA M dimension.  Work is split stream-K style: the (tile, 64-wide K chunk) units are
+// divided evenly over one CTA per SM; tiles cut between CTAs are finished by whichever CTA
+// contributes last (fp32 partials in L2-resident scratch, summed in a fixed order so results
+// are deterministic).  Warp roles: warp 0 issues TMA loads, warp 1 owns TMEM and issues
+// tcgen05.mma, warps 2-5 drain the accumulator through the fused epilogue.
+//
+// fp32 path (SIMT FFMA): the same tiles and epilogues for fp32 models, where a tf32 MMA would
+// not hold the 1e-4 tolerance.
+#include "gemm.h"
+
+namespace smdm {
+
+constexpr int kGemmThreads = 192;
+constexpr int kATileBytes = 128 * 128;   // 128 rows x 64 bf16
+
+struct SmemLayout {
+  int stage_bytes, a_bytes, b_bytes;
+  int nstages;
+  int stage_off;   // after 1024 alignment
+  int staging_off; // 2 x 16 x 128 floats
+  int bar_off;
+  int total;       // bytes of dynamic smem requested (incl. alignment slack)
+};
+
+static SmemLayout gemm_smem_layout(int RT, int max_stages) {
+  SmemLayout L;
+  L.a_bytes = kATileBytes;
+  L.b_bytes = RT * 128;
+  L.stage_bytes = L.a_bytes + L.b_bytes;
+  const int budget = 227 * 1024 - 1024 /*align*/ - 2 * 16 * 128 * 4 - 512 /*barriers*/;
+  L.nstages = budget / L.stage_bytes;
+  if (L.nstages > max_stages) L.nstages = max_stages;
+  L.stage_off = 0;
+  L.staging_off = L.nstages * L.stage_bytes;
+  L.bar_off = L.staging_off + 2 * 16 * 128 * 4;
+  L.total = L.bar_off + 512 + 1024;
+  return L;
+}
+
+struct GemmDev {
+  int KC;          // K / 64
+  int n_tiles;     // tiles of 128 A rows
+  int row_blocks;
+  int RT;          // activation rows per row block (multiple of 16; multiple of 32 if > 256)
+  int rows;        // valid activation rows
+  int row0;        // first activation row (TMA y offset)
+  long long units; // n_tiles * row_blocks * KC
+  int swiglu;
+  int nstages, stage_bytes, staging_off, bar_off;
+  int n_acc, tmem_cols;
+  float* partial;
+  unsigned* counters;
+  uint32_t* status;
+};
+
+SMDM_DEV bool from_tmem_release(bool full_tile, bool additive) { return full_tile || additive; }
+
+SMDM_DEV long long cta_start(long long g, long long U, long long G) { return g * U / G; }
+// CTA whose unit range contains unit u (inverse of cta_start).
+SMDM_DEV long long cta_of(long long u, long long U, long long G) { return ((u + 1) * G - 1) / U; }
+
+template <typename T>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+                   const __grid_constant__ CUtensorMap tmB, const GemmDev g, const EpiParams ep) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  float(*staging)[16][128] = reinterpret_cast<float(*)[16][128]>(smem + g.staging_off);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + g.bar_off);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + g.nstages;
+  uint64_t* acc_full = bars + 2 * g.nstages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_holder + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < g.nstages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (g.swiglu) tma_prefetch_desc(&tmA2);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, g.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+
+  const long long U = g.units, G = gridDim.x;
+  const long long u_begin = cta_start(blockIdx.x, U, G), u_end = cta_start(blockIdx.x + 1, U, G);
+  const int KC = g.KC;
+  const int part_rows = (g.RT > 256) ? (g.RT >> 1) : g.RT;
+  const int nparts = (g.RT > 256) ? 2 : 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (long long u = u_begin; u < u_end; ++u) {
+        const long long tile = u / KC;
+        const int kc = (int)(u % KC);
+        const int nt = (int)(tile / g.row_blocks), rb = (int)(tile % g.row_blocks);
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, g.status)) break;
+        uint8_t* A = smem + stage * g.stage_bytes;
+        uint8_t* B = A + kATileBytes;
+        mbar_arrive_expect_tx(&full[stage], g.stage_bytes);
+        if (g.swiglu) {
+          tma_load_2d(A, &tmA, &full[stage], kc * 64, nt * 64, pol_w);
+          tma_load_2d(A + kATileBytes / 2, &tmA2, &full[stage], kc * 64, nt * 64, pol_w);
+        } else {
+          tma_load_2d(A, &tmA, &full[stage], kc * 64, nt * 128, pol_w);
+        }
+        for (int p = 0; p < nparts; ++p)
+          tma_load_2d(B + p * part_rows * 128, &tmB, &full[stage], kc * 64,
+                      g.row0 + rb * g.RT + p * part_rows, pol_x);
+        if (++stage == g.nstages) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, part_rows, 0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      long long u = u_begin;
+      bool ok = true;
+      while (u < u_end && ok) {
+        const long long tile = u / KC;
+        const long long seg_end = min(u_end, (tile + 1) * KC);
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag, g.status)) break;
+        tc_fence_after();
+        const uint32_t dcol = tbase + acc * g.RT;
+        bool first = true;
+        for (; u < seg_end; ++u) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, g.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * g.stage_bytes);
+          const uint32_t b_addr = a_addr + kATileBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t adesc = sdesc_sw128(a_addr + kk * 32, 16, 1024);
+            for (int p = 0; p < nparts; ++p) {
+              const uint64_t bdesc = sdesc_sw128(b_addr + p * part_rows * 128 + kk * 32, 16, 1024);
+              umma_f16(dcol + p * part_rows, adesc, bdesc, idesc, (first && kk == 0) ? 0u : 1u);
+            }
+          }
+          umma_commit(&empty[stage]);
+          first = false;
+          if (++stage == g.nstages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[acc]);
+        if (g.n_acc == 2) {
+          acc ^= 1;
+          if (acc == 0) acc_phase ^= 1;
+        } else {
+          acc_phase ^= 1;
+        }
+      }
+    }
+  } else {
+    // Epilogue warps 2..5: TMEM lane quarter = warp % 4 -> output feature m.
+    const int q = warp & 3;
+    const int m = q * 32 + lane;
+    const int et = threadIdx.x - 64;   // 0..127, barrier participant index
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int sbuf = 0;
+    long long u = u_begin;
+    while (u < u_end) {
+      const long long tile = u / KC;
+      const long long tstart = tile * KC, tend = tstart + KC;
+      const long long seg_end = min(u_end, tend);
+      const bool full_tile = (u == tstart) && (seg_end == tend);
+      const int nt = (int)(tile / g.row_blocks), rb = (int)(tile % g.row_blocks);
+      const int rbase = rb * g.RT;                       // first row of this block (relative)
+      const int nvalid_rows = min(g.RT, g.rows - rbase);
+      const int nchunks = (nvalid_rows + 15) >> 4;
+      u = seg_end;
+      if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, g.status)) break;
+      tc_fence_after();
+      const uint32_t tacc = tbase + (uint32_t(q * 32) << 16) + acc * g.RT;
+      bool do_epi = true;
+      // Residual epilogues are additive: split segments add straight into x (fp32 atomics).
+      const bool additive = (ep.kind == kEpiResid);
+      long long g_first = 0, g_last = -1;
+      if (!full_tile && !additive) {
+        const long long me = blockIdx.x;
+        const int slot = (cta_start(me, U, G) < tstart) ? 1 : 0;
+        float* P = g.partial + ((size_t)me * 2 + slot) * (size_t)g.RT * 128;
+        for (int c = 0; c < nchunks; ++c) {
+          float v[16];
+          tmem_ld16(tacc + c * 16, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) __stcg(&P[(size_t)(c * 16 + j) * 128 + m], v[j]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        __threadfence();
+        named_bar_sync(1, 128);
+        g_first = cta_of(tstart, U, G);
+        g_last = cta_of(tend - 1, U, G);
+        if (et == 0) {
+          const unsigned nseg = (unsigned)(g_last - g_first + 1);
+          const unsigned prev = atomicAdd(&g.counters[tile], 1u);
+          const int is_last = (prev == nseg - 1) ? 1 : 0;
+          if (is_last) g.counters[tile] = 0u;   // ready for the next launch
+          *last_flag = is_last;
+        }
+        named_bar_sync(1, 128);
+        do_epi = (*last_flag != 0);
+        __threadfence();
+      }
+      if (do_epi) {
+        const bool from_tmem = full_tile || additive;
+        for (int c = 0; c < nchunks; ++c) {
+          float v[16];
+          if (from_tmem) {
+            tmem_ld16(tacc + c * 16, v);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = 0.f;
+            // fixed summation order (segment order) -> deterministic results
+            for (long long gg = g_first; gg <= g_last; ++gg) {
+              const int sl = (cta_start(gg, U, G) < tstart) ? 1 : 0;
+              const float* P = g.partial + ((size_t)gg * 2 + sl) * (size_t)g.RT * 128;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] += __ldcg(&P[(size_t)(c * 16 + j) * 128 + m]);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) staging[sbuf][j][m] = v[j];
+          named_bar_sync(1, 128);
+          epilogue_tile<T>(ep, staging[sbuf], nt * 128, rbase + c * 16, m, !full_tile);
+          sbuf ^= 1;
+        }
+      }
+      if (from_tmem_release(full_tile, additive)) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      }
+      if (g.n_acc == 2) {
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      } else {
+        acc_phase ^= 1;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, g.tmem_cols);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// fp32 SIMT GEMM: CTA = 128 features x 16 rows, 128 threads, K in steps of 32.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(128)
+    gemm_simt_kernel(const float* __restrict__ W, const float* __restrict__ W2,
+                     const float* __restrict__ X, int ldx, int K, int n_rows_w, int rows,
+                     int swiglu, EpiParams ep) {
+  __shared__ float Ws[128][33];
+  __shared__ float Xs[16][33];
+  __shared__ float S[16][128];
+  const int m = threadIdx.x;
+  const int nt = blockIdx.x, r0 = blockIdx.y * 16;
+  float acc[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+  for (int k0 = 0; k0 < K; k0 += 32) {
+    // load W tile rows (128) x 32
+    for (int idx = m; idx < 128 * 32; idx += 128) {
+      const int rr = idx / 32, kk = idx % 32;
+      int wrow;
+      const float* src;
+      if (swiglu) {
+        wrow = nt * 64 + (rr & 63);
+        src = (rr < 64) ? W : W2;
+      } else {
+        wrow = nt * 128 + rr;
+        src = W;
+      }
+      Ws[rr][kk] = (wrow < n_rows_w && k0 + kk < K) ? src[(size_t)wrow * K + k0 + kk] : 0.f;
+    }
+    for (int idx = m; idx < 16 * 32; idx += 128) {
+      const int j = idx / 32, kk = idx % 32;
+      Xs[j][kk] = (r0 + j < rows && k0 + kk < K) ? X[(size_t)(r0 + j) * ldx + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < 32; ++kk) {
+      const float w = Ws[m][kk];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) acc[j] = fmaf(w, Xs[j][kk], acc[j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) S[j][m] = acc[j];
+  __syncthreads();
+  epilogue_tile<float>(ep, S, nt * 128, r0, m, false);
+}
+
+// ------------------------------------------------------------------------------------------
+// Host side
+// ------------------------------------------------------------------------------------------
+
+int gemm_tc_row_tile(int rows) {
+  // One row block of up to 512 rows keeps every weight tile streamed exactly once.
+  const int R16 = (rows + 15) & ~15;
+  if (R16 <= 256) return R16;
+  if (R16 <= 512) return (rows + 31) & ~31;
+  return 256;
+}
+
+int gemm_tc_box_rows(int rows) {
+  const int RT = gemm_tc_row_tile(rows);
+  return RT > 256 ? RT / 2 : RT;
+}
+
+static int pow2_ceil(int x) {
+  int p = 32;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+cudaError_t gemm_tc_set_smem_attr() {
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<__nv_bfloat16>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  return e;
+}
+
+cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream) {
+  if (c.rows <= 0) return cudaSuccess;
+  GemmDev g{};
+  g.KC = c.K / 64;
+  g.swiglu = c.swiglu;
+  g.n_tiles = c.swiglu ? (c.n_out + 63) / 64 : (c.n_out + 127) / 128;
+  g.RT = gemm_tc_row_tile(c.rows);
+  g.row_blocks = (c.rows + g.RT - 1) / g.RT;
+  g.rows = c.rows;
+  g.row0 = c.row0;
+  g.units = (long long)g.n_tiles * g.row_blocks * g.KC;
+  const SmemLayout L = gemm_smem_layout(g.RT, c.max_stages > 0 ? c.max_stages : 8);
+  g.nstages = L.nstages;
+  g.stage_bytes = L.stage_bytes;
+  g.staging_off = L.staging_off;
+  g.bar_off = L.bar_off;
+  g.n_acc = (g.RT <= 256) ? 2 : 1;
+  g.tmem_cols = pow2_ceil(g.n_acc * g.RT);
+  g.partial = c.partial;
+  g.counters = c.counters;
+  g.status = c.status;
+  long long G = c.num_ctas;
+  if (G > g.units) G = g.units;
+  if (G < 1) G = 1;
+  if (g.n_tiles * g.row_blocks > c.max_tiles) return cudaErrorInvalidValue;
+  if ((long long)g.RT * 128 * 2 * G * 4 > (long long)c.partial_bytes)
+    return cudaErrorInvalidValue;  // split-K scratch too small for this row tile
+  gemm_tc_kernel<__nv_bfloat16><<<(unsigned)G, kGemmThreads, L.total, stream>>>(
+      *c.tmA, c.swiglu ? *c.tmA2 : *c.tmA, *c.tmB, g, c.epi);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_simt(const float* W, const float* W2, const float* X, int ldx, int K,
+                             int n_out, int rows, int swiglu, const EpiParams& ep,
+                             cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  const int n_tiles = swiglu ? (n_out + 63) / 64 : (n_out + 127) / 128;
+  dim3 grid(n_tiles, (rows + 15) / 16);
+  gemm_simt_kernel<<<grid, 128, 0, stream>>>(W, W2, X, ldx, K, n_out, rows, swiglu, ep);
+  return cudaGetLastError();
+}
+
+
+}  // namespace smdm

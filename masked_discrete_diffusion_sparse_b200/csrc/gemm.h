@@ -1,0 +1,34 @@
+// Host-side interface of the GEMM kernels (see gemm.cu).
+#pragma once
+#include "kernels.cuh"
+
+namespace smdm {
+
+struct GemmCall {
+  const CUtensorMap* tmA;   // weights [n_out][K] bf16, box {64, 128} (SwiGLU: gate, box {64, 64})
+  const CUtensorMap* tmA2;  // SwiGLU: up weights, box {64, 64}
+  const CUtensorMap* tmB;   // activations [*][K] bf16, box {64, gemm_tc_box_rows(rows)}
+  int K;
+  int n_out;                // output features (SwiGLU: ffn)
+  int rows;                 // activation rows
+  int row0;                 // first activation row in tmB
+  int swiglu;
+  int num_ctas;             // persistent grid size (one CTA per SM)
+  int max_stages;           // 0 = as many as fit
+  float* partial;           // split-K scratch: [num_ctas][2][row_tile][128] fp32
+  size_t partial_bytes;
+  unsigned* counters;       // [max_tiles], zero-initialised; restored to zero by the kernel
+  int max_tiles;
+  uint32_t* status;
+  EpiParams epi;
+};
+
+int gemm_tc_row_tile(int rows);
+int gemm_tc_box_rows(int rows);
+cudaError_t gemm_tc_set_smem_attr();
+cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream);
+cudaError_t launch_gemm_simt(const float* W, const float* W2, const float* X, int ldx, int K,
+                             int n_out, int rows, int swiglu, const EpiParams& ep,
+                             cudaStream_t stream);
+
+}  // namespace smdm

@@ -1,0 +1,316 @@
+// The non-contraction kernels of the sparse sampling step:
+//   pack        — builds the step's sparse row set (Sparse-LaViDa Sec. 3.1 / Appendix 7.2:
+//                 |A| + |C| + m rows) and the per-row attention prefixes;
+//   embed_norm  — embedding gather into the fp32 residual stream + first RMSNorm;
+//   rmsnorm     — RMSNorm (optionally gathering the decode-set rows for the LM head);
+//   unmask      — confidence/argmax from the LM-head partials, top-n selection and the
+//                 scatter of committed tokens into the grid (Figure-3 example, Sec. 3.2);
+//   debug_mask  — the device step-causal predicate as a bitmap (test hook).
+#include "misc.h"
+
+namespace smdm {
+
+// ------------------------------------------------------------------------------------------
+// pack: one CTA per sequence of a sampling step.  Rows of sequence s, in order:
+//   new cache  (tokens decoded at step k-1; id from the grid; CLEAN, label k-1),
+//   queries    (the decode set C_k; id [MASK]; MASK, label k),
+//   registers  (ids V+2+j, positions L+1+j; REG, label k).
+// kvlen: new-cache rows see the cache plus the new-cache rows; query and register rows see
+// every row of the step.  slot: K/V of row i go to cache slot ctx + i.
+// ------------------------------------------------------------------------------------------
+__global__ void pack_step_kernel(PackArgs a) {
+  const PackSeq& s = a.s[blockIdx.x];
+  __shared__ int qbuf_count;
+  __shared__ int warp_counts[32];
+  const int tid = threadIdx.x;
+  const int L = s.P + s.Lg;
+  const int R = s.n_new + s.n_q + s.n_reg;
+  const int q0 = s.row0 + s.n_new;
+  if (s.qpos == nullptr) {
+    // Block mode: C = every still-masked position of [block_lo, block_hi), in position order.
+    if (tid == 0) qbuf_count = 0;
+    __syncthreads();
+    for (int base = s.block_lo; base < s.block_hi; base += blockDim.x) {
+      const int p = base + tid;
+      const bool masked = (p < s.block_hi) && (s.grid[p - s.P - 1] < 0);
+      const unsigned ballot = __ballot_sync(0xffffffffu, masked);
+      const int lane = tid & 31, w = tid >> 5;
+      if (lane == 0) warp_counts[w] = __popc(ballot);
+      __syncthreads();
+      int before = 0;
+      for (int i = 0; i < w; ++i) before += warp_counts[i];
+      const int idx = qbuf_count + before + __popc(ballot & ((1u << lane) - 1u));
+      if (masked && idx < s.n_q) {
+        const int r = q0 + idx;
+        a.rows.pos[r] = p;
+        a.rows.qpos[s.qbase + idx] = p;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int tot = 0;
+        for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += warp_counts[i];
+        qbuf_count += tot;
+      }
+      __syncthreads();
+    }
+    if (tid == 0 && qbuf_count != s.n_q) atomicOr(a.status, kStatusBounds);
+  }
+  for (int i = tid; i < R; i += blockDim.x) {
+    const int r = s.row0 + i;
+    int id, pos, type, label, kvlen;
+    if (i < s.n_new) {
+      pos = s.newpos[i];
+      const bool ok = pos > s.P && pos <= L;
+      id = ok ? s.grid[pos - s.P - 1] : 0;
+      if (!ok || id < 0) {
+        atomicOr(a.status, kStatusBounds);
+        id = 0;
+      }
+      type = kTypeClean;
+      label = s.label - 1;
+      kvlen = s.ctx + s.n_new;
+    } else if (i < s.n_new + s.n_q) {
+      const int j = i - s.n_new;
+      if (s.qpos != nullptr) {
+        pos = s.qpos[j];
+        a.rows.pos[r] = pos;
+        a.rows.qpos[s.qbase + j] = pos;
+      } else {
+        pos = -1;   // written by the scan above
+      }
+      id = a.vocab;   // [MASK]
+      type = kTypeMask;
+      label = s.label;
+      kvlen = s.ctx + R;
+      a.rows.qrow[s.qbase + j] = r;
+    } else {
+      const int j = i - s.n_new - s.n_q;
+      pos = L + 1 + j;
+      id = a.vocab + 2 + j;
+      type = kTypeReg;
+      label = s.label;
+      kvlen = s.ctx + R;
+    }
+    a.rows.ids[r] = id;
+    if (pos >= 0) a.rows.pos[r] = pos;
+    a.rows.type[r] = type;
+    a.rows.label[r] = label;
+    a.rows.seq[r] = s.seq;
+    a.rows.slot[r] = s.ctx + i;
+    a.rows.kvlen[r] = kvlen;
+  }
+  if (s.qpos != nullptr) {
+    // checked: every explicit query position lies in the generated part and is still masked
+    for (int j = tid; j < s.n_q; j += blockDim.x) {
+      const int p = s.qpos[j];
+      if (p <= s.P || p > L || s.grid[p - s.P - 1] >= 0) atomicOr(a.status, kStatusBounds);
+    }
+  }
+}
+
+// Prefill / dense / training-form rows: one thread per row.
+__global__ void pack_linear_kernel(LinearPackArgs a) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= a.n) return;
+  int id, pos, type, label;
+  if (a.mode == kPackPrefill) {
+    id = a.prompt[i];
+    pos = i + 1;
+    type = kTypePrompt;
+    label = 0;
+  } else if (a.mode == kPackDense) {
+    pos = i + 1;
+    if (i < a.P) {
+      id = a.prompt[i];
+      type = kTypePrompt;
+    } else {
+      const int g = a.grid[i - a.P];
+      id = g < 0 ? a.vocab : g;
+      type = g < 0 ? kTypeMask : kTypeClean;
+      a.rows.qrow[i - a.P] = i;
+      a.rows.qpos[i - a.P] = pos;
+    }
+    label = 0;
+  } else {
+    id = a.ids[i];
+    pos = a.pos[i];
+    type = a.type[i];
+    label = a.label[i];
+  }
+  if (id < 0 || id >= a.emb_rows || pos < 0 || pos >= a.max_pos) {
+    atomicOr(a.status, kStatusBounds);
+    id = 0;
+    pos = 0;
+  }
+  a.rows.ids[i] = id;
+  a.rows.pos[i] = pos;
+  a.rows.type[i] = type;
+  a.rows.label[i] = label;
+  a.rows.seq[i] = a.seq;
+  a.rows.slot[i] = i;
+  a.rows.kvlen[i] = a.n;
+}
+
+__global__ void gather_rows_kernel(const int* __restrict__ src_rows, int n, int* __restrict__ qrow) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) qrow[i] = src_rows[i];
+}
+
+// ------------------------------------------------------------------------------------------
+// RMSNorm: out[r] = x[src] / sqrt(mean(x[src]^2) + eps) * g.  With emb != nullptr the source
+// row is first gathered from the embedding table into the fp32 residual stream x.
+// ------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void rmsnorm_kernel(NormArgs a) {
+  const int r = blockIdx.x;
+  const int src = a.gather ? a.gather[r] : r;
+  float* xr = a.x + (size_t)src * a.d;
+  const T* g = reinterpret_cast<const T*>(a.gain);
+  __shared__ float red[32];
+  float ss = 0.f;
+  if (a.emb) {
+    const int id = a.ids[src];
+    const T* e = reinterpret_cast<const T*>(a.emb) + (size_t)id * a.d;
+    for (int i = threadIdx.x; i < a.d; i += blockDim.x) {
+      const float v = to_f(e[i]);
+      xr[i] = v;
+      ss += v * v;
+    }
+  } else {
+    for (int i = threadIdx.x; i < a.d; i += blockDim.x) {
+      const float v = xr[i];
+      ss += v * v;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float t = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (threadIdx.x == 0) red[0] = t;
+  }
+  __syncthreads();
+  const float rstd = rsqrtf(red[0] / (float)a.d + a.eps);
+  T* out = reinterpret_cast<T*>(a.out) + (size_t)r * a.d;
+  for (int i = threadIdx.x; i < a.d; i += blockDim.x) out[i] = from_f<T>(xr[i] * rstd * to_f(g[i]));
+}
+
+// ------------------------------------------------------------------------------------------
+// unmask: one CTA per sequence.
+// ------------------------------------------------------------------------------------------
+__global__ void unmask_kernel(UnmaskArgs a) {
+  const UnmaskSeq& s = a.s[blockIdx.x];
+  extern __shared__ float sh[];
+  float* conf = sh;                                     // [n_q]
+  int* tok = reinterpret_cast<int*>(sh + s.n_q);        // [n_q]
+  int* commit = tok + s.n_q;                            // [n_q]
+  for (int j = threadIdx.x; j < s.n_q; j += blockDim.x) {
+    const int lr = s.dense ? (a.qpos_of[s.qbase + j] - s.P - 1) : (s.qbase + j);
+    const float* pm = a.pmax + (size_t)(s.lbase + lr) * a.n_vt;
+    const float* ps = a.psum + (size_t)(s.lbase + lr) * a.n_vt;
+    const int* pa = a.parg + (size_t)(s.lbase + lr) * a.n_vt;
+    float M = -INFINITY;
+    int arg = 0;
+    for (int t = 0; t < a.n_vt; ++t) {
+      if (pm[t] > M) { M = pm[t]; arg = pa[t]; }   // first tile wins ties -> lowest id
+    }
+    float z = 0.f;
+    for (int t = 0; t < a.n_vt; ++t) z += ps[t] * __expf(pm[t] - M);
+    conf[j] = 1.f / z;
+    tok[j] = arg;
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < s.n_q; j += blockDim.x) {
+    int c = 1;
+    if (s.policy == 1) {
+      int rank = 0;
+      const float cj = conf[j];
+      for (int i = 0; i < s.n_q; ++i) rank += (conf[i] > cj) || (conf[i] == cj && i < j);
+      c = rank < s.n_commit;
+    }
+    commit[j] = c;
+    if (a.tok_out) a.tok_out[s.qbase + j] = tok[j];
+    if (a.conf_out) a.conf_out[s.qbase + j] = conf[j];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int j = 0; j < s.n_q; ++j) {
+      if (!commit[j]) continue;
+      const int p = a.qpos_of[s.qbase + j];
+      if (p <= s.P || p > s.P + s.Lg) {
+        atomicOr(a.status, kStatusBounds);
+        continue;
+      }
+      s.grid[p - s.P - 1] = tok[j];
+      if (s.newpos) s.newpos[n] = p;
+      ++n;
+    }
+  }
+}
+
+__global__ void debug_mask_kernel(const int* type, const int* label, int n, uint32_t* bitmap) {
+  const int i = blockIdx.x;
+  const int words = (n + 31) / 32;
+  for (int w = threadIdx.x; w < words; w += blockDim.x) {
+    uint32_t bits = 0;
+    for (int b = 0; b < 32; ++b) {
+      const int j = w * 32 + b;
+      if (j < n && step_causal_allowed(type[i], label[i], type[j], label[j])) bits |= 1u << b;
+    }
+    bitmap[(size_t)i * words + w] = bits;
+  }
+}
+
+__global__ void fill_i32_kernel(int* p, int n, int v) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = v;
+}
+
+// ------------------------------------------------------------------------------------------
+// launchers
+// ------------------------------------------------------------------------------------------
+cudaError_t launch_pack_step(const PackArgs& a, cudaStream_t st) {
+  pack_step_kernel<<<a.n_seq, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+cudaError_t launch_pack_linear(const LinearPackArgs& a, cudaStream_t st) {
+  if (a.n <= 0) return cudaSuccess;
+  pack_linear_kernel<<<(a.n + 255) / 256, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+cudaError_t launch_gather_rows(const int* src, int n, int* qrow, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  gather_rows_kernel<<<(n + 255) / 256, 256, 0, st>>>(src, n, qrow);
+  return cudaGetLastError();
+}
+template <typename T>
+cudaError_t launch_rmsnorm(const NormArgs& a, int rows, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  rmsnorm_kernel<T><<<rows, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+template cudaError_t launch_rmsnorm<float>(const NormArgs&, int, cudaStream_t);
+template cudaError_t launch_rmsnorm<__nv_bfloat16>(const NormArgs&, int, cudaStream_t);
+
+cudaError_t launch_unmask(const UnmaskArgs& a, int max_nq, cudaStream_t st) {
+  const size_t smem = (size_t)max_nq * 12;
+  unmask_kernel<<<a.n_seq, 256, smem, st>>>(a);
+  return cudaGetLastError();
+}
+cudaError_t launch_debug_mask(const int* type, const int* label, int n, uint32_t* bitmap,
+                              cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  debug_mask_kernel<<<n, 128, 0, st>>>(type, label, n, bitmap);
+  return cudaGetLastError();
+}
+cudaError_t launch_fill_i32(int* p, int n, int v, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  fill_i32_kernel<<<(n + 255) / 256, 256, 0, st>>>(p, n, v);
+  return cudaGetLastError();
+}
+
+}  // namespace smdm

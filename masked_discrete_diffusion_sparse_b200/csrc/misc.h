@@ -1,0 +1,91 @@
+// Host-side interface of the pack / norm / unmask kernels (see misc.cu).
+#pragma once
+#include "kernels.cuh"
+
+namespace smdm {
+
+struct PackSeq {
+  int seq;          // sequence slot
+  int row0;         // first forward row of this sequence
+  int n_new, n_q, n_reg;
+  int ctx;          // cache length before this step
+  int P, Lg;
+  int label;        // step number k
+  int qbase;        // first logit row of this sequence
+  int block_lo, block_hi;   // block mode (qpos == nullptr)
+  const int* qpos;  // explicit decode set or nullptr
+  const int* grid;  // [Lg]
+  const int* newpos;// [n_new] positions decoded at the previous step
+};
+
+struct PackArgs {
+  int n_seq;
+  PackSeq s[kMaxBatch];
+  int vocab;
+  Rows rows;
+  uint32_t* status;
+};
+
+enum { kPackPrefill = 0, kPackDense = 1, kPackTrain = 2 };
+
+struct LinearPackArgs {
+  int mode;
+  int n;            // rows
+  int seq;
+  int P;
+  int vocab, emb_rows, max_pos;
+  const int* prompt;    // prefill / dense
+  const int* grid;      // dense
+  const int* ids;       // training form
+  const int* pos;
+  const int* type;
+  const int* label;
+  Rows rows;
+  uint32_t* status;
+};
+
+struct NormArgs {
+  float* x;           // fp32 residual rows [*][d]
+  const void* gain;   // [d], weight dtype
+  void* out;          // [rows][d], activation dtype
+  const int* gather;  // optional: out row r normalises x row gather[r]
+  const void* emb;    // optional: x[src] = emb[ids[src]] first
+  const int* ids;
+  int d;
+  float eps;
+};
+
+struct UnmaskSeq {
+  int qbase, n_q;     // this sequence's decode-set rows: qbase .. qbase + n_q - 1
+  int lbase;          // first LM-head row of this sequence
+  int dense;          // LM-head row of decode row j = qpos - P - 1 (dense comparator)
+  int policy, n_commit;
+  int P, Lg;
+  int* grid;
+  int* newpos;        // committed positions in row order (next step's new-cache rows)
+};
+
+struct UnmaskArgs {
+  int n_seq;
+  UnmaskSeq s[kMaxBatch];
+  int n_vt;           // vocab tiles of 128
+  const float* pmax;
+  const float* psum;
+  const int* parg;
+  const int* qpos_of; // decode row -> position
+  int* tok_out;       // optional
+  float* conf_out;    // optional
+  uint32_t* status;
+};
+
+cudaError_t launch_pack_step(const PackArgs& a, cudaStream_t st);
+cudaError_t launch_pack_linear(const LinearPackArgs& a, cudaStream_t st);
+cudaError_t launch_gather_rows(const int* src, int n, int* qrow, cudaStream_t st);
+template <typename T>
+cudaError_t launch_rmsnorm(const NormArgs& a, int rows, cudaStream_t st);
+cudaError_t launch_unmask(const UnmaskArgs& a, int max_nq, cudaStream_t st);
+cudaError_t launch_debug_mask(const int* type, const int* label, int n, uint32_t* bitmap,
+                              cudaStream_t st);
+cudaError_t launch_fill_i32(int* p, int n, int v, cudaStream_t st);
+
+}  // namespace smdm

@@ -1,0 +1,53 @@
+"""The C ABI library loads and exports every entry point that include/smdm.h declares (CPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import masked_discrete_diffusion_sparse_b200 as smdm
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "smdm.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(smdm_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for s in ("smdm_create", "smdm_prefill", "smdm_step", "smdm_generate",
+              "smdm_forward_stepcausal"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol():
+    if not os.path.exists(smdm.LIB_PATH):
+        from masked_discrete_diffusion_sparse_b200 import build
+        build.build()
+    lib = smdm.lib()
+    for s in declared_symbols():
+        assert hasattr(lib, s), s
+    assert set(declared_symbols()) <= set(smdm.EXPORTED)
+
+
+def test_invalid_config_is_rejected_without_gpu():
+    lib = smdm.lib()
+    bad = smdm.make_config(2, 100, 3, 33, 64, 10, dtype=smdm.SMDM_BF16, max_batch=1, max_len=10,
+                           max_step_rows=10, max_rows=10)
+    assert lib.smdm_workspace_bytes(ctypes.byref(bad)) == 0
+    bad2 = smdm.make_config(2, 256, 2, 128, 704, 1000, dtype=smdm.SMDM_BF16, max_batch=99,
+                            max_len=10, max_step_rows=10, max_rows=10)
+    assert lib.smdm_workspace_bytes(ctypes.byref(bad2)) == 0
+
+
+def test_model_refuses_to_run_without_cuda():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    cfg = smdm.make_config(2, 256, 2, 128, 704, 1000, max_batch=1, max_len=300,
+                           max_step_rows=200, max_rows=300)
+    with pytest.raises(RuntimeError):
+        smdm.Model(cfg, {})
