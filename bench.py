@@ -1,0 +1,502 @@
+#!/usr/bin/env python
+"""Benchmark: decoded tokens/s of full sparse masked-diffusion sampling runs on B200.
+
+One bench "step" = one full sampling run of the workload: prefill of the prompt plus every
+sampling step of the plan (pack -> transformer stack under the step-causal mask -> sparse LM head
+-> unmask), i.e. every stage of the hot path once per sampling step.  The timed region replays
+the run as one CUDA graph with all inputs resident in HBM; `e2e` repeats the measurement through
+the public API (smdm_generate) with the prompt and plan copied from pinned host memory and the
+token grid read back every run.
+
+Default workload: text-to-image 4096 tokens — 4-layer bf16 transformer, d=4096, 32 heads x 128,
+SwiGLU ffn 11008, vocab 8192; prompt 256, 64x64 grid, 64 registers, 64 cosine steps, stratified
+2-D order; batch 1.  Weights are synthetic N(0, 0.02) drawn on the device from a seed (1.69 GB,
+far larger than the 126 MB L2, so every run streams them from HBM; no L2 flush is needed).
+
+N > 1 GPUs (torchrun): independent replicas, one sequence set per rank, no collective on the
+data path; value = all ranks' decoded tokens / the slowest rank's time.
+
+`--impl reference` times the fp64 CPU oracle on the host cores on a bounded sample of the same
+workload (prefill + the first sampling step) and prints the same JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "decoded tokens/s per full sparse-MDM sampling run"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10, help="timed full runs")
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="D", choices=["A", "B", "C", "D", "D4", "E"])
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------------------------
+# workload description and algorithmic roofline (what the method must move / compute)
+# ----------------------------------------------------------------------------------------------
+
+def describe(wl: synth.Workload) -> dict:
+    m = wl.model
+    return {"workload": {"A": "tiny-fp32", "B": "text-semiAR", "C": "T2I-1024", "D": "T2I-4096",
+                         "D4": "T2I-4096-batch4", "E": "image-editing"}.get(wl.name, wl.name),
+            "layers": m.n_layers, "d_model": m.d_model, "heads": f"{m.n_heads}x{m.d_head}",
+            "d_ffn": m.d_ffn, "vocab": m.vocab, "registers": m.n_reg, "prompt": wl.prompt_len,
+            "gen_len": wl.gen_len, "sampling_steps": wl.n_steps, "batch": wl.batch,
+            "plan": wl.plan}
+
+
+def step_shapes(wl: synth.Workload, plan: synth.Plan):
+    """Per sampling step: (rows R, decode rows q, cache length ctx before the step, n_new)."""
+    P, Lg, m = wl.prompt_len, wl.gen_len, wl.model
+    out = []
+    ctx, n_new = P, 0
+    for k in range(1, wl.n_steps + 1):
+        if plan.kind == "order":
+            q = int(plan.n_per_step[k - 1])
+            c = q
+        else:
+            j = (k - 1) % plan.steps_per_block
+            q = plan.block - j * plan.commit
+            c = plan.commit
+        R = n_new + q + m.n_reg
+        out.append((R, q, ctx, n_new))
+        ctx += n_new
+        n_new = c
+    return out
+
+
+def layer_params(m: synth.ModelShape) -> int:
+    d, f = m.d_model, m.d_ffn
+    return 4 * d * d + 3 * d * f
+
+
+def forward_cost(m: synth.ModelShape, R: int, q: int, kv_sum: int, kv_keys: int, es: int = 2):
+    """Algorithmic (bytes, flops) of one forward over R rows with q logit rows.
+    kv_sum = sum over rows of visible keys; kv_keys = distinct keys read per layer."""
+    d, V, L = m.d_model, m.vocab, m.n_layers
+    wbytes = es * (L * layer_params(m) + (V * d if q else 0))
+    act = L * R * es * (d + 3 * d + d + d + d + 2 * m.d_ffn + m.d_ffn + d) + L * R * 4 * d * 4
+    kv = L * (kv_keys * 2 * d * es + R * 2 * d * es)
+    flops = 2 * R * L * layer_params(m) + 2 * q * V * d + L * 4 * d * kv_sum
+    return wbytes + act + kv, flops
+
+
+def run_cost(wl: synth.Workload, plan: synth.Plan):
+    """List of (bytes, flops) per forward of one full run (prefill first)."""
+    m, P = wl.model, wl.prompt_len
+    costs = [forward_cost(m, P, 0, P * P, P)] if P else []
+    for (R, q, ctx, n_new) in step_shapes(wl, plan):
+        kv_sum = n_new * (ctx + n_new) + (R - n_new) * (ctx + R)
+        costs.append(forward_cost(m, R, q, kv_sum, ctx + R))
+    return costs
+
+
+def gemm_bytes_per_run(wl: synth.Workload, plan: synth.Plan, es=2):
+    """Algorithmic bytes of the GEMM launches of one full run: weights once per launch plus
+    activation operand reads and output writes."""
+    m = wl.model
+    d, f, V, L = m.d_model, m.d_ffn, m.vocab, m.n_layers
+    tot = 0
+    fwd = ([(wl.prompt_len, 0)] if wl.prompt_len else []) + \
+          [(R, q) for (R, q, _, _) in step_shapes(wl, plan)]
+    for R, q in fwd:
+        per_layer = (es * (3 * d * d + R * d + R * 3 * d)            # qkv: W, X, q/k/v out
+                     + es * (d * d + R * d) + 4 * 2 * R * d          # o-proj: W, X, x rmw
+                     + es * (2 * f * d + R * d + R * f)              # gate/up: W, X, act out
+                     + es * (d * f + R * f) + 4 * 2 * R * d)         # down: W, X, x rmw
+        tot += L * per_layer
+        if q:
+            tot += es * (V * d + q * d) + 4 * 3 * q * ((V + 127) // 128)
+    return tot
+
+
+# ----------------------------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"smdm_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(loaded)}
+
+
+# ----------------------------------------------------------------------------------------------
+# CPU oracle (reported baseline and the reference arm)
+# ----------------------------------------------------------------------------------------------
+
+def oracle_sample(wl: synth.Workload):
+    """Time the fp64 oracle on the host: prefill + the first sampling step of sequence 0.
+    Returns (seconds, decoded tokens, description, threads)."""
+    import oracle
+    w = synth.make_weights(wl.model, wl.seed)
+    om = oracle.Model(w)
+    prompt = synth.make_prompt(wl)
+    plan = synth.make_plan(wl)
+    t0 = time.perf_counter()
+    st = oracle.Incremental(om, prompt, wl.gen_len)
+    qp = oracle.query_set(plan, st, 1)
+    lg = st.step_logits(qp)
+    tok, conf, rows = oracle.unmask(lg, oracle.POLICY_ALL if plan.kind == "order"
+                                    else oracle.POLICY_TOPN, plan.commit)
+    dt = time.perf_counter() - t0
+    n_dec = len(rows)
+    threads = _blas_threads()
+    desc = (f"oracle prefill ({wl.prompt_len} rows) + sampling step 1 ({len(qp)} decode rows, "
+            f"{n_dec} tokens committed) of the same workload, fp64 numpy")
+    return dt, n_dec, desc, threads
+
+
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    times = []
+    n_dec = 1
+    desc = ""
+    threads = 1
+    for i in range(args.warmup + args.steps):
+        dt, n_dec, desc, threads = oracle_sample(wl)
+        if i >= args.warmup:
+            times.append(dt)
+    mean = sum(times) / len(times)
+    value = n_dec * wl.batch / mean
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": mean * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": describe(wl),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------------------------
+# native arm
+# ----------------------------------------------------------------------------------------------
+
+def device_weights(wl: synth.Workload, seed: int, device):
+    import torch
+    m = wl.model
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    dt = torch.bfloat16 if m.dtype == synth.BF16 else torch.float32
+
+    def rnd(*shape):
+        return (torch.randn(*shape, generator=g, device=device, dtype=torch.float32) * 0.02).to(dt)
+
+    def ones(n):
+        return torch.ones(n, device=device, dtype=dt)
+
+    d, f, V = m.d_model, m.d_ffn, m.vocab
+    w = {"emb": rnd(m.emb_rows, d), "final_norm": ones(d), "lm_head": rnd(V, d)}
+    for k in ("attn_norm", "w_qkv", "w_o", "mlp_norm", "w_gate", "w_up", "w_down"):
+        w[k] = []
+    for _ in range(m.n_layers):
+        w["attn_norm"].append(ones(d))
+        w["w_qkv"].append(rnd(3 * d, d))
+        w["w_o"].append(rnd(d, d))
+        w["mlp_norm"].append(ones(d))
+        w["w_gate"].append(rnd(f, d))
+        w["w_up"].append(rnd(f, d))
+        w["w_down"].append(rnd(d, f))
+    return w
+
+
+def capacities(wl, plans):
+    m = wl.model
+    msr = 1
+    for plan in plans:
+        for (R, q, ctx, n_new) in step_shapes(wl, plan):
+            msr = max(msr, R)
+    L = wl.prompt_len + wl.gen_len
+    return msr, max(wl.batch * msr, wl.prompt_len, L)
+
+
+def main():
+    args = parse()
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+
+    import torch
+    import torch.distributed as dist
+    import masked_discrete_diffusion_sparse_b200 as smdm
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    m = wl.model
+    B = wl.batch
+    plans = [synth.make_plan(wl, rank * B + s) for s in range(B)]
+    prompts_np = np.stack([synth.make_prompt(wl, rank * B + s) for s in range(B)])
+    msr, max_rows = capacities(wl, plans)
+    cfg = smdm.make_config(m.n_layers, m.d_model, m.n_heads, m.d_head, m.d_ffn, m.vocab,
+                           n_reg=m.n_reg,
+                           dtype=smdm.SMDM_BF16 if m.dtype == synth.BF16 else smdm.SMDM_F32,
+                           rope_theta=m.rope_theta, rms_eps=m.rms_eps, max_batch=B,
+                           max_len=wl.prompt_len + wl.gen_len, max_step_rows=msr,
+                           max_rows=max_rows)
+    weights = device_weights(wl, wl.seed + 7919 * rank, dev)
+    model = smdm.Model(cfg, weights)
+    stream = torch.cuda.Stream(device=dev)
+
+    P, Lg = wl.prompt_len, wl.gen_len
+    d_prompts = torch.as_tensor(prompts_np.astype(np.int32), device=dev)
+    d_orders = [torch.as_tensor(p.order, device=dev) if p.order is not None else None for p in plans]
+    d_grids = torch.empty((B, Lg), dtype=torch.int32, device=dev)
+
+    def plan_dicts():
+        out = []
+        for i, p in enumerate(plans):
+            if p.kind == "order":
+                out.append(dict(kind=smdm.SMDM_PLAN_ORDER, n_steps=p.n_steps,
+                                n_per_step=list(p.n_per_step), order=d_orders[i]))
+            else:
+                out.append(dict(kind=smdm.SMDM_PLAN_SEMIAR, n_steps=p.n_steps, block=p.block,
+                                steps_per_block=p.steps_per_block, commit=p.commit))
+        return out
+
+    pd = plan_dicts()
+
+    def generate(mode=smdm.SMDM_MODE_SPARSE, prompts=d_prompts, plans_=pd, grids=d_grids):
+        model.smdm_generate(prompts, Lg, plans_, grids, mode=mode, stream=stream)
+
+    # eager sanity run + per-kernel-class profile (events on the launching stream)
+    with torch.cuda.stream(stream):
+        generate()
+        stream.synchronize()
+        assert model.smdm_device_status(stream) == 0
+        g = d_grids.cpu().numpy()
+        assert (g >= 0).all() and (g < m.vocab).all(), "incomplete generation"
+        model.smdm_profile_begin(timed=True)
+        generate()
+        prof = model.smdm_profile_end(stream)
+    launches_per_run = prof["launches"]
+
+    # capture one full run as a CUDA graph
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream, capture_error_mode="thread_local"):
+        generate()
+    torch.cuda.synchronize()
+
+    def timed(fn, n):
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(n):
+            fn()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return ev0.elapsed_time(ev1) / n
+
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        ms = timed(graph.replay, args.steps)
+    clocks = sampler.stop()
+    ms_t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    tokens_per_run = Lg * B
+    value = tokens_per_run * world / (ms_max / 1e3)
+    assert model.smdm_device_status(stream) == 0
+
+    # e2e: public API, pinned host inputs -> device, grid -> host, every run
+    e2e = None
+    if not args.no_e2e:
+        h_prompts = torch.from_numpy(prompts_np.astype(np.int32)).pin_memory()
+        h_orders = [torch.from_numpy(p.order.astype(np.int32)).pin_memory() if p.order is not None
+                    else None for p in plans]
+        h_grid = torch.empty((B, Lg), dtype=torch.int32).pin_memory()
+        e_prompts = torch.empty_like(d_prompts)
+        e_orders = [torch.empty_like(o) if o is not None else None for o in d_orders]
+        e_grids = torch.empty_like(d_grids)
+        e_plans = plan_dicts()
+        for i, p in enumerate(e_plans):
+            if "order" in p:
+                p["order"] = e_orders[i]
+        h2d = h_prompts.numel() * 4 + sum(o.numel() * 4 for o in h_orders if o is not None)
+        d2h = h_grid.numel() * 4
+
+        def e2e_run():
+            e_prompts.copy_(h_prompts, non_blocking=True)
+            for i, o in enumerate(h_orders):
+                if o is not None:
+                    e_orders[i].copy_(o, non_blocking=True)
+            model.smdm_generate(e_prompts, Lg, e_plans, e_grids, stream=stream)
+            h_grid.copy_(e_grids, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(max(1, args.warmup)):
+                e2e_run()
+            e_ms = timed(e2e_run, max(3, args.steps // 2))
+        et = torch.tensor([e_ms], device=dev)
+        if world > 1:
+            dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        e2e = {"value": tokens_per_run * world / (float(et.item()) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": float(et.item()), "path": "smdm_generate (eager launches)"}
+
+    # dense comparator: the same library's dense full-sequence MDM step, full run
+    dense = None
+    if not args.no_dense and rank == 0:
+        dgrids = torch.empty_like(d_grids)
+        with torch.cuda.stream(stream):
+            generate(mode=smdm.SMDM_MODE_DENSE, grids=dgrids)   # warm-up
+            d_ms = timed(lambda: generate(mode=smdm.SMDM_MODE_DENSE, grids=dgrids), 1)
+        dense = {"value": tokens_per_run / (d_ms / 1e3), "unit": UNIT, "ms_per_run": d_ms,
+                 "sparse_speedup": d_ms / ms}
+
+    # roofline
+    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(peaks_path):
+        pk = json.load(open(peaks_path))
+        hbm, tfl, tfl_s, peak_src = pk["hbm_gbs"], pk["bf16_tflops"], \
+            pk.get("bf16_tflops_sustained", pk["bf16_tflops"]), "measured"
+    else:
+        hbm, tfl, tfl_s, peak_src = 6650.0, 1590.0, 1400.0, "fallback"
+    gemm_cls = ["gemm_qkv", "gemm_o", "gemm_gateup", "gemm_down", "gemm_lmhead"]
+    gemm_ms = sum(prof["class_ms"][c] for c in gemm_cls)
+    gemm_n = sum(prof["class_launches"][c] for c in gemm_cls)
+    gb = sum(gemm_bytes_per_run(wl, p) for p in plans) / B if B == 1 else \
+        gemm_bytes_per_run(wl, plans[0])
+    achieved = gb / (gemm_ms / 1e3) / 1e9 if gemm_ms > 0 else None
+    costs = run_cost(wl, plans[0])
+    roof_s = sum(max(b / (hbm * 1e9), f / (tfl_s * 1e12)) for b, f in costs)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if m.dtype == synth.BF16 else "f32",
+        "data": "synthetic (seeded N(0,0.02) weights drawn on device; seeded prompts/orders)",
+        "config": {**describe(wl), "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "l2": "weights 1.69 GB >> 126 MB L2 stream from HBM every run (no flush)",
+                   "timed": "CUDA-graph replay of prefill + all sampling steps"},
+        "clocks": clocks,
+        "e2e": e2e,
+        "gpu_launches": launches_per_run * args.steps,
+        "roofline": {"bound": "hbm", "kernel": "gemm_tc_kernel (all weight GEMMs)",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": (achieved / hbm) if achieved else None, "traffic": None,
+                     "peak_source": peak_src,
+                     "gemm_ms_per_run": gemm_ms, "gemm_launches_per_run": gemm_n,
+                     "gemm_algorithmic_gb_per_run": gb / 1e9},
+        "step_roofline": {"roofline_ms_per_run": roof_s * 1e3, "measured_ms_per_run": ms,
+                          "frac": roof_s * 1e3 / ms,
+                          "peaks": {"hbm_gbs": hbm, "bf16_tflops_sustained": tfl_s}},
+        "per_class_ms_per_run": {k: round(v, 4) for k, v in prof["class_ms"].items()},
+        "per_step_ms": ms / wl.n_steps,
+        "dense": dense,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        try:
+            dt, n_dec, desc, threads = oracle_sample(wl)
+            line["cpu_baseline"] = {"value": n_dec * B / dt, "unit": UNIT, "cores": threads,
+                                    "kind": "oracle", "sample": desc, "seconds": dt}
+        except MemoryError:
+            line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

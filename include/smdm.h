@@ -197,6 +197,26 @@ smdm_status smdm_debug_rows(smdm_handle* h, int32_t* d_ids, int32_t* d_pos, int3
 /* Cache length (prompt + cached clean tokens) of a sequence slot, host bookkeeping. */
 int smdm_context_length(const smdm_handle* h, int seq);
 
+/* Kernel classes for profiling. */
+enum {
+  SMDM_K_PACK = 0, SMDM_K_NORM = 1, SMDM_K_GEMM_QKV = 2, SMDM_K_ATTN = 3, SMDM_K_GEMM_O = 4,
+  SMDM_K_GEMM_GATEUP = 5, SMDM_K_GEMM_DOWN = 6, SMDM_K_GEMM_LMHEAD = 7, SMDM_K_UNMASK = 8,
+  SMDM_K_OTHER = 9, SMDM_K_CLASSES = 10
+};
+
+typedef struct {
+  unsigned long long launches;                      /* kernels launched since profile_begin */
+  unsigned long long class_launches[SMDM_K_CLASSES];
+  double class_ms[SMDM_K_CLASSES];  /* device time per class from CUDA events recorded on the
+                                       launching stream around every launch (timed mode only) */
+} smdm_profile;
+
+/* Start counting kernel launches.  timed != 0 also records a CUDA event pair around every
+ * launch (do not enable while capturing a CUDA graph).  Resets the counters. */
+smdm_status smdm_profile_begin(smdm_handle* h, int timed);
+/* Synchronise `stream`, fill *out and stop profiling. */
+smdm_status smdm_profile_end(smdm_handle* h, smdm_profile* out, cudaStream_t stream);
+
 /* Synchronise `stream` and return the device status word (0 = no device-side error) and clear
  * it.  Returns SMDM_ETIMEOUT / SMDM_EDEVICE when a bit is set. */
 smdm_status smdm_device_status(smdm_handle* h, unsigned* h_bits, cudaStream_t stream);

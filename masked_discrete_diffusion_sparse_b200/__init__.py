@@ -32,7 +32,11 @@ STATUS_NAMES = {0: "SMDM_OK", 1: "SMDM_EINVAL", 2: "SMDM_ESHAPE", 3: "SMDM_ENOME
 EXPORTED = ["smdm_workspace_bytes", "smdm_create", "smdm_destroy", "smdm_last_error",
             "smdm_prefill", "smdm_step", "smdm_dense_step", "smdm_generate",
             "smdm_forward_stepcausal", "smdm_debug_mask", "smdm_debug_rows",
-            "smdm_context_length", "smdm_device_status"]
+            "smdm_context_length", "smdm_device_status", "smdm_profile_begin",
+            "smdm_profile_end"]
+
+K_CLASSES = ["pack", "norm", "gemm_qkv", "attn", "gemm_o", "gemm_gateup", "gemm_down",
+             "gemm_lmhead", "unmask", "other"]
 
 
 class SmdmError(RuntimeError):
@@ -70,6 +74,11 @@ class smdm_plan(ctypes.Structure):
                 ("h_n_per_step", ctypes.POINTER(ctypes.c_int32)), ("d_order", ctypes.c_void_p),
                 ("block", ctypes.c_int), ("steps_per_block", ctypes.c_int),
                 ("commit", ctypes.c_int)]
+
+
+class smdm_profile(ctypes.Structure):
+    _fields_ = [("launches", ctypes.c_ulonglong), ("class_launches", ctypes.c_ulonglong * 10),
+                ("class_ms", ctypes.c_double * 10)]
 
 
 _lib = None
@@ -112,6 +121,10 @@ def lib() -> ctypes.CDLL:
     L.smdm_context_length.restype = ctypes.c_int
     L.smdm_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint), vp]
     L.smdm_device_status.restype = st
+    L.smdm_profile_begin.argtypes = [vp, i32]
+    L.smdm_profile_begin.restype = st
+    L.smdm_profile_end.argtypes = [vp, ctypes.POINTER(smdm_profile), vp]
+    L.smdm_profile_end.restype = st
     _lib = L
     return L
 
@@ -257,6 +270,16 @@ class Model:
 
     def smdm_context_length(self, seq: int) -> int:
         return lib().smdm_context_length(self.h, seq)
+
+    def smdm_profile_begin(self, timed: bool = False):
+        self._check(lib().smdm_profile_begin(self.h, 1 if timed else 0))
+
+    def smdm_profile_end(self, stream=None) -> dict:
+        p = smdm_profile()
+        self._check(lib().smdm_profile_end(self.h, ctypes.byref(p), _stream(stream)))
+        return {"launches": int(p.launches),
+                "class_launches": {K_CLASSES[i]: int(p.class_launches[i]) for i in range(10)},
+                "class_ms": {K_CLASSES[i]: float(p.class_ms[i]) for i in range(10)}}
 
     def smdm_device_status(self, stream=None) -> int:
         bits = ctypes.c_uint(0)

@@ -151,8 +151,18 @@ struct SeqState {
 
 }  // namespace
 
+struct Profiler {
+  bool on = false, timed = false;
+  unsigned long long launches = 0;
+  unsigned long long class_launches[SMDM_K_CLASSES] = {};
+  std::vector<cudaEvent_t> ev;   // pairs
+  std::vector<int> cls;
+  size_t used = 0;
+};
+
 struct smdm_handle {
   smdm_config cfg;
+  Profiler prof;
   Layout L;
   bool bf16;
   const void* emb;
@@ -192,6 +202,36 @@ smdm_status fail(smdm_handle* h, smdm_status st, const char* fmt, ...) {
     if (e_ != cudaSuccess)                                                          \
       return fail(h, SMDM_ECUDA, "%s failed: %s", #call, cudaGetErrorString(e_)); \
   } while (0)
+
+// Launch bookkeeping: every kernel launch of the library goes through Launch{h, class, stream}.
+struct Launch {
+  smdm_handle* h;
+  cudaStream_t st;
+  Launch(smdm_handle* h_, int cls, cudaStream_t st_) : h(h_), st(st_) {
+    Profiler& p = h->prof;
+    p.launches++;
+    p.class_launches[cls]++;
+    if (p.on && p.timed) {
+      if (p.used * 2 + 2 > p.ev.size()) {
+        cudaEvent_t a, b;
+        cudaEventCreate(&a);
+        cudaEventCreate(&b);
+        p.ev.push_back(a);
+        p.ev.push_back(b);
+      }
+      p.cls.resize(p.used + 1);
+      p.cls[p.used] = cls;
+      cudaEventRecord(p.ev[p.used * 2], st);
+    }
+  }
+  ~Launch() {
+    Profiler& p = h->prof;
+    if (p.on && p.timed) {
+      cudaEventRecord(p.ev[p.used * 2 + 1], st);
+      p.used++;
+    }
+  }
+};
 
 Rows rows_at(smdm_handle* h, size_t off) {
   const size_t MR = align_up((size_t)h->cfg.max_rows, 256);
@@ -245,10 +285,11 @@ struct FwdSpec {
   float* logits;              // optional [n_logit][V]
 };
 
-smdm_status gemm(smdm_handle* h, const CUtensorMap* tmA, const CUtensorMap* tmA2, const void* W,
-                 const void* W2, void* X, int K, int n_out, int rows, int swiglu,
+smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensorMap* tmA2,
+                 const void* W, const void* W2, void* X, int K, int n_out, int rows, int swiglu,
                  const EpiParams& ep, cudaStream_t st) {
   if (rows <= 0) return SMDM_OK;
+  Launch lg(h, cls, st);
   if (h->bf16) {
     CUtensorMap tmB;
     const size_t MR = align_up((size_t)h->cfg.max_rows, 256);
@@ -289,6 +330,7 @@ smdm_status norm(smdm_handle* h, float* x, const void* gain, void* out, const in
   a.ids = ids;
   a.d = h->cfg.d_model;
   a.eps = h->cfg.rms_eps;
+  Launch lg(h, SMDM_K_NORM, st);
   if (h->bf16) CK(launch_rmsnorm<__nv_bfloat16>(a, rows, st));
   else CK(launch_rmsnorm<float>(a, rows, st));
   return SMDM_OK;
@@ -324,7 +366,7 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
     ep.row_slot = rw.slot;
     ep.row_pos = rw.pos;
     ep.rope = h->at<float2>(h->L.rope);
-    if ((s = gemm(h, h->bf16 ? &h->tm_qkv[l] : nullptr, nullptr, h->w_qkv[l], nullptr, hb, d,
+    if ((s = gemm(h, SMDM_K_GEMM_QKV, h->bf16 ? &h->tm_qkv[l] : nullptr, nullptr, h->w_qkv[l], nullptr, hb, d,
                   3 * d, R, 0, ep, st)))
       return s;
     // step-causal attention
@@ -347,6 +389,7 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
       a.cap = kv.cap;
       a.out = ao;
       a.status = h->status();
+      Launch lg(h, SMDM_K_ATTN, st);
       CK(launch_attn_tc(a, st));
     } else {
       AttnSimtArgs a{};
@@ -362,6 +405,7 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
       a.type = rw.type;
       a.label = rw.label;
       a.scale = 1.0f / sqrtf((float)c.d_head);
+      Launch lg(h, SMDM_K_ATTN, st);
       CK(launch_attn_simt<float>(static_cast<const float*>(q), static_cast<float*>(ao), kv, a, st));
     }
     // O-projection + residual
@@ -371,7 +415,7 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
     eo.n_valid = d;
     eo.x = x;
     eo.ld_x = d;
-    if ((s = gemm(h, h->bf16 ? &h->tm_o[l] : nullptr, nullptr, h->w_o[l], nullptr, ao, d, d, R,
+    if ((s = gemm(h, SMDM_K_GEMM_O, h->bf16 ? &h->tm_o[l] : nullptr, nullptr, h->w_o[l], nullptr, ao, d, d, R,
                   0, eo, st)))
       return s;
     if ((s = norm(h, x, h->mlp_norm[l], hb, nullptr, nullptr, nullptr, R, st))) return s;
@@ -382,12 +426,12 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
     eg.n_valid = c.d_ffn;
     eg.act = act;
     eg.ld_act = c.d_ffn;
-    if ((s = gemm(h, h->bf16 ? &h->tm_gate[l] : nullptr, h->bf16 ? &h->tm_up[l] : nullptr,
+    if ((s = gemm(h, SMDM_K_GEMM_GATEUP, h->bf16 ? &h->tm_gate[l] : nullptr, h->bf16 ? &h->tm_up[l] : nullptr,
                   h->w_gate[l], h->w_up[l], hb, d, c.d_ffn, R, 1, eg, st)))
       return s;
     // down + residual
     EpiParams ed = eo;
-    if ((s = gemm(h, h->bf16 ? &h->tm_down[l] : nullptr, nullptr, h->w_down[l], nullptr, act,
+    if ((s = gemm(h, SMDM_K_GEMM_DOWN, h->bf16 ? &h->tm_down[l] : nullptr, nullptr, h->w_down[l], nullptr, act,
                   c.d_ffn, d, R, 0, ed, st)))
       return s;
     if (l + 1 < c.n_layers)
@@ -405,7 +449,7 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
     el.psum = h->at<float>(h->L.psum);
     el.parg = h->at<int>(h->L.parg);
     el.n_vt = h->L.n_vt;
-    if ((s = gemm(h, h->bf16 ? &h->tm_lm : nullptr, nullptr, h->lm_head, nullptr, hq, d, c.vocab,
+    if ((s = gemm(h, SMDM_K_GEMM_LMHEAD, h->bf16 ? &h->tm_lm : nullptr, nullptr, h->lm_head, nullptr, hq, d, c.vocab,
                   f.n_logit, 0, el, st)))
       return s;
   }
@@ -565,7 +609,11 @@ smdm_status smdm_create(const smdm_config* cfg, const smdm_weights* w, void* d_w
   return SMDM_OK;
 }
 
-void smdm_destroy(smdm_handle* h) { delete h; }
+void smdm_destroy(smdm_handle* h) {
+  if (!h) return;
+  for (cudaEvent_t e : h->prof.ev) cudaEventDestroy(e);
+  delete h;
+}
 
 const char* smdm_last_error(const smdm_handle* h) { return h ? h->err.c_str() : "null handle"; }
 
@@ -583,7 +631,7 @@ smdm_status smdm_prefill(smdm_handle* h, int seq, const int32_t* d_prompt, int P
     return fail(h, SMDM_ESHAPE, "P=%d, Lgen=%d outside max_len %d", P, Lgen, h->cfg.max_len);
   if (P > h->cfg.max_rows) return fail(h, SMDM_ESHAPE, "prompt longer than max_rows");
   if (!d_grid || (P > 0 && !d_prompt)) return fail(h, SMDM_EINVAL, "null prompt or grid");
-  CK(launch_fill_i32(d_grid, Lgen, -1, st));
+  { Launch lg_(h, SMDM_K_OTHER, st); CK(launch_fill_i32(d_grid, Lgen, -1, st)); }
   if (P > 0)
     CK(cudaMemcpyAsync(h->prompt(seq), d_prompt, (size_t)P * 4, cudaMemcpyDeviceToDevice, st));
   SeqState& q = h->seq[seq];
@@ -603,7 +651,7 @@ smdm_status smdm_prefill(smdm_handle* h, int seq, const int32_t* d_prompt, int P
     a.prompt = h->prompt(seq);
     a.rows = h->rows;
     a.status = h->status();
-    CK(launch_pack_linear(a, st));
+    { Launch lg_(h, SMDM_K_PACK, st); CK(launch_pack_linear(a, st)); }
     FwdSpec f{};
     f.R = P;
     f.attn_mode = 0;
@@ -680,7 +728,7 @@ smdm_status smdm_step(smdm_handle* h, int n_seq, const smdm_step_desc* hd, float
     qbase += d.n_query;
     max_nq = std::max(max_nq, d.n_query);
   }
-  CK(launch_pack_step(pa, st));
+  { Launch lg_(h, SMDM_K_PACK, st); CK(launch_pack_step(pa, st)); }
   if ((s = forward(h, f, st))) return s;
   ua.n_vt = h->L.n_vt;
   ua.pmax = h->at<float>(h->L.pmax);
@@ -690,7 +738,7 @@ smdm_status smdm_step(smdm_handle* h, int n_seq, const smdm_step_desc* hd, float
   ua.tok_out = d_tok;
   ua.conf_out = d_conf;
   ua.status = h->status();
-  CK(launch_unmask(ua, max_nq, st));
+  { Launch lg_(h, SMDM_K_UNMASK, st); CK(launch_unmask(ua, max_nq, st)); }
   for (int i = 0; i < n_seq; ++i) {
     SeqState& q = h->seq[hd[i].seq];
     q.ctx += q.n_new;
@@ -732,7 +780,7 @@ smdm_status smdm_dense_step(smdm_handle* h, const smdm_step_desc* d, float* d_lo
   p.qpos = d->d_query_pos;
   p.grid = q.grid;
   p.newpos = h->newpos(d->seq);
-  CK(launch_pack_step(pa, st));
+  { Launch lg_(h, SMDM_K_PACK, st); CK(launch_pack_step(pa, st)); }
   LinearPackArgs a{};
   a.mode = kPackDense;
   a.n = L;
@@ -745,7 +793,7 @@ smdm_status smdm_dense_step(smdm_handle* h, const smdm_step_desc* d, float* d_lo
   a.grid = q.grid;
   a.rows = h->rows;
   a.status = h->status();
-  CK(launch_pack_linear(a, st));
+  { Launch lg_(h, SMDM_K_PACK, st); CK(launch_pack_linear(a, st)); }
   FwdSpec f{};
   f.R = L;
   f.attn_mode = 0;
@@ -775,7 +823,7 @@ smdm_status smdm_dense_step(smdm_handle* h, const smdm_step_desc* d, float* d_lo
   ua.tok_out = d_tok;
   ua.conf_out = d_conf;
   ua.status = h->status();
-  CK(launch_unmask(ua, d->n_query, st));
+  { Launch lg_(h, SMDM_K_UNMASK, st); CK(launch_unmask(ua, d->n_query, st)); }
   q.k += 1;
   return SMDM_OK;
 }
@@ -867,8 +915,8 @@ smdm_status smdm_forward_stepcausal(smdm_handle* h, const int32_t* d_ids, const 
   a.label = d_label;
   a.rows = h->rows;
   a.status = h->status();
-  CK(launch_pack_linear(a, st));
-  CK(launch_gather_rows(d_logit_rows, n_rows, h->rows.qrow, st));
+  { Launch lg_(h, SMDM_K_PACK, st); CK(launch_pack_linear(a, st)); }
+  { Launch lg_(h, SMDM_K_OTHER, st); CK(launch_gather_rows(d_logit_rows, n_rows, h->rows.qrow, st)); }
   FwdSpec f{};
   f.R = n;
   f.attn_mode = 1;
@@ -884,7 +932,7 @@ smdm_status smdm_debug_mask(smdm_handle* h, const int32_t* d_type, const int32_t
                             uint32_t* d_bitmap, cudaStream_t st) {
   if (!h) return SMDM_EINVAL;
   if (!d_type || !d_label || !d_bitmap || n < 1) return fail(h, SMDM_EINVAL, "bad arguments");
-  CK(launch_debug_mask(d_type, d_label, n, d_bitmap, st));
+  { Launch lg_(h, SMDM_K_OTHER, st); CK(launch_debug_mask(d_type, d_label, n, d_bitmap, st)); }
   return SMDM_OK;
 }
 
@@ -900,6 +948,37 @@ smdm_status smdm_debug_rows(smdm_handle* h, int32_t* d_ids, int32_t* d_pos, int3
     if (d_type) CK(cudaMemcpyAsync(d_type, h->rows.type, b, cudaMemcpyDeviceToDevice, st));
     if (d_label) CK(cudaMemcpyAsync(d_label, h->rows.label, b, cudaMemcpyDeviceToDevice, st));
   }
+  return SMDM_OK;
+}
+
+smdm_status smdm_profile_begin(smdm_handle* h, int timed) {
+  if (!h) return SMDM_EINVAL;
+  Profiler& p = h->prof;
+  p.on = true;
+  p.timed = timed != 0;
+  p.launches = 0;
+  for (int i = 0; i < SMDM_K_CLASSES; ++i) p.class_launches[i] = 0;
+  p.used = 0;
+  return SMDM_OK;
+}
+
+smdm_status smdm_profile_end(smdm_handle* h, smdm_profile* out, cudaStream_t st) {
+  if (!h || !out) return SMDM_EINVAL;
+  Profiler& p = h->prof;
+  CK(cudaStreamSynchronize(st));
+  std::memset(out, 0, sizeof(*out));
+  out->launches = p.launches;
+  for (int i = 0; i < SMDM_K_CLASSES; ++i) out->class_launches[i] = p.class_launches[i];
+  if (p.timed) {
+    for (size_t i = 0; i < p.used; ++i) {
+      float ms = 0.f;
+      CK(cudaEventElapsedTime(&ms, p.ev[2 * i], p.ev[2 * i + 1]));
+      out->class_ms[p.cls[i]] += ms;
+    }
+  }
+  p.on = false;
+  p.timed = false;
+  p.used = 0;
   return SMDM_OK;
 }
 
