@@ -217,6 +217,29 @@ smdm_status smdm_profile_begin(smdm_handle* h, int timed);
 /* Synchronise `stream`, fill *out and stop profiling. */
 smdm_status smdm_profile_end(smdm_handle* h, smdm_profile* out, cudaStream_t stream);
 
+/* Allocation-free training-form forward (no counterpart in the paper; it exists for callers
+ * that cannot allocate device memory when they need a forward — code under an allocator that
+ * is frozen after start-up, a plug-in that is only handed pointers by its host application).
+ * Same computation and arguments as smdm_forward_stepcausal, but without a handle: the caller
+ * passes the model config, the weights and the inputs/outputs, and every byte of scratch
+ * (activations, KV rows, split-K partial sums and tile counters, LM-head statistics, RoPE
+ * table) lives in one 16 MiB static device array inside the library, which every GPU that
+ * loads the library holds until the process exits.  It calls no cudaMalloc/cudaFree.
+ *  - Size limit: the scratch this call needs (a one-sequence workspace for max(n, n_rows) rows
+ *    with the config's max_len, split-K over 32 CTAs) must fit in 16 MiB; otherwise the call
+ *    returns SMDM_ESHAPE before launching anything.  A 2-layer d=256 model with a few hundred
+ *    rows fits.
+ *  - The first call on each device looks up the array's device address and sets kernel
+ *    attributes; make that first call before any stream capture.
+ *  - Every call shares the array and overwrites it (the call clears it first); calls that
+ *    overlap on the GPU — on different streams, or from different host threads — race.
+ *    Serialise them.  Device-side status bits of this path are not reported. */
+smdm_status smdm_forward_stepcausal_noalloc(const smdm_config* cfg, const smdm_weights* w,
+                                            const int32_t* d_ids, const int32_t* d_pos,
+                                            const int32_t* d_type, const int32_t* d_label, int n,
+                                            const int32_t* d_logit_rows, int n_rows,
+                                            float* d_logits, cudaStream_t stream);
+
 /* Synchronise `stream` and return the device status word (0 = no device-side error) and clear
  * it.  Returns SMDM_ETIMEOUT / SMDM_EDEVICE when a bit is set. */
 smdm_status smdm_device_status(smdm_handle* h, unsigned* h_bits, cudaStream_t stream);

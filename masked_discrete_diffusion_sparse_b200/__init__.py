@@ -33,7 +33,7 @@ EXPORTED = ["smdm_workspace_bytes", "smdm_create", "smdm_destroy", "smdm_last_er
             "smdm_prefill", "smdm_step", "smdm_dense_step", "smdm_generate",
             "smdm_forward_stepcausal", "smdm_debug_mask", "smdm_debug_rows",
             "smdm_context_length", "smdm_device_status", "smdm_profile_begin",
-            "smdm_profile_end"]
+            "smdm_profile_end", "smdm_forward_stepcausal_noalloc"]
 
 K_CLASSES = ["pack", "norm", "gemm_qkv", "attn", "gemm_o", "gemm_gateup", "gemm_down",
              "gemm_lmhead", "unmask", "other"]
@@ -125,6 +125,10 @@ def lib() -> ctypes.CDLL:
     L.smdm_profile_begin.restype = st
     L.smdm_profile_end.argtypes = [vp, ctypes.POINTER(smdm_profile), vp]
     L.smdm_profile_end.restype = st
+    L.smdm_forward_stepcausal_noalloc.argtypes = [ctypes.POINTER(smdm_config),
+                                                  ctypes.POINTER(smdm_weights), vp, vp, vp, vp,
+                                                  i32, vp, i32, vp, vp]
+    L.smdm_forward_stepcausal_noalloc.restype = st
     _lib = L
     return L
 
@@ -285,6 +289,35 @@ class Model:
         bits = ctypes.c_uint(0)
         self._check(lib().smdm_device_status(self.h, ctypes.byref(bits), _stream(stream)))
         return bits.value
+
+
+def smdm_forward_stepcausal_noalloc(cfg: smdm_config, weights: dict, ids, pos, types, labels,
+                                    logit_rows, logits, stream=None):
+    """Training-form forward without a handle and without any device allocation.
+
+    For callers that may not allocate device memory at the point of the call (a frozen
+    allocator, a plug-in handed only pointers by its host program): all scratch lives in a
+    16 MiB array built into the library.  Same arguments and result as
+    Model.smdm_forward_stepcausal, plus the config and the weights dict.  Shapes whose scratch
+    does not fit raise SmdmError(SMDM_ESHAPE).  Calls share that array: do not overlap them on
+    the GPU.  Make the first call on a device outside CUDA-graph capture (it looks up the
+    array's device address).
+    """
+    keep = []
+    arr = {}
+    for k in ("attn_norm", "w_qkv", "w_o", "mlp_norm", "w_gate", "w_up", "w_down"):
+        a = (ctypes.c_void_p * cfg.n_layers)(*[t.data_ptr() for t in weights[k]])
+        keep.append(a)
+        arr[k] = ctypes.cast(a, _PP)
+    w = smdm_weights(weights["emb"].data_ptr(), weights["final_norm"].data_ptr(),
+                     weights["lm_head"].data_ptr(), arr["attn_norm"], arr["w_qkv"], arr["w_o"],
+                     arr["mlp_norm"], arr["w_gate"], arr["w_up"], arr["w_down"])
+    s = lib().smdm_forward_stepcausal_noalloc(
+        ctypes.byref(cfg), ctypes.byref(w), _ptr(_i32(ids)), _ptr(_i32(pos)), _ptr(_i32(types)),
+        _ptr(_i32(labels)), ids.numel(), _ptr(_i32(logit_rows)), logit_rows.numel(),
+        _ptr(logits), _stream(stream))
+    if s != SMDM_OK:
+        raise SmdmError(s, "smdm_forward_stepcausal_noalloc failed")
 
 
 def make_config(n_layers, d_model, n_heads, d_head, d_ffn, vocab, n_reg=64, dtype=SMDM_BF16,

@@ -996,3 +996,131 @@ smdm_status smdm_device_status(smdm_handle* h, unsigned* h_bits, cudaStream_t st
 }
 
 }  // extern "C"
+
+// ==============================================================================================
+// Allocation-free training-form forward.
+//
+// Some callers cannot allocate device memory at the point where they need a forward pass: code
+// running under an allocator that forbids new device allocations after start-up, a plug-in
+// that only receives pointers from its host application, or a caller that is recording into a
+// stream while a memory pool is frozen.  They cannot create a handle (its workspace is caller
+// memory), so this entry point keeps all of its scratch — activations, the KV rows of the
+// forward, the split-K partial sums and tile counters of the GEMMs, the LM-head statistics and
+// the RoPE table — in one statically sized device array that the library carries with it.
+// ==============================================================================================
+
+#define SMDM_NOALLOC_SCRATCH_BYTES (16u << 20)   /* 16 MiB, held by every GPU that loads the library */
+#define SMDM_NOALLOC_GEMM_CTAS 32                /* split-K width; bounds the partial-sum scratch */
+#define SMDM_NOALLOC_MAX_DEVICES 64
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SMDM_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+struct NoAllocDevice {
+  bool ready = false;
+  void* scratch = nullptr;          // device address of g_noalloc_scratch on this device
+  smdm_handle* handle = nullptr;    // host-side bookkeeping reused by every call
+};
+NoAllocDevice g_noalloc[SMDM_NOALLOC_MAX_DEVICES];
+
+__global__ void noalloc_rope_kernel(float2* tab, int max_pos, int half, double theta, int d_head) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)max_pos * half) return;
+  const int p = (int)(i / half), j = (int)(i % half);
+  const double ang = (double)p * pow(theta, -2.0 * j / d_head);
+  double s, c;
+  sincos(ang, &s, &c);
+  tab[i] = make_float2((float)c, (float)s);
+}
+
+}  // namespace
+
+extern "C" smdm_status smdm_forward_stepcausal_noalloc(
+    const smdm_config* cfg, const smdm_weights* w, const int32_t* d_ids, const int32_t* d_pos,
+    const int32_t* d_type, const int32_t* d_label, int n, const int32_t* d_logit_rows,
+    int n_rows, float* d_logits, cudaStream_t st) {
+  if (!config_ok(cfg, nullptr)) return SMDM_ESHAPE;
+  if (!w || !w->emb || !w->final_norm || !w->lm_head || !w->attn_norm || !w->w_qkv || !w->w_o ||
+      !w->mlp_norm || !w->w_gate || !w->w_up || !w->w_down)
+    return SMDM_EINVAL;
+  if (!d_ids || !d_pos || !d_type || !d_label || !d_logit_rows || !d_logits || n < 1 ||
+      n_rows < 1)
+    return SMDM_EINVAL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= SMDM_NOALLOC_MAX_DEVICES)
+    return SMDM_ECUDA;
+  NoAllocDevice& D = g_noalloc[dev];
+  if (!D.ready) {
+    // Once per device, with that device current: the host-side name of the array is only a
+    // stand-in, so fetch its real device address.
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SMDM_ECUDA;
+    if (gemm_tc_set_smem_attr() != cudaSuccess || attn_tc_set_smem_attr() != cudaSuccess)
+      return SMDM_ECUDA;
+    D.scratch = p;
+    D.handle = new smdm_handle();
+    D.ready = true;
+  }
+  // The scratch is laid out like a one-sequence handle sized for exactly this call.
+  smdm_config vc = *cfg;
+  vc.max_batch = 1;
+  vc.max_step_rows = 1;
+  vc.max_rows = std::max(n, n_rows);
+  const Layout L = make_layout(&vc, SMDM_NOALLOC_GEMM_CTAS);
+  if (L.total > SMDM_NOALLOC_SCRATCH_BYTES) return SMDM_ESHAPE;
+  smdm_handle* h = D.handle;
+  h->cfg = vc;
+  h->L = L;
+  h->bf16 = vc.dtype == SMDM_BF16;
+  h->ws = static_cast<uint8_t*>(D.scratch);
+  h->emb = w->emb;
+  h->final_norm = w->final_norm;
+  h->lm_head = w->lm_head;
+  const int nl = vc.n_layers;
+  h->attn_norm.assign(w->attn_norm, w->attn_norm + nl);
+  h->w_qkv.assign(w->w_qkv, w->w_qkv + nl);
+  h->w_o.assign(w->w_o, w->w_o + nl);
+  h->mlp_norm.assign(w->mlp_norm, w->mlp_norm + nl);
+  h->w_gate.assign(w->w_gate, w->w_gate + nl);
+  h->w_up.assign(w->w_up, w->w_up + nl);
+  h->w_down.assign(w->w_down, w->w_down + nl);
+  h->rows = rows_at(h, L.rows);
+  h->aux = rows_at(h, L.aux);
+  h->err.clear();
+  // Every call starts from zero: tile counters, status word and the KV rows.
+  if (cudaMemsetAsync(D.scratch, 0, L.total, st) != cudaSuccess) return SMDM_ECUDA;
+  {
+    const int half = vc.d_head / 2;
+    const long long cnt = (long long)L.max_pos * half;
+    noalloc_rope_kernel<<<(unsigned)((cnt + 255) / 256), 256, 0, st>>>(
+        h->at<float2>(L.rope), L.max_pos, half, (double)vc.rope_theta, vc.d_head);
+    if (cudaGetLastError() != cudaSuccess) return SMDM_ECUDA;
+  }
+  if (h->bf16) {
+    const int d = vc.d_model, f = vc.d_ffn, H = vc.n_heads, dh = vc.d_head;
+    bool ok = true;
+    h->tm_qkv.resize(nl);
+    h->tm_o.resize(nl);
+    h->tm_gate.resize(nl);
+    h->tm_up.resize(nl);
+    h->tm_down.resize(nl);
+    for (int l = 0; l < nl; ++l) {
+      ok &= encode_2d(&h->tm_qkv[l], w->w_qkv[l], d, 3 * d, (uint64_t)d * 2, 64, 128);
+      ok &= encode_2d(&h->tm_o[l], w->w_o[l], d, d, (uint64_t)d * 2, 64, 128);
+      ok &= encode_2d(&h->tm_gate[l], w->w_gate[l], d, f, (uint64_t)d * 2, 64, 64);
+      ok &= encode_2d(&h->tm_up[l], w->w_up[l], d, f, (uint64_t)d * 2, 64, 64);
+      ok &= encode_2d(&h->tm_down[l], w->w_down[l], f, d, (uint64_t)f * 2, 64, 128);
+    }
+    ok &= encode_2d(&h->tm_lm, w->lm_head, d, vc.vocab, (uint64_t)d * 2, 64, 128);
+    const size_t MR = align_up((size_t)vc.max_rows, 256);
+    ok &= encode_2d(&h->tm_kscr, h->at<uint8_t>(L.kscr), dh, (uint64_t)H * MR, (uint64_t)dh * 2,
+                    64, 128);
+    ok &= encode_2d(&h->tm_vscr, h->at<uint8_t>(L.vscr), dh, (uint64_t)H * MR, (uint64_t)dh * 2,
+                    64, 128);
+    ok &= encode_2d(&h->tm_q, h->at<uint8_t>(L.q), d, MR, (uint64_t)d * 2, 64, 128);
+    if (!ok) return SMDM_ECUDA;
+  }
+  return smdm_forward_stepcausal(h, d_ids, d_pos, d_type, d_label, n, d_logit_rows, n_rows,
+                                 d_logits, st);
+}
