@@ -51,11 +51,42 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
   return r == CUDA_SUCCESS;
 }
 
+// Rotary-interleaved view of W_qkv [3d][d] for the GEMM's A tiles: a 128-row tile is loaded so
+// that A-tile row 2i holds weight row i of the first half of a head and row 2i + 1 the matching
+// row of the second half (the RoPE partner), putting the two on adjacent TMEM lanes.
+//   d_head 128: dims {d, 2 (half, 64 rows), 64 (i, 1 row), 3d/128 (tile, 128 rows)}
+//   d_head  64: dims {d, 2 (half, 32 rows), 32 (i, 1 row), 2 (head in tile, 64 rows), tiles}
+bool encode_qkv_interleaved(CUtensorMap* m, const void* w, uint64_t d, int d_head) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const uint64_t rb = d * 2;   // bytes per weight row
+  const uint64_t tiles = 3 * d / 128;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r;
+  if (d_head == 128) {
+    cuuint64_t dims[4] = {d, 2, 64, tiles};
+    cuuint64_t strides[3] = {64 * rb, rb, 128 * rb};
+    cuuint32_t box[4] = {64, 2, 64, 1};
+    r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(w), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    cuuint64_t dims[5] = {d, 2, 32, 2, tiles};
+    cuuint64_t strides[4] = {32 * rb, rb, 64 * rb, 128 * rb};
+    cuuint32_t box[5] = {64, 2, 32, 2, 1};
+    r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(w), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
+  return r == CUDA_SUCCESS;
+}
+
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
   size_t kc, vc, kscr, vscr, x, h, q, ao, act, hq, pmax, psum, parg, rows, rope, partial,
-      counters, status, newpos, prompts, aux, total;
+      counters, status, newpos, prompts, aux, attn_part, total;
+  size_t attn_part_bytes;
   int cap, max_pos, n_vt, rt_max, max_tiles, n_sms;
   size_t partial_bytes;
 };
@@ -71,6 +102,7 @@ bool config_ok(const smdm_config* c, std::string* why) {
     return fail("non-positive model dimension");
   if (c->n_heads * c->d_head != c->d_model) return fail("n_heads * d_head != d_model");
   if (c->d_head % 2) return fail("d_head must be even (rotary pairs)");
+  if (c->d_model > 8192) return fail("d_model > 8192 is not supported");
   if (c->max_batch < 1 || c->max_batch > SMDM_MAX_BATCH) return fail("max_batch out of range");
   if (c->max_len < 1 || c->max_step_rows < 1 || c->max_rows < 1) return fail("bad capacity");
   if (c->dtype == SMDM_BF16) {
@@ -123,7 +155,7 @@ Layout make_layout(const smdm_config* c, int n_sms) {
   L.rows = take(9 * MR * 4);
   L.aux = take(9 * MR * 4);
   L.rope = take((size_t)L.max_pos * (dh / 2) * 8);
-  L.rt_max = c->max_rows > 256 ? 512 : (int)align_up(c->max_rows, 16);
+  L.rt_max = c->max_rows > 256 ? 512 : (int)align_up(c->max_rows, 32);
   L.partial_bytes = (size_t)n_sms * 2 * L.rt_max * 128 * 4;
   L.partial = take(L.partial_bytes);
   int max_nt = 3 * c->d_model / 128 + 1;
@@ -135,6 +167,10 @@ Layout make_layout(const smdm_config* c, int n_sms) {
   L.status = take(256);
   L.newpos = take((size_t)c->max_batch * c->max_step_rows * 4);
   L.prompts = take((size_t)c->max_batch * c->max_len * 4);
+  // split-KV partials for up to 16 key splits of a sampling step's rows
+  const size_t step_rows = std::min((size_t)c->max_rows, (size_t)c->max_batch * c->max_step_rows);
+  L.attn_part_bytes = 16 * step_rows * ((size_t)d * 4 + H * 8);
+  L.attn_part = take(L.attn_part_bytes);
   L.total = off + 1024;
   return L;
 }
@@ -287,7 +323,7 @@ struct FwdSpec {
 
 smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensorMap* tmA2,
                  const void* W, const void* W2, void* X, int K, int n_out, int rows, int swiglu,
-                 const EpiParams& ep, cudaStream_t st) {
+                 const EpiParams& ep, cudaStream_t st, int a_interleave = 0) {
   if (rows <= 0) return SMDM_OK;
   Launch lg(h, cls, st);
   if (h->bf16) {
@@ -304,6 +340,7 @@ smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensor
     c.rows = rows;
     c.row0 = 0;
     c.swiglu = swiglu;
+    c.a_interleave = a_interleave;
     c.num_ctas = h->L.n_sms;
     c.partial = h->at<float>(h->L.partial);
     c.partial_bytes = h->L.partial_bytes;
@@ -367,7 +404,7 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
     ep.row_pos = rw.pos;
     ep.rope = h->at<float2>(h->L.rope);
     if ((s = gemm(h, SMDM_K_GEMM_QKV, h->bf16 ? &h->tm_qkv[l] : nullptr, nullptr, h->w_qkv[l], nullptr, hb, d,
-                  3 * d, R, 0, ep, st)))
+                  3 * d, R, 0, ep, st, c.d_head)))
       return s;
     // step-causal attention
     if (h->bf16) {
@@ -389,6 +426,10 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
       a.cap = kv.cap;
       a.out = ao;
       a.status = h->status();
+      a.part_o = h->at<float>(h->L.attn_part);
+      a.part_bytes = h->L.attn_part_bytes;
+      a.num_sms = h->L.n_sms;
+      a.rows_total = R;
       Launch lg(h, SMDM_K_ATTN, st);
       CK(launch_attn_tc(a, st));
     } else {
@@ -578,7 +619,7 @@ smdm_status smdm_create(const smdm_config* cfg, const smdm_weights* w, void* d_w
     h->tm_up.resize(nl);
     h->tm_down.resize(nl);
     for (int l = 0; l < nl; ++l) {
-      ok &= encode_2d(&h->tm_qkv[l], w->w_qkv[l], d, 3 * d, (uint64_t)d * 2, 64, 128);
+      ok &= encode_qkv_interleaved(&h->tm_qkv[l], w->w_qkv[l], d, dh);
       ok &= encode_2d(&h->tm_o[l], w->w_o[l], d, d, (uint64_t)d * 2, 64, 128);
       ok &= encode_2d(&h->tm_gate[l], w->w_gate[l], d, f, (uint64_t)d * 2, 64, 64);
       ok &= encode_2d(&h->tm_up[l], w->w_up[l], d, f, (uint64_t)d * 2, 64, 64);
@@ -1106,7 +1147,7 @@ extern "C" smdm_status smdm_forward_stepcausal_noalloc(
     h->tm_up.resize(nl);
     h->tm_down.resize(nl);
     for (int l = 0; l < nl; ++l) {
-      ok &= encode_2d(&h->tm_qkv[l], w->w_qkv[l], d, 3 * d, (uint64_t)d * 2, 64, 128);
+      ok &= encode_qkv_interleaved(&h->tm_qkv[l], w->w_qkv[l], d, dh);
       ok &= encode_2d(&h->tm_o[l], w->w_o[l], d, d, (uint64_t)d * 2, 64, 128);
       ok &= encode_2d(&h->tm_gate[l], w->w_gate[l], d, f, (uint64_t)d * 2, 64, 64);
       ok &= encode_2d(&h->tm_up[l], w->w_up[l], d, f, (uint64_t)d * 2, 64, 64);

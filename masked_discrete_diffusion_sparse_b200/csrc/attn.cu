@@ -15,6 +15,8 @@
 // only moved (and O rescaled) when it grows by more than 2^8, so most tiles skip the rescale;
 // the result is exact because numerator and denominator share the reference maximum.
 // fp32 path: one warp per (row, head), SIMT.
+#include <algorithm>
+
 #include "attn.h"
 
 namespace smdm {
@@ -36,6 +38,10 @@ struct AttnDev {
   int q_off, k_off, v_off, p_off, bar_off, stage_bytes;
   void* out;                      // [rows][d_model] bf16
   uint32_t* status;
+  int nsplit;                     // key splits per query tile
+  int rows_total;
+  float* part_o;                  // [nsplit][rows_total][d_model]
+  float* part_ml;                 // [nsplit][rows_total][H][2]
 };
 
 SMDM_DEV void p_store_swizzled(uint8_t* P, int row, int key8, uint4 val) {
@@ -72,7 +78,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int blk = blockIdx.x, h = blockIdx.y;
+  const int blk = blockIdx.x / a.nsplit, split = blockIdx.x % a.nsplit, h = blockIdx.y;
   int si = 0;
   while (si + 1 < a.n_seg && a.seg[si + 1].tile0 <= blk) ++si;
   const AttnSeg sg = a.seg[si];
@@ -80,8 +86,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int qrow0 = sg.row0 + tile * 128;            // first forward row of this tile
   const int nq = min(128, sg.rows - tile * 128);     // valid query rows
   const int nkeys = sg.nkeys;
-  const int nkv = (nkeys + 127) / 128;
+  const int nkv_all = (nkeys + 127) / 128;
+  const int j0 = split * nkv_all / a.nsplit, j1 = (split + 1) * nkv_all / a.nsplit;
+  const int nkv = j1 - j0;                           // key tiles of this split
   const int dh = a.dh;
+  if (nkv == 0) {
+    // empty split: contribute nothing to the combine
+    for (int r = threadIdx.x; r < nq; r += blockDim.x) {
+      float* ml = a.part_ml + (((size_t)split * a.rows_total + qrow0 + r) * a.H + h) * 2;
+      ml[0] = -INFINITY;
+      ml[1] = 0.f;
+    }
+    return;
+  }
   const int nsub = dh / 64;                          // 64-wide chunks of the head dim
   const long long cache_base = (long long)sg.seq * a.cache_rows_per_seq +
                                ((long long)a.layer * a.H + h) * a.cap;
@@ -124,7 +141,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!mbar_wait(&kv_empty[stage], phase ^ 1, abort_flag, a.status)) break;
         uint8_t* Ks = smem + a.k_off + stage * a.stage_bytes;
         uint8_t* Vs = smem + a.v_off + stage * a.stage_bytes;
-        const int y = (int)(cache_base + (long long)j * 128);
+        const int y = (int)(cache_base + (long long)(j0 + j) * 128);
         mbar_arrive_expect_tx(&k_full[stage], 128 * dh * 2);
         for (int c = 0; c < nsub; ++c) tma_load_2d(Ks + c * 16384, &tmK, &k_full[stage], c * 64, y, pol_kv);
         mbar_arrive_expect_tx(&v_full[stage], 128 * dh * 2);
@@ -189,24 +206,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       else { tq = a.type[row]; lq = a.label[row]; kv_lim = nkeys; }
     }
     float m_ref = -INFINITY, l = 0.f;
+    const bool warp_any = __any_sync(0xffffffffu, valid);
     for (int j = 0; j < nkv; ++j) {
       const int b = j & 1;
       if (!mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag, a.status)) break;
       tc_fence_after();
       float s[128];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) tmem_ld16(tbase + lane_off + b * 128 + c * 16, s + c * 16);
+      if (warp_any) {
+        tmem_ld64(tbase + lane_off + b * 128, s);
+        tmem_ld64(tbase + lane_off + b * 128 + 64, s + 64);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[b]);
-      const int key0 = j * 128;
+      if (!warp_any) {
+        // no valid query row in this warp: keep the barrier protocol, skip the math
+        if (j >= 1 && !mbar_wait(pv_done, (j - 1) & 1, abort_flag, a.status)) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+        continue;
+      }
+      const int key0 = (j0 + j) * 128;
       float mx = -INFINITY;
+      // visibility of the 128 keys as four 32-bit masks (registers only, no local arrays)
+      uint32_t mw[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int kb = key0 + w * 32;
+        uint32_t bits;
+        if (a.mode == 0) {
+          const int n_ok = min(max(kv_lim - kb, 0), 32);
+          bits = n_ok == 32 ? 0xffffffffu : ((1u << n_ok) - 1u);
+        } else {
+          bits = 0;
+          for (int b = 0; b < 32; ++b) {
+            const int key = kb + b;
+            if (key < kv_lim && step_causal_allowed(tq, lq, a.type[key], a.label[key]))
+              bits |= 1u << b;
+          }
+        }
+        mw[w] = bits;
+      }
 #pragma unroll
       for (int c = 0; c < 128; ++c) {
-        const int key = key0 + c;
-        bool ok = valid && key < kv_lim;
-        if (ok && a.mode == 1) ok = step_causal_allowed(tq, lq, a.type[key], a.label[key]);
-        s[c] = ok ? s[c] * a.scale_log2 : -INFINITY;
+        s[c] = ((mw[c >> 5] >> (c & 31)) & 1u) ? s[c] * a.scale_log2 : -INFINITY;
         mx = fmaxf(mx, s[c]);
       }
       float alpha = 1.f;
@@ -249,26 +292,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    // Final: O / l
+    // Final: O / l (one split), or the unnormalised partial for the combine pass.
     if (nkv > 0 && mbar_wait(pv_done, (nkv - 1) & 1, abort_flag, a.status)) {
       tc_fence_after();
-      const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (size_t)row * a.d_model + h * dh;
-      for (int c = 0; c < dh / 16; ++c) {
-        float o[16];
-        tmem_ld16(t_o + lane_off + c * 16, o);
+      if (a.nsplit == 1) {
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+        __nv_bfloat16* out =
+            reinterpret_cast<__nv_bfloat16*>(a.out) + (size_t)row * a.d_model + h * dh;
+        for (int c = 0; c < dh / 16; ++c) {
+          float o[16];
+          tmem_ld16(t_o + lane_off + c * 16, o);
+          if (valid) {
+            uint4 w0, w1;
+            w0.x = pack_bf16x2(o[0] * inv, o[1] * inv);
+            w0.y = pack_bf16x2(o[2] * inv, o[3] * inv);
+            w0.z = pack_bf16x2(o[4] * inv, o[5] * inv);
+            w0.w = pack_bf16x2(o[6] * inv, o[7] * inv);
+            w1.x = pack_bf16x2(o[8] * inv, o[9] * inv);
+            w1.y = pack_bf16x2(o[10] * inv, o[11] * inv);
+            w1.z = pack_bf16x2(o[12] * inv, o[13] * inv);
+            w1.w = pack_bf16x2(o[14] * inv, o[15] * inv);
+            reinterpret_cast<uint4*>(out + c * 16)[0] = w0;
+            reinterpret_cast<uint4*>(out + c * 16)[1] = w1;
+          }
+        }
+      } else {
+        float* po = a.part_o + ((size_t)split * a.rows_total + row) * a.d_model + h * dh;
+        for (int c = 0; c < dh / 16; ++c) {
+          float o[16];
+          tmem_ld16(t_o + lane_off + c * 16, o);
+          if (valid) {
+#pragma unroll
+            for (int t = 0; t < 16; t += 4)
+              *reinterpret_cast<float4*>(po + c * 16 + t) = make_float4(o[t], o[t + 1], o[t + 2], o[t + 3]);
+          }
+        }
         if (valid) {
-          uint4 w0, w1;
-          w0.x = pack_bf16x2(o[0] * inv, o[1] * inv);
-          w0.y = pack_bf16x2(o[2] * inv, o[3] * inv);
-          w0.z = pack_bf16x2(o[4] * inv, o[5] * inv);
-          w0.w = pack_bf16x2(o[6] * inv, o[7] * inv);
-          w1.x = pack_bf16x2(o[8] * inv, o[9] * inv);
-          w1.y = pack_bf16x2(o[10] * inv, o[11] * inv);
-          w1.z = pack_bf16x2(o[12] * inv, o[13] * inv);
-          w1.w = pack_bf16x2(o[14] * inv, o[15] * inv);
-          reinterpret_cast<uint4*>(out + c * 16)[0] = w0;
-          reinterpret_cast<uint4*>(out + c * 16)[1] = w1;
+          float* ml = a.part_ml + (((size_t)split * a.rows_total + row) * a.H + h) * 2;
+          ml[0] = m_ref;
+          ml[1] = l;
         }
       }
     }
@@ -279,6 +341,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
+}
+
+// Merge the key splits: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.  One warp per
+// (row, head).
+__global__ void attn_combine_kernel(const float* __restrict__ part_o,
+                                    const float* __restrict__ part_ml, int nsplit, int rows,
+                                    int H, int dh, int d_model, __nv_bfloat16* __restrict__ out) {
+  const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= rows * H) return;
+  const int row = w / H, h = w % H;
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s)
+    M = fmaxf(M, part_ml[(((size_t)s * rows + row) * H + h) * 2]);
+  float den = 0.f;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const int per = dh / 32;
+  for (int s = 0; s < nsplit; ++s) {
+    const float* ml = part_ml + (((size_t)s * rows + row) * H + h) * 2;
+    const float m = ml[0];
+    if (m == -INFINITY) continue;
+    const float wgt = exp2f(m - M);
+    den += wgt * ml[1];
+    const float* po = part_o + ((size_t)s * rows + row) * d_model + h * dh;
+    for (int t = 0; t < per; ++t) acc[t] += wgt * po[lane * per + t];
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  for (int t = 0; t < per; ++t)
+    out[(size_t)row * d_model + h * dh + lane * per + t] = __float2bfloat16_rn(acc[t] * inv);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -350,6 +441,31 @@ cudaError_t attn_tc_set_smem_attr() {
                               227 * 1024);
 }
 
+int attn_tc_splits(const AttnCall& c) {
+  int qt = 0, nkv = 1;
+  for (int s = 0; s < c.n_seg; ++s) {
+    qt += (c.seg[s].rows + 127) / 128;
+    nkv = std::max(nkv, (c.seg[s].nkeys + 127) / 128);
+  }
+  const long long base = (long long)qt * c.H;
+  const int sms = c.num_sms > 0 ? c.num_sms : 148;
+  const size_t per_split = (size_t)c.rows_total * ((size_t)c.d_model * 4 + (size_t)c.H * 8);
+  int best = 1;
+  double best_cost = 1e30;
+  for (int s = 1; s <= 16; ++s) {
+    if (s > 1 && (s * 2 > nkv || (size_t)s * per_split > c.part_bytes || !c.part_o)) break;
+    // one CTA per SM: cost ~ waves x (key tiles per split + fixed prologue/epilogue)
+    const long long ctas = base * s;
+    const double waves = (double)((ctas + sms - 1) / sms);
+    const double cost = waves * ((nkv + s - 1) / s + 2.0) + (s > 1 ? 0.5 : 0.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
 cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t stream) {
   AttnDev d{};
   d.mode = c.mode;
@@ -374,9 +490,19 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t stream) {
     nb += (c.seg[s].rows + 127) / 128;
   }
   if (nb == 0) return cudaSuccess;
+  d.nsplit = attn_tc_splits(c);
+  d.rows_total = c.rows_total;
+  d.part_o = c.part_o;
+  d.part_ml = c.part_o ? c.part_o + (size_t)d.nsplit * c.rows_total * c.d_model : nullptr;
   const int smem = attn_layout(c.dh, d);
-  dim3 grid(nb, c.H);
+  dim3 grid(nb * d.nsplit, c.H);
   attn_tc_kernel<<<grid, kAttnThreads, smem, stream>>>(*c.tmQ, *c.tmK, *c.tmV, d);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || d.nsplit == 1) return e;
+  const long long warps = (long long)c.rows_total * c.H;
+  attn_combine_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, stream>>>(
+      d.part_o, d.part_ml, d.nsplit, c.rows_total, c.H, c.dh, c.d_model,
+      reinterpret_cast<__nv_bfloat16*>(c.out));
   return cudaGetLastError();
 }
 

@@ -28,6 +28,12 @@ struct AttnCall {
   int cap;
   void* out;                // [rows][d_model] bf16
   uint32_t* status;
+  // split-KV: partial results of `nsplit` key ranges, merged by a combine kernel
+  float* part_o;            // [nsplit][rows][d_model] fp32 (unnormalised)
+  float* part_ml;           // [nsplit][rows][H][2] (reference max in the exp2 domain, sum)
+  size_t part_bytes;        // capacity of part_o + part_ml
+  int num_sms;
+  int rows_total;
 };
 
 struct AttnSimtArgs {
@@ -42,6 +48,8 @@ struct AttnSimtArgs {
 };
 
 cudaError_t attn_tc_set_smem_attr();
+// Number of key splits the launcher will use for this call (1 = no combine pass).
+int attn_tc_splits(const AttnCall& c);
 cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t stream);
 template <typename T>
 cudaError_t launch_attn_simt(const T* q, T* out, const KVAddr& kv, const AttnSimtArgs& a,

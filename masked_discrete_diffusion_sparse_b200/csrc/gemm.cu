@@ -17,12 +17,14 @@ namespace smdm {
 
 constexpr int kGemmThreads = 192;
 constexpr int kATileBytes = 128 * 128;   // 128 rows x 64 bf16
+constexpr int kRing = 16;                // max landing slots (16 KB each) for split-K partials
 
 struct SmemLayout {
   int stage_bytes, a_bytes, b_bytes;
   int nstages;
   int stage_off;   // after 1024 alignment
-  int staging_off; // 2 x 16 x 128 floats
+  int staging_off; // 2 x 32 x 128 floats
+  int meta_off;    // 512 positions + 512 cache offsets
   int bar_off;
   int total;       // bytes of dynamic smem requested (incl. alignment slack)
 };
@@ -32,12 +34,15 @@ static SmemLayout gemm_smem_layout(int RT, int max_stages) {
   L.a_bytes = kATileBytes;
   L.b_bytes = RT * 128;
   L.stage_bytes = L.a_bytes + L.b_bytes;
-  const int budget = 227 * 1024 - 1024 /*align*/ - 2 * 16 * 128 * 4 - 512 /*barriers*/;
+  const int budget = 227 * 1024 - 1024 /*align*/ - 2 * 32 * 128 * 4 - 6144 /*meta*/ - 512;
+  // (the two 16 KB staging buffers serve the split-K partial bulk copies and the epilogues
+  //  that combine lanes)
   L.nstages = budget / L.stage_bytes;
   if (L.nstages > max_stages) L.nstages = max_stages;
   L.stage_off = 0;
   L.staging_off = L.nstages * L.stage_bytes;
-  L.bar_off = L.staging_off + 2 * 16 * 128 * 4;
+  L.meta_off = L.staging_off + 2 * 32 * 128 * 4;
+  L.bar_off = L.meta_off + 6144;
   L.total = L.bar_off + 512 + 1024;
   return L;
 }
@@ -51,14 +56,15 @@ struct GemmDev {
   int row0;        // first activation row (TMA y offset)
   long long units; // n_tiles * row_blocks * KC
   int swiglu;
-  int nstages, stage_bytes, staging_off, bar_off;
+  int a_mode;      // 0: 2-D box {64,128}; 1: SwiGLU gate+up boxes {64,64};
+                   // 2: 4-D rotary interleave (d_head 128); 3: 5-D rotary interleave (d_head 64)
+  int RTp;         // partial-sum row stride (RT rounded up to 32)
+  int nstages, stage_bytes, staging_off, meta_off, bar_off;
   int n_acc, tmem_cols;
   float* partial;
   unsigned* counters;
   uint32_t* status;
 };
-
-SMDM_DEV bool from_tmem_release(bool full_tile, bool additive) { return full_tile || additive; }
 
 SMDM_DEV long long cta_start(long long g, long long U, long long G) { return g * U / G; }
 // CTA whose unit range contains unit u (inverse of cta_start).
@@ -71,13 +77,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  float(*staging)[16][128] = reinterpret_cast<float(*)[16][128]>(smem + g.staging_off);
+  float(*staging)[32][128] = reinterpret_cast<float(*)[32][128]>(smem + g.staging_off);
+  int* meta_pos = reinterpret_cast<int*>(smem + g.meta_off);
+  long long* meta_kv = reinterpret_cast<long long*>(smem + g.meta_off + 2048);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + g.bar_off);
   uint64_t* full = bars;
   uint64_t* empty = bars + g.nstages;
   uint64_t* acc_full = bars + 2 * g.nstages;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* io_bar = acc_empty + 2;   // [2] partial bulk loads (staging buffers)
+  uint64_t* ring_bar = io_bar + 2;    // [kRing] partial bulk loads landing in the idle stages
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ring_bar + kRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_holder + 2);
 
@@ -90,7 +100,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 4);
+      mbar_init(&io_bar[a], 1);
     }
+    for (int r = 0; r < kRing; ++r) mbar_init(&ring_bar[r], 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -118,17 +130,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint64_t pol_x = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
+      // incremental (tile, k-chunk) walk: no 64-bit divisions on the per-chunk path
+      int tile_i = (int)(u_begin / KC), kc = (int)(u_begin % KC);
+      int nt = tile_i / g.row_blocks, rb = tile_i % g.row_blocks;
       for (long long u = u_begin; u < u_end; ++u) {
-        const long long tile = u / KC;
-        const int kc = (int)(u % KC);
-        const int nt = (int)(tile / g.row_blocks), rb = (int)(tile % g.row_blocks);
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, g.status)) break;
         uint8_t* A = smem + stage * g.stage_bytes;
         uint8_t* B = A + kATileBytes;
         mbar_arrive_expect_tx(&full[stage], g.stage_bytes);
-        if (g.swiglu) {
+        if (g.a_mode == 1) {
           tma_load_2d(A, &tmA, &full[stage], kc * 64, nt * 64, pol_w);
           tma_load_2d(A + kATileBytes / 2, &tmA2, &full[stage], kc * 64, nt * 64, pol_w);
+        } else if (g.a_mode == 2) {
+          tma_load_4d(A, &tmA, &full[stage], kc * 64, 0, 0, nt, pol_w);
+        } else if (g.a_mode == 3) {
+          tma_load_5d(A, &tmA, &full[stage], kc * 64, 0, 0, 0, nt, pol_w);
         } else {
           tma_load_2d(A, &tmA, &full[stage], kc * 64, nt * 128, pol_w);
         }
@@ -136,6 +152,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_2d(B + p * part_rows * 128, &tmB, &full[stage], kc * 64,
                       g.row0 + rb * g.RT + p * part_rows, pol_x);
         if (++stage == g.nstages) { stage = 0; phase ^= 1; }
+        if (++kc == KC) {
+          kc = 0;
+          if (++rb == g.row_blocks) { rb = 0; ++nt; }
+        }
       }
     }
   } else if (warp == 1) {
@@ -182,13 +202,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else {
-    // Epilogue warps 2..5: TMEM lane quarter = warp % 4 -> output feature m.
+    // Epilogue warps 2..5: TMEM lane quarter = warp % 4 -> A-tile row m.
     const int q = warp & 3;
     const int m = q * 32 + lane;
-    const int et = threadIdx.x - 64;   // 0..127, barrier participant index
+    const int et = threadIdx.x - 64;   // 0..127
     int acc = 0;
     uint32_t acc_phase = 0;
     int sbuf = 0;
+    uint32_t io_phase[2] = {0u, 0u};
     long long u = u_begin;
     while (u < u_end) {
       const long long tile = u / KC;
@@ -196,70 +217,214 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const long long seg_end = min(u_end, tend);
       const bool full_tile = (u == tstart) && (seg_end == tend);
       const int nt = (int)(tile / g.row_blocks), rb = (int)(tile % g.row_blocks);
-      const int rbase = rb * g.RT;                       // first row of this block (relative)
+      const int rbase = rb * g.RT;                       // first activation row of the block
       const int nvalid_rows = min(g.RT, g.rows - rbase);
-      const int nchunks = (nvalid_rows + 15) >> 4;
+      const int nblk = (nvalid_rows + 31) >> 5;
       u = seg_end;
-      if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, g.status)) break;
+      // A failed (timed-out) wait only flags the status word: the epilogue threads keep going so
+      // that their named barriers stay matched; the results are then garbage but the kernel ends.
+      mbar_wait_sleep(&acc_full[acc], acc_phase, abort_flag, g.status);
       tc_fence_after();
       const uint32_t tacc = tbase + (uint32_t(q * 32) << 16) + acc * g.RT;
-      bool do_epi = true;
       // Residual epilogues are additive: split segments add straight into x (fp32 atomics).
       const bool additive = (ep.kind == kEpiResid);
+      const bool from_tmem = full_tile || additive;
+      bool do_epi = true;
       long long g_first = 0, g_last = -1;
-      if (!full_tile && !additive) {
-        const long long me = blockIdx.x;
-        const int slot = (cta_start(me, U, G) < tstart) ? 1 : 0;
-        float* P = g.partial + ((size_t)me * 2 + slot) * (size_t)g.RT * 128;
-        for (int c = 0; c < nchunks; ++c) {
-          float v[16];
-          tmem_ld16(tacc + c * 16, v);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) __stcg(&P[(size_t)(c * 16 + j) * 128 + m], v[j]);
+      // Split tile (non-additive epilogue): every contributing CTA except the last parks its
+      // fp32 segment in a slot ([blocks of 32 columns][128 rows], bulk stores); the last one
+      // sums all segments in segment order (deterministic) and runs the epilogue.  A CTA that
+      // finds every other segment already published (the usual case for the CTA finishing a
+      // tile, whose neighbour did its part first) skips parking its own segment and adds it
+      // straight from TMEM.
+      bool own_in_tmem = false;
+      if (!from_tmem) {
+        g_first = cta_of(tstart, U, G);
+        g_last = cta_of(tend - 1, U, G);
+        const unsigned nseg_u = (unsigned)(g_last - g_first + 1);
+        if (et == 0) {
+          const unsigned done = atomicAdd(&g.counters[tile], 0u);
+          *last_flag = (done == nseg_u - 1) ? 2 : 0;
         }
+        named_bar_sync(1, 128);
+        if (*last_flag == 2) {
+          own_in_tmem = true;
+          if (et == 0) {
+            __threadfence();
+            asm volatile("fence.proxy.async;" ::: "memory");   // partials are read by bulk copies
+            g.counters[tile] = 0u;                // nobody else touches it in this launch
+          }
+        } else {
+          const long long me = blockIdx.x;
+          const int slot = (cta_start(me, U, G) < tstart) ? 1 : 0;
+          float* P = g.partial + ((size_t)me * 2 + slot) * (size_t)g.RTp * 128;
+          for (int b = 0; b < nblk; ++b) {
+            float* buf = &staging[b & 1][0][0];
+            if (et == 0) bulk_wait_read<1>();    // the store issued from this buffer 2 blocks ago
+            named_bar_sync(1, 128);
+            float v[32];
+            tmem_ld32(tacc + b * 32, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) buf[j * 128 + m] = v[j];
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (et == 0) {
+              bulk_store(P + (size_t)b * 32 * 128, buf, 32 * 128 * 4);
+              bulk_commit();
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          if (et == 0) {
+            bulk_wait_all();                      // partial writes performed
+            asm volatile("fence.proxy.async;" ::: "memory");
+            __threadfence();
+            const unsigned prev = atomicAdd(&g.counters[tile], 1u);
+            const int is_last = (prev == nseg_u - 1) ? 1 : 0;
+            if (is_last) g.counters[tile] = 0u;   // ready for the next launch
+            __threadfence();
+            asm volatile("fence.proxy.async;" ::: "memory");
+            *last_flag = is_last;
+          }
+          named_bar_sync(1, 128);
+          do_epi = (*last_flag != 0);
+        }
+      }
+      if (do_epi) {
+        if (ep.kind == kEpiQKV) {
+          for (int r = et; r < nvalid_rows; r += 128) {
+            const int row = rbase + r;
+            meta_pos[r] = ep.row_pos[row];
+            meta_kv[r] = (long long)ep.row_seq[row] * ep.kv.seq_stride +
+                         (long long)ep.row_slot[row] * ep.d_head;
+          }
+          named_bar_sync(1, 128);
+        }
+        const int nseg = (int)(g_last - g_first + 1);
+        const int own_idx = (int)(blockIdx.x - g_first);
+        auto src = [&](int sidx, int b) {
+          const long long gg = g_first + sidx;
+          const int sl = (cta_start(gg, U, G) < tstart) ? 1 : 0;
+          return g.partial + ((size_t)gg * 2 + sl) * (size_t)g.RTp * 128 + (size_t)b * 32 * 128;
+        };
+        // Segments to fetch from memory (all but our own when it is still in TMEM).
+        const int nfetch = (from_tmem) ? 0 : (own_in_tmem ? nseg - 1 : nseg);
+        // When this was the CTA's final segment the pipeline stages are idle: use them as a
+        // ring of 16 KB landing slots so that several blocks' partial loads are in flight.
+        const int ring_cap = min(kRing, (g.nstages * g.stage_bytes) / 16384);
+        const bool use_ring = !from_tmem && nfetch > 0 && (seg_end == u_end) && ring_cap >= nfetch;
+        const int nload = use_ring ? nblk * nfetch : 0;
+        int issued = 0;
+        auto load_src = [&](int k) {    // k-th load: block k / nfetch, k % nfetch-th fetched segment
+          const int b = k / nfetch, kf = k % nfetch;
+          int c = -1, sidx = 0;
+          for (; sidx < nseg; ++sidx) {
+            if (own_in_tmem && sidx == own_idx) continue;
+            if (++c == kf) break;
+          }
+          return src(sidx, b);
+        };
+        if (use_ring) {
+          named_bar_sync(1, 128);
+          if (et == 0) {
+            for (; issued < min(ring_cap, nload); ++issued) {
+              const int slot = issued % ring_cap;
+              mbar_arrive_expect_tx(&ring_bar[slot], 16384);
+              bulk_load(smem + (size_t)slot * 16384, load_src(issued), 16384, &ring_bar[slot]);
+            }
+          }
+        }
+        for (int b = 0; b < nblk; ++b) {
+          float v[32];
+          if (from_tmem) {
+            tmem_ld32(tacc + b * 32, v);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+            if (use_ring) {
+              int kf = 0;
+              for (int sidx = 0; sidx < nseg; ++sidx) {
+                if (own_in_tmem && sidx == own_idx) {
+                  float w[32];
+                  tmem_ld32(tacc + b * 32, w);
+#pragma unroll
+                  for (int j = 0; j < 32; ++j) v[j] += w[j];
+                } else {
+                  const int k = b * nfetch + kf;
+                  const int slot = k % ring_cap;
+                  mbar_wait(&ring_bar[slot], (uint32_t)((k / ring_cap) & 1), abort_flag, g.status);
+                  const float* blkp = reinterpret_cast<const float*>(smem + (size_t)slot * 16384);
+#pragma unroll
+                  for (int j = 0; j < 32; ++j) v[j] += blkp[j * 128 + m];
+                  ++kf;
+                }
+              }
+            } else {
+              // two staging buffers, two loads in flight
+              named_bar_sync(1, 128);
+              int order[2];
+              int nf = 0;
+              auto fetch_index = [&](int k) {   // k-th fetched segment index
+                int c = -1;
+                for (int sidx = 0; sidx < nseg; ++sidx) {
+                  if (own_in_tmem && sidx == own_idx) continue;
+                  if (++c == k) return sidx;
+                }
+                return -1;
+              };
+              if (et == 0) {
+                for (int k = 0; k < min(2, nfetch); ++k) {
+                  mbar_arrive_expect_tx(&io_bar[k], 16384);
+                  bulk_load(&staging[k][0][0], src(fetch_index(k), b), 16384, &io_bar[k]);
+                }
+              }
+              (void)order;
+              (void)nf;
+              int k = 0;
+              for (int sidx = 0; sidx < nseg; ++sidx) {
+                if (own_in_tmem && sidx == own_idx) {
+                  float w[32];
+                  tmem_ld32(tacc + b * 32, w);
+#pragma unroll
+                  for (int j = 0; j < 32; ++j) v[j] += w[j];
+                  continue;
+                }
+                const int bi = k & 1;
+                mbar_wait(&io_bar[bi], io_phase[bi], abort_flag, g.status);
+                io_phase[bi] ^= 1;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] += staging[bi][j][m];
+                named_bar_sync(1, 128);           // everyone done with this buffer
+                if (et == 0 && k + 2 < nfetch) {
+                  mbar_arrive_expect_tx(&io_bar[bi], 16384);
+                  bulk_load(&staging[bi][0][0], src(fetch_index(k + 2), b), 16384, &io_bar[bi]);
+                }
+                ++k;
+              }
+            }
+          }
+          epilogue_block<T>(ep, v, staging[sbuf], nt * 128, rbase + b * 32, m,
+                            min(32, nvalid_rows - b * 32), !full_tile, meta_pos, meta_kv, rbase);
+          sbuf ^= 1;
+          // every thread passed the barrier inside the epilogue, so block b's slots are free
+          if (use_ring && et == 0) {
+            const int consumed = (b + 1) * nfetch;
+            for (; issued < min(nload, consumed + ring_cap); ++issued) {
+              const int slot = issued % ring_cap;
+              mbar_arrive_expect_tx(&ring_bar[slot], 16384);
+              bulk_load(smem + (size_t)slot * 16384, load_src(issued), 16384, &ring_bar[slot]);
+            }
+          }
+        }
+        named_bar_sync(1, 128);   // meta / staging / stages are reused afterwards
+      }
+      if (own_in_tmem) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        __threadfence();
-        named_bar_sync(1, 128);
-        g_first = cta_of(tstart, U, G);
-        g_last = cta_of(tend - 1, U, G);
-        if (et == 0) {
-          const unsigned nseg = (unsigned)(g_last - g_first + 1);
-          const unsigned prev = atomicAdd(&g.counters[tile], 1u);
-          const int is_last = (prev == nseg - 1) ? 1 : 0;
-          if (is_last) g.counters[tile] = 0u;   // ready for the next launch
-          *last_flag = is_last;
-        }
-        named_bar_sync(1, 128);
-        do_epi = (*last_flag != 0);
-        __threadfence();
       }
-      if (do_epi) {
-        const bool from_tmem = full_tile || additive;
-        for (int c = 0; c < nchunks; ++c) {
-          float v[16];
-          if (from_tmem) {
-            tmem_ld16(tacc + c * 16, v);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = 0.f;
-            // fixed summation order (segment order) -> deterministic results
-            for (long long gg = g_first; gg <= g_last; ++gg) {
-              const int sl = (cta_start(gg, U, G) < tstart) ? 1 : 0;
-              const float* P = g.partial + ((size_t)gg * 2 + sl) * (size_t)g.RT * 128;
-#pragma unroll
-              for (int j = 0; j < 16; ++j) v[j] += __ldcg(&P[(size_t)(c * 16 + j) * 128 + m]);
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 16; ++j) staging[sbuf][j][m] = v[j];
-          named_bar_sync(1, 128);
-          epilogue_tile<T>(ep, staging[sbuf], nt * 128, rbase + c * 16, m, !full_tile);
-          sbuf ^= 1;
-        }
-      }
-      if (from_tmem_release(full_tile, additive)) {
+      if (from_tmem) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
@@ -363,6 +528,7 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream) {
   GemmDev g{};
   g.KC = c.K / 64;
   g.swiglu = c.swiglu;
+  g.a_mode = c.swiglu ? 1 : c.a_interleave == 128 ? 2 : c.a_interleave == 64 ? 3 : 0;
   g.n_tiles = c.swiglu ? (c.n_out + 63) / 64 : (c.n_out + 127) / 128;
   g.RT = gemm_tc_row_tile(c.rows);
   g.row_blocks = (c.rows + g.RT - 1) / g.RT;
@@ -370,23 +536,30 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream) {
   g.row0 = c.row0;
   g.units = (long long)g.n_tiles * g.row_blocks * g.KC;
   const SmemLayout L = gemm_smem_layout(g.RT, c.max_stages > 0 ? c.max_stages : 8);
+  g.RTp = (g.RT + 31) & ~31;
   g.nstages = L.nstages;
   g.stage_bytes = L.stage_bytes;
   g.staging_off = L.staging_off;
+  g.meta_off = L.meta_off;
   g.bar_off = L.bar_off;
   g.n_acc = (g.RT <= 256) ? 2 : 1;
   g.tmem_cols = pow2_ceil(g.n_acc * g.RT);
   g.partial = c.partial;
   g.counters = c.counters;
   g.status = c.status;
+  // Grid: one CTA per SM, units split stream-K style.  When the tile count is close to the SM
+  // count, one whole tile per CTA (no split-K fixups, tight tail) beats splitting.
   long long G = c.num_ctas;
+  const long long tiles_total = (long long)g.n_tiles * g.row_blocks;
+  if (tiles_total <= G && tiles_total * 10 >= G * 6) G = tiles_total;
   if (G > g.units) G = g.units;
   if (G < 1) G = 1;
   if (g.n_tiles * g.row_blocks > c.max_tiles) return cudaErrorInvalidValue;
-  if ((long long)g.RT * 128 * 2 * G * 4 > (long long)c.partial_bytes)
+  if ((long long)g.RTp * 128 * 2 * G * 4 > (long long)c.partial_bytes)
     return cudaErrorInvalidValue;  // split-K scratch too small for this row tile
   gemm_tc_kernel<__nv_bfloat16><<<(unsigned)G, kGemmThreads, L.total, stream>>>(
       *c.tmA, c.swiglu ? *c.tmA2 : *c.tmA, *c.tmB, g, c.epi);
+  // (kEpiQKV requires a rotary-interleaved A map: a_interleave == d_head)
   return cudaGetLastError();
 }
 

@@ -13,9 +13,10 @@ struct GemmCall {
   int rows;                 // activation rows
   int row0;                 // first activation row in tmB
   int swiglu;
+  int a_interleave;         // 0, or d_head: tmA is the rotary-interleaved 4-D/5-D QKV map
   int num_ctas;             // persistent grid size (one CTA per SM)
   int max_stages;           // 0 = as many as fit
-  float* partial;           // split-K scratch: [num_ctas][2][row_tile][128] fp32
+  float* partial;           // split-K scratch: [num_ctas][2][128][row_tile rounded to 32] fp32
   size_t partial_bytes;
   unsigned* counters;       // [max_tiles], zero-initialised; restored to zero by the kernel
   int max_tiles;

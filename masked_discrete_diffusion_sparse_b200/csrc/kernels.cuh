@@ -112,10 +112,19 @@ SMDM_DEV void epilogue_tile(const EpiParams& p, const float (*S)[128], int n0, i
     case kEpiResid: {
       const int n = n0 + m;
       if (n < p.n_valid) {
+        float* __restrict__ x = p.x + (size_t)r0 * p.ld_x + n;
         if (atomic_resid) {
-          for (int j = 0; j < nrows; ++j) atomicAdd(&p.x[(size_t)(r0 + j) * p.ld_x + n], S[j][m]);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (j < nrows) atomicAdd(x + (size_t)j * p.ld_x, S[j][m]);
         } else {
-          for (int j = 0; j < nrows; ++j) p.x[(size_t)(r0 + j) * p.ld_x + n] += S[j][m];
+          // all loads first, then all stores: the rows are independent
+          float old[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) old[j] = (j < nrows) ? x[(size_t)j * p.ld_x] : 0.f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (j < nrows) x[(size_t)j * p.ld_x] = old[j] + S[j][m];
         }
       }
       break;
@@ -141,26 +150,44 @@ SMDM_DEV void epilogue_tile(const EpiParams& p, const float (*S)[128], int n0, i
       const int h = nn / p.d_head, i = nn % p.d_head;
       const int half = p.d_head >> 1;
       const int partner = (i < half) ? m + half : m - half;
-      T* kc = reinterpret_cast<T*>(p.kv.k);
-      T* vc = reinterpret_cast<T*>(p.kv.v);
-      T* qo = reinterpret_cast<T*>(p.q_out);
-      for (int j = 0; j < nrows; ++j) {
-        const int r = r0 + j;
-        float val = S[j][m];
-        if (region < 2) {
-          const float2 cs = p.rope[(size_t)p.row_pos[r] * half + (i % half)];
-          const float other = S[j][partner];
-          val = (i < half) ? (val * cs.x - other * cs.y) : (other * cs.y + val * cs.x);
+      T* __restrict__ kc = reinterpret_cast<T*>(p.kv.k);
+      T* __restrict__ vc = reinterpret_cast<T*>(p.kv.v);
+      T* __restrict__ qo = reinterpret_cast<T*>(p.q_out);
+      // metadata for the 16 rows first (independent loads), then the rotary table, then stores
+      int pos[16], seq[16], slot[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int r = r0 + min(j, nrows - 1);
+        pos[j] = __ldg(p.row_pos + r);
+        seq[j] = __ldg(p.row_seq + r);
+        slot[j] = __ldg(p.row_slot + r);
+      }
+      float val[16];
+      if (region < 2) {
+        float2 cs[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) cs[j] = __ldg(p.rope + (size_t)pos[j] * half + (i % half));
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float a = S[j][m], b = S[j][partner];
+          val[j] = (i < half) ? (a * cs[j].x - b * cs[j].y) : (b * cs[j].y + a * cs[j].x);
         }
-        if (region == 0) {
-          qo[(size_t)r * p.d_model + nn] = from_f<T>(val);
-        } else {
-          const long long off = (long long)p.row_seq[r] * p.kv.seq_stride +
-                                (long long)p.layer * p.kv.layer_stride +
-                                (long long)h * p.kv.head_stride +
-                                (long long)p.row_slot[r] * p.d_head + i;
-          (region == 1 ? kc : vc)[off] = from_f<T>(val);
-        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) val[j] = S[j][m];
+      }
+      if (region == 0) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (j < nrows) qo[(size_t)(r0 + j) * p.d_model + nn] = from_f<T>(val[j]);
+      } else {
+        T* __restrict__ base = (region == 1 ? kc : vc) + (long long)p.layer * p.kv.layer_stride +
+                               (long long)h * p.kv.head_stride + i;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (j < nrows)
+            base[(long long)seq[j] * p.kv.seq_stride + (long long)slot[j] * p.d_head] =
+                from_f<T>(val[j]);
       }
       break;
     }
@@ -199,6 +226,193 @@ SMDM_DEV void epilogue_tile(const EpiParams& p, const float (*S)[128], int n0, i
           p.pmax[idx] = best;
           p.parg[idx] = arg;
           p.psum[idx] = s;
+        }
+      }
+      break;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Register epilogue of the tcgen05 GEMM: one block of 32 activation rows (TMEM columns) for the
+// A-tile row held by TMEM lane m; v[j] = accumulator of activation row r0 + j.
+//   - QKV tiles are loaded with rotary partners interleaved (A-tile row 2i <- weight row i of
+//     the first half of a head, row 2i + 1 <- row i of the second half), so the rotation needs
+//     only a lane exchange with lane m ^ 1.
+//   - SwiGLU and the LM-head statistics combine values of different lanes through `stage`
+//     ([32][128] fp32 shared memory, one barrier per block, callers alternate two buffers).
+//   - meta_pos / meta_kv: per-row position and K/V cache offset of the tile's rows (shared
+//     memory, filled once per tile), indexed by row - meta_r0.
+// ------------------------------------------------------------------------------------------
+SMDM_DEV int qkv_lane_feature(int m, int d_head) {
+  if (d_head == 128) return (m & 1) * 64 + (m >> 1);
+  return (m >> 6) * 64 + (m & 1) * 32 + ((m >> 1) & 31);     // d_head == 64
+}
+
+SMDM_DEV void store8(__nv_bfloat16* dst, const float* f) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]), b = __floats2bfloat162_rn(f[2], f[3]),
+                 c = __floats2bfloat162_rn(f[4], f[5]), d = __floats2bfloat162_rn(f[6], f[7]);
+  uint4 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  u.z = *reinterpret_cast<uint32_t*>(&c);
+  u.w = *reinterpret_cast<uint32_t*>(&d);
+  *reinterpret_cast<uint4*>(dst) = u;
+}
+
+// Epilogue of one block of 32 activation rows.  v[j]: accumulator of row r0 + j for A-tile row
+// m (TMEM lane).  Register step: rotary on q/k (lane pairs m, m ^ 1 hold x_i, x_{i+d/2}).
+// Then the block is staged in shared memory as S[32 rows][128 features] and written row-major
+// with 16-byte vectors (scattered 2-byte stores would stall on outstanding-request slots).
+// One named barrier (128 epilogue threads); callers alternate two staging buffers.
+template <typename T>
+SMDM_DEV void epilogue_block(const EpiParams& p, float* v, float (*S)[128], int n0, int r0, int m,
+                             int nrows, bool atomic_resid, const int* meta_pos,
+                             const long long* meta_kv, int meta_r0) {
+  int f = m;   // feature (0..127 within the tile) held by this lane
+  if (p.kind == kEpiQKV) {
+    const int dh = p.d_head, half = dh >> 1;
+    f = qkv_lane_feature(m, dh);
+    const int region = n0 / p.d_model;
+    if (region < 2) {
+      const int ih = (f % dh) % half;
+      const bool second = (m & 1) != 0;
+#pragma unroll
+      for (int g = 0; g < 32; g += 8) {
+        float2 cs[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int jj = min(g + j, nrows - 1);
+          cs[j] = __ldg(p.rope + (size_t)meta_pos[r0 + jj - meta_r0] * half + ih);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float a = v[g + j];
+          const float b = __shfl_xor_sync(0xffffffffu, a, 1);
+          v[g + j] = second ? (b * cs[j].y + a * cs[j].x) : (a * cs[j].x - b * cs[j].y);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) S[j][f] = v[j];
+  named_bar_sync(1, 128);
+  const int t = m;   // 0..127 consumer index
+  switch (p.kind) {
+    case kEpiStore: {
+      T* out = reinterpret_cast<T*>(p.out);
+      if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int idx = t + 128 * q, j = idx >> 4, c = (idx & 15) * 8;
+          if (j < nrows && n0 + c < p.n_valid)
+            store8(reinterpret_cast<__nv_bfloat16*>(out) + (size_t)(r0 + j) * p.ld_out + n0 + c, &S[j][c]);
+        }
+      }
+      break;
+    }
+    case kEpiQKV: {
+      const int dh = p.d_head;
+      const int region = n0 / p.d_model;
+      const int nn0 = n0 - region * p.d_model;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int idx = t + 128 * q, j = idx >> 4, c = (idx & 15) * 8;
+        if (j >= nrows) continue;
+        __nv_bfloat16* dst;
+        if (region == 0) {
+          dst = reinterpret_cast<__nv_bfloat16*>(p.q_out) + (size_t)(r0 + j) * p.d_model + nn0 + c;
+        } else {
+          const int h = (nn0 + c) / dh, i = (nn0 + c) % dh;
+          dst = reinterpret_cast<__nv_bfloat16*>(region == 1 ? p.kv.k : p.kv.v) +
+                (long long)p.layer * p.kv.layer_stride + (long long)h * p.kv.head_stride +
+                meta_kv[r0 + j - meta_r0] + i;
+        }
+        store8(dst, &S[j][c]);
+      }
+      break;
+    }
+    case kEpiResid: {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int idx = t + 128 * q, j = idx >> 5, c = (idx & 31) * 4;
+        if (j >= nrows || n0 + c >= p.n_valid) continue;
+        float* x = p.x + (size_t)(r0 + j) * p.ld_x + n0 + c;
+        const float4 a = *reinterpret_cast<const float4*>(&S[j][c]);
+        if (atomic_resid) {
+          asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(x), "f"(a.x),
+                       "f"(a.y), "f"(a.z), "f"(a.w)
+                       : "memory");
+        } else {
+          float4 o = *reinterpret_cast<const float4*>(x);
+          o.x += a.x;
+          o.y += a.y;
+          o.z += a.z;
+          o.w += a.w;
+          *reinterpret_cast<float4*>(x) = o;
+        }
+      }
+      break;
+    }
+    case kEpiSwiGLU: {
+      // features 0..63 = gate rows f0 + i, 64..127 = up rows f0 + i
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int idx = t + 128 * q, j = idx >> 3, c = (idx & 7) * 8;
+        if (j >= nrows || (n0 >> 1) + c >= p.n_valid) continue;
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = silu_f(S[j][c + e]) * S[j][64 + c + e];
+        if constexpr (sizeof(T) == 2)
+          store8(reinterpret_cast<__nv_bfloat16*>(p.act) + (size_t)(r0 + j) * p.ld_act + (n0 >> 1) + c, o);
+      }
+      break;
+    }
+    case kEpiLMHead: {
+      if (p.logits) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int idx = t + 128 * q, j = idx >> 5, c = (idx & 31) * 4;
+          if (j >= nrows) continue;
+          float* dst = p.logits + (size_t)(r0 + j) * p.ld_logits + n0 + c;
+          if (n0 + c + 4 <= p.n_valid && (p.ld_logits & 3) == 0) {
+            *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(&S[j][c]);
+          } else {
+            for (int e = 0; e < 4; ++e)
+              if (n0 + c + e < p.n_valid) dst[e] = S[j][c + e];
+          }
+        }
+      }
+      const int warp = t >> 5, lane = t & 31;
+      const int vt = n0 >> 7;
+      for (int j = warp * 8; j < min(warp * 8 + 8, nrows); ++j) {
+        float best = -INFINITY;
+        int arg = 0x7fffffff;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int ff = lane + 32 * u;
+          const float x = (n0 + ff < p.n_valid) ? S[j][ff] : -INFINITY;
+          if (x > best) { best = x; arg = n0 + ff; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+          const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
+          if (ob > best || (ob == best && oa < arg)) { best = ob; arg = oa; }
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int ff = lane + 32 * u;
+          if (n0 + ff < p.n_valid) sum += __expf(S[j][ff] - best);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0) {
+          const size_t idx = (size_t)(r0 + j) * p.n_vt + vt;
+          p.pmax[idx] = best;
+          p.parg[idx] = arg;
+          p.psum[idx] = sum;
         }
       }
       break;

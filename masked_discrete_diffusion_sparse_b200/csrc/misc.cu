@@ -160,42 +160,73 @@ __global__ void gather_rows_kernel(const int* __restrict__ src_rows, int n, int*
 // RMSNorm: out[r] = x[src] / sqrt(mean(x[src]^2) + eps) * g.  With emb != nullptr the source
 // row is first gathered from the embedding table into the fp32 residual stream x.
 // ------------------------------------------------------------------------------------------
+template <typename T> struct Vec4;
+template <> struct Vec4<float> {
+  using type = float4;
+  static SMDM_DEV float4 load(const float* p) { return *reinterpret_cast<const float4*>(p); }
+  static SMDM_DEV void store(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+};
+template <> struct Vec4<__nv_bfloat16> {
+  static SMDM_DEV float4 load(const __nv_bfloat16* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+  }
+  static SMDM_DEV void store(__nv_bfloat16* p, float4 v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+  }
+};
+
+// One CTA of 256 threads per row; the row stays in registers (d <= 8192, d % 4 == 0).
 template <typename T>
-__global__ void rmsnorm_kernel(NormArgs a) {
+__global__ void __launch_bounds__(256) rmsnorm_kernel(NormArgs a) {
+  constexpr int kMaxV = 8;
   const int r = blockIdx.x;
   const int src = a.gather ? a.gather[r] : r;
   float* xr = a.x + (size_t)src * a.d;
   const T* g = reinterpret_cast<const T*>(a.gain);
-  __shared__ float red[32];
+  __shared__ float red[8];
+  const int d4 = a.d >> 2;
+  float4 v[kMaxV];
   float ss = 0.f;
-  if (a.emb) {
-    const int id = a.ids[src];
-    const T* e = reinterpret_cast<const T*>(a.emb) + (size_t)id * a.d;
-    for (int i = threadIdx.x; i < a.d; i += blockDim.x) {
-      const float v = to_f(e[i]);
-      xr[i] = v;
-      ss += v * v;
-    }
-  } else {
-    for (int i = threadIdx.x; i < a.d; i += blockDim.x) {
-      const float v = xr[i];
-      ss += v * v;
+  const T* e = a.emb ? reinterpret_cast<const T*>(a.emb) + (size_t)a.ids[src] * a.d : nullptr;
+#pragma unroll
+  for (int t = 0; t < kMaxV; ++t) {
+    const int i4 = threadIdx.x + t * 256;
+    if (i4 < d4) {
+      if (e) {
+        v[t] = Vec4<T>::load(e + 4 * i4);
+        *reinterpret_cast<float4*>(xr + 4 * i4) = v[t];
+      } else {
+        v[t] = *reinterpret_cast<const float4*>(xr + 4 * i4);
+      }
+      ss += v[t].x * v[t].x + v[t].y * v[t].y + v[t].z * v[t].z + v[t].w * v[t].w;
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
-  if (threadIdx.x < 32) {
-    float t = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.f;
+  float tot = 0.f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-    if (threadIdx.x == 0) red[0] = t;
-  }
-  __syncthreads();
-  const float rstd = rsqrtf(red[0] / (float)a.d + a.eps);
+  for (int i = 0; i < 8; ++i) tot += red[i];
+  const float rstd = rsqrtf(tot / (float)a.d + a.eps);
   T* out = reinterpret_cast<T*>(a.out) + (size_t)r * a.d;
-  for (int i = threadIdx.x; i < a.d; i += blockDim.x) out[i] = from_f<T>(xr[i] * rstd * to_f(g[i]));
+#pragma unroll
+  for (int t = 0; t < kMaxV; ++t) {
+    const int i4 = threadIdx.x + t * 256;
+    if (i4 < d4) {
+      const float4 gg = Vec4<T>::load(g + 4 * i4);
+      Vec4<T>::store(out + 4 * i4, make_float4(v[t].x * rstd * gg.x, v[t].y * rstd * gg.y,
+                                               v[t].z * rstd * gg.z, v[t].w * rstd * gg.w));
+    }
+  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -207,20 +238,32 @@ __global__ void unmask_kernel(UnmaskArgs a) {
   float* conf = sh;                                     // [n_q]
   int* tok = reinterpret_cast<int*>(sh + s.n_q);        // [n_q]
   int* commit = tok + s.n_q;                            // [n_q]
-  for (int j = threadIdx.x; j < s.n_q; j += blockDim.x) {
+  const int lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int j = threadIdx.x >> 5; j < s.n_q; j += nwarps) {
     const int lr = s.dense ? (a.qpos_of[s.qbase + j] - s.P - 1) : (s.qbase + j);
     const float* pm = a.pmax + (size_t)(s.lbase + lr) * a.n_vt;
     const float* ps = a.psum + (size_t)(s.lbase + lr) * a.n_vt;
     const int* pa = a.parg + (size_t)(s.lbase + lr) * a.n_vt;
     float M = -INFINITY;
-    int arg = 0;
-    for (int t = 0; t < a.n_vt; ++t) {
-      if (pm[t] > M) { M = pm[t]; arg = pa[t]; }   // first tile wins ties -> lowest id
+    int arg = 0x7fffffff;
+    for (int t = lane; t < a.n_vt; t += 32) {
+      const float v = pm[t];
+      if (v > M) { M = v; arg = pa[t]; }   // tiles in vocab order: first max = lowest id
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float oM = __shfl_xor_sync(0xffffffffu, M, o);
+      const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
+      if (oM > M || (oM == M && oa < arg)) { M = oM; arg = oa; }
     }
     float z = 0.f;
-    for (int t = 0; t < a.n_vt; ++t) z += ps[t] * __expf(pm[t] - M);
-    conf[j] = 1.f / z;
-    tok[j] = arg;
+    for (int t = lane; t < a.n_vt; t += 32) z += ps[t] * __expf(pm[t] - M);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane == 0) {
+      conf[j] = 1.f / z;
+      tok[j] = arg;
+    }
   }
   __syncthreads();
   for (int j = threadIdx.x; j < s.n_q; j += blockDim.x) {
@@ -236,19 +279,37 @@ __global__ void unmask_kernel(UnmaskArgs a) {
     if (a.conf_out) a.conf_out[s.qbase + j] = conf[j];
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int n = 0;
-    for (int j = 0; j < s.n_q; ++j) {
-      if (!commit[j]) continue;
+  // Committed rows keep their row order: index = number of committed rows before them
+  // (block-wide exclusive scan over the commit flags, one tile of blockDim rows at a time).
+  __shared__ int warp_sums[32];
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < s.n_q; base += blockDim.x) {
+    const int j = base + threadIdx.x;
+    const int c = (j < s.n_q) ? commit[j] : 0;
+    const unsigned ballot = __ballot_sync(0xffffffffu, c);
+    if (lane == 0) warp_sums[threadIdx.x >> 5] = __popc(ballot);
+    __syncthreads();
+    int before = carry;
+    for (int w = 0; w < (int)(threadIdx.x >> 5); ++w) before += warp_sums[w];
+    before += __popc(ballot & ((1u << lane) - 1u));
+    if (c) {
       const int p = a.qpos_of[s.qbase + j];
       if (p <= s.P || p > s.P + s.Lg) {
         atomicOr(a.status, kStatusBounds);
-        continue;
+      } else {
+        s.grid[p - s.P - 1] = tok[j];
+        if (s.newpos) s.newpos[before] = p;
       }
-      s.grid[p - s.P - 1] = tok[j];
-      if (s.newpos) s.newpos[n] = p;
-      ++n;
     }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int t = 0;
+      for (int w = 0; w < nwarps; ++w) t += warp_sums[w];
+      carry += t;
+    }
+    __syncthreads();
   }
 }
 
@@ -298,7 +359,7 @@ template cudaError_t launch_rmsnorm<__nv_bfloat16>(const NormArgs&, int, cudaStr
 
 cudaError_t launch_unmask(const UnmaskArgs& a, int max_nq, cudaStream_t st) {
   const size_t smem = (size_t)max_nq * 12;
-  unmask_kernel<<<a.n_seq, 256, smem, st>>>(a);
+  unmask_kernel<<<a.n_seq, 512, smem, st>>>(a);
   return cudaGetLastError();
 }
 cudaError_t launch_debug_mask(const int* type, const int* label, int n, uint32_t* bitmap,
