@@ -144,12 +144,15 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, vis: np.ndarray) -> n
     q: [nq][H][dh]; k, v: [nk][H][dh]; vis: bool [nq][nk].  Every query must see >= 1 key.
     """
     dh = q.shape[-1]
-    s = np.einsum("qhd,khd->hqk", q, k) / math.sqrt(dh)
+    qh = np.ascontiguousarray(q.transpose(1, 0, 2))        # [H][nq][dh]
+    kh = np.ascontiguousarray(k.transpose(1, 2, 0))        # [H][dh][nk]
+    vh = np.ascontiguousarray(v.transpose(1, 0, 2))        # [H][nk][dh]
+    s = np.matmul(qh, kh) / math.sqrt(dh)                  # [H][nq][nk]
     s = np.where(vis[None, :, :], s, -np.inf)
     s = s - np.max(s, axis=-1, keepdims=True)
     p = np.exp(s)
     p = p / np.sum(p, axis=-1, keepdims=True)
-    return np.einsum("hqk,khd->qhd", p, v)
+    return np.matmul(p, vh).transpose(1, 0, 2)             # [nq][H][dh]
 
 
 class Model:
