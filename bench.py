@@ -188,26 +188,32 @@ class ClockSampler:
 # CPU oracle (reported baseline and the reference arm)
 # ----------------------------------------------------------------------------------------------
 
-def oracle_sample(wl: synth.Workload):
-    """Time the fp64 oracle on the host: prefill + the first sampling step of sequence 0.
-    Returns (seconds, decoded tokens, description, threads)."""
-    import oracle
-    w = synth.make_weights(wl.model, wl.seed)
-    om = oracle.Model(w)
-    prompt = synth.make_prompt(wl)
-    plan = synth.make_plan(wl)
-    t0 = time.perf_counter()
-    st = oracle.Incremental(om, prompt, wl.gen_len)
-    qp = oracle.query_set(plan, st, 1)
-    lg = st.step_logits(qp)
-    tok, conf, rows = oracle.unmask(lg, oracle.POLICY_ALL if plan.kind == "order"
-                                    else oracle.POLICY_TOPN, plan.commit)
-    dt = time.perf_counter() - t0
-    n_dec = len(rows)
-    threads = _blas_threads()
-    desc = (f"oracle prefill ({wl.prompt_len} rows) + sampling step 1 ({len(qp)} decode rows, "
-            f"{n_dec} tokens committed) of the same workload, fp64 numpy")
-    return dt, n_dec, desc, threads
+class OracleSample:
+    """The fp64 oracle on the host cores, timed on a bounded sample of the workload: prefill of
+    sequence 0 plus its first sampling step.  Weights are generated once, outside the timing."""
+
+    def __init__(self, wl: synth.Workload):
+        import oracle
+        self.oracle = oracle
+        self.wl = wl
+        self.om = oracle.Model(synth.make_weights(wl.model, wl.seed))
+        self.prompt = synth.make_prompt(wl)
+        self.plan = synth.make_plan(wl)
+
+    def run(self):
+        """Returns (seconds, decoded tokens, description, threads)."""
+        o, wl = self.oracle, self.wl
+        t0 = time.perf_counter()
+        st = o.Incremental(self.om, self.prompt, wl.gen_len)
+        qp = o.query_set(self.plan, st, 1)
+        lg = st.step_logits(qp)
+        tok, conf, rows = o.unmask(lg, o.POLICY_ALL if self.plan.kind == "order"
+                                   else o.POLICY_TOPN, self.plan.commit)
+        dt = time.perf_counter() - t0
+        n_dec = len(rows)
+        desc = (f"oracle prefill ({wl.prompt_len} rows) + sampling step 1 ({len(qp)} decode rows, "
+                f"{n_dec} tokens committed) of the same workload, fp64 numpy")
+        return dt, n_dec, desc, _blas_threads()
 
 
 def _blas_threads() -> int:
@@ -229,8 +235,9 @@ def run_reference(args, wl):
     n_dec = 1
     desc = ""
     threads = 1
+    sample = OracleSample(wl)
     for i in range(args.warmup + args.steps):
-        dt, n_dec, desc, threads = oracle_sample(wl)
+        dt, n_dec, desc, threads = sample.run()
         if i >= args.warmup:
             times.append(dt)
     mean = sum(times) / len(times)
@@ -484,7 +491,7 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         try:
-            dt, n_dec, desc, threads = oracle_sample(wl)
+            dt, n_dec, desc, threads = OracleSample(wl).run()
             line["cpu_baseline"] = {"value": n_dec * B / dt, "unit": UNIT, "cores": threads,
                                     "kind": "oracle", "sample": desc, "seconds": dt}
         except MemoryError:
