@@ -51,6 +51,13 @@ SMDM_DEV void p_store_swizzled(uint8_t* P, int row, int key8, uint4 val) {
   *reinterpret_cast<uint4*>(dst) = val;
 }
 
+// 2^x with the hardware approximation (PTX ex2.approx.ftz.f32).
+SMDM_DEV float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 SMDM_DEV uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -211,23 +218,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int b = j & 1;
       if (!mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag, a.status)) break;
       tc_fence_after();
-      float s[128];
-      if (warp_any) {
-        tmem_ld64(tbase + lane_off + b * 128, s);
-        tmem_ld64(tbase + lane_off + b * 128 + 64, s + 64);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[b]);
       if (!warp_any) {
         // no valid query row in this warp: keep the barrier protocol, skip the math
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[b]);
         if (j >= 1 && !mbar_wait(pv_done, (j - 1) & 1, abort_flag, a.status)) break;
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
         continue;
       }
       const int key0 = (j0 + j) * 128;
-      float mx = -INFINITY;
       // visibility of the 128 keys as four 32-bit masks (registers only, no local arrays)
       uint32_t mw[4];
 #pragma unroll
@@ -239,22 +240,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           bits = n_ok == 32 ? 0xffffffffu : ((1u << n_ok) - 1u);
         } else {
           bits = 0;
-          for (int b = 0; b < 32; ++b) {
-            const int key = kb + b;
+          for (int bb = 0; bb < 32; ++bb) {
+            const int key = kb + bb;
             if (key < kv_lim && step_causal_allowed(tq, lq, a.type[key], a.label[key]))
-              bits |= 1u << b;
+              bits |= 1u << bb;
           }
         }
         mw[w] = bits;
       }
+      // pass 1: row maximum over the visible keys (two 64-column halves)
+      float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        s[c] = ((mw[c >> 5] >> (c & 31)) & 1u) ? s[c] * a.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, s[c]);
+      for (int hh = 0; hh < 2; ++hh) {
+        float sv[64];
+        tmem_ld64(tbase + lane_off + b * 128 + hh * 64, sv);
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if ((mw[hh * 2 + (c >> 5)] >> (c & 31)) & 1u) mx = fmaxf(mx, sv[c]);
       }
+      mx *= a.scale_log2;
       float alpha = 1.f;
       if (mx > m_ref + 8.f) {          // move the reference maximum (also the first time)
-        alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
+        alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mx);
         m_ref = mx;
       }
       float rs = 0.f;
@@ -270,22 +277,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_st16(t_o + lane_off + c * 16, o);
         }
       }
+      // pass 2: P = 2^(s*scale - m_ref) as bf16 into swizzled shared memory
+      const float mref_eff = (m_ref == -INFINITY) ? 0.f : m_ref;
 #pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
-        float p[8];
+      for (int hh = 0; hh < 2; ++hh) {
+        float sv[64];
+        tmem_ld64(tbase + lane_off + b * 128 + hh * 64, sv);
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const float sv = s[c8 * 8 + t];
-          p[t] = (sv == -INFINITY) ? 0.f : exp2f(sv - m_ref);
-          rs += p[t];
+        for (int c8 = 0; c8 < 8; ++c8) {
+          float p[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int c = c8 * 8 + t;
+            const bool vis = (mw[hh * 2 + (c >> 5)] >> (c & 31)) & 1u;
+            p[t] = vis ? ex2_approx(fmaf(sv[c], a.scale_log2, -mref_eff)) : 0.f;
+            rs += p[t];
+          }
+          uint4 pk;
+          pk.x = pack_bf16x2(p[0], p[1]);
+          pk.y = pack_bf16x2(p[2], p[3]);
+          pk.z = pack_bf16x2(p[4], p[5]);
+          pk.w = pack_bf16x2(p[6], p[7]);
+          p_store_swizzled(Ps, em, hh * 8 + c8, pk);
         }
-        uint4 pk;
-        pk.x = pack_bf16x2(p[0], p[1]);
-        pk.y = pack_bf16x2(p[2], p[3]);
-        pk.z = pack_bf16x2(p[4], p[5]);
-        pk.w = pack_bf16x2(p[6], p[7]);
-        p_store_swizzled(Ps, em, c8, pk);
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[b]);
       l = l * alpha + rs;
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
