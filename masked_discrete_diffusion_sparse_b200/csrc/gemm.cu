@@ -15,7 +15,7 @@
 
 namespace smdm {
 
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 224;   // 7 warps: 2 producers, MMA, 4 epilogue
 constexpr int kATileBytes = 128 * 128;   // 128 rows x 64 bf16
 constexpr int kRing = 16;                // max landing slots (16 KB each) for split-K partials
 
@@ -59,6 +59,7 @@ struct GemmDev {
   int a_mode;      // 0: 2-D box {64,128}; 1: SwiGLU gate+up boxes {64,64};
                    // 2: 4-D rotary interleave (d_head 128); 3: 5-D rotary interleave (d_head 64)
   int RTp;         // partial-sum row stride (RT rounded up to 32)
+  int np;          // TMA producer threads (1 or 2; stages alternate between them)
   int nstages, stage_bytes, staging_off, meta_off, bar_off;
   int n_acc, tmem_cols;
   float* partial;
@@ -70,7 +71,12 @@ SMDM_DEV long long cta_start(long long g, long long U, long long G) { return g *
 // CTA whose unit range contains unit u (inverse of cta_start).
 SMDM_DEV long long cta_of(long long u, long long U, long long G) { return ((u + 1) * G - 1) / U; }
 
-template <typename T>
+// kPair == 1: one CTA per SM.  kPair == 2: clusters of two CTAs on an SM pair running M=256
+// tcgen05 MMAs (cta_group::2): each CTA streams its own 128 weight rows but only half of the
+// activation rows, which halves the per-SM activation traffic.  The pair's first CTA issues the
+// MMAs; both CTAs run their own epilogue on their 128 rows of the accumulator.
+// NP: MMA N-parts per k-step (2 when the row tile exceeds 256 activation rows).
+template <typename T, int kPair, int NP>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                    const __grid_constant__ CUtensorMap tmB, const GemmDev g, const EpiParams ep) {
@@ -92,6 +98,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_holder + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = (kPair == 2) ? cluster_ctarank() : 0u;
+  const bool leader = (rank == 0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < g.nstages; ++s) {
       mbar_init(&full[s], 1);
@@ -99,7 +107,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], 4 * kPair);
       mbar_init(&io_bar[a], 1);
     }
     for (int r = 0; r < kRing; ++r) mbar_init(&ring_bar[r], 1);
@@ -109,58 +117,109 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tmB);
     if (g.swiglu) tma_prefetch_desc(&tmA2);
   }
+  // Pair: both CTAs are running and their barriers initialised before any cross-CTA signal or
+  // the pair's joint TMEM allocation (one warp in each CTA allocates collectively).
+  if constexpr (kPair == 2) cluster_sync_all();
   if (warp == 1) {
-    tmem_alloc(tmem_holder, g.tmem_cols);
-    tmem_relinquish();
+    if constexpr (kPair == 2) {
+      tmem_alloc_pair(tmem_holder, g.tmem_cols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, g.tmem_cols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
 
-  const long long U = g.units, G = gridDim.x;
-  const long long u_begin = cta_start(blockIdx.x, U, G), u_end = cta_start(blockIdx.x + 1, U, G);
+  // Work is split over pairs (kPair == 2) or CTAs; a tile is kPair * 128 weight rows.
+  const long long U = g.units, G = gridDim.x / kPair;
+  const long long gp = blockIdx.x / kPair;
+  const long long u_begin = cta_start(gp, U, G), u_end = cta_start(gp + 1, U, G);
   const int KC = g.KC;
-  const int part_rows = (g.RT > 256) ? (g.RT >> 1) : g.RT;
-  const int nparts = (g.RT > 256) ? 2 : 1;
+  const int part_rows = g.RT / NP;                             // MMA N per part
+  constexpr int nparts = NP;
+  const int b_rows = part_rows / kPair;                        // B rows per part in this CTA
+  // barriers that the pair's TMA and epilogue arrivals target live in the first CTA
+  auto lead_addr = [&](uint64_t* bar) -> uint32_t {
+    return (kPair == 2) ? mapa_shared(smem_u32(bar), 0) : smem_u32(bar);
+  };
 
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp == 0 || warp == 6) {
+    // Producers: with np == 2, warp 0 fills the CTA's even units and warp 6 the odd ones (a
+    // single thread issuing every TMA copy caps the SM's copy rate well below its bandwidth).
+    const int pidx = (warp == 0) ? 0 : 1;
+    if (lane == 0 && pidx < g.np) {
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
+      const int np = g.np, NS = g.nstages;
+      int stage = pidx % NS;
+      uint32_t phase = (uint32_t)((pidx / NS) & 1);
       // incremental (tile, k-chunk) walk: no 64-bit divisions on the per-chunk path
-      int tile_i = (int)(u_begin / KC), kc = (int)(u_begin % KC);
+      const long long u_first = u_begin + pidx;
+      int tile_i = (int)(u_first / KC), kc = (int)(u_first % KC);
       int nt = tile_i / g.row_blocks, rb = tile_i % g.row_blocks;
-      for (long long u = u_begin; u < u_end; ++u) {
+      for (long long u = u_first; u < u_end; u += np) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, g.status)) break;
         uint8_t* A = smem + stage * g.stage_bytes;
         uint8_t* B = A + kATileBytes;
-        mbar_arrive_expect_tx(&full[stage], g.stage_bytes);
-        if (g.a_mode == 1) {
-          tma_load_2d(A, &tmA, &full[stage], kc * 64, nt * 64, pol_w);
-          tma_load_2d(A + kATileBytes / 2, &tmA2, &full[stage], kc * 64, nt * 64, pol_w);
-        } else if (g.a_mode == 2) {
-          tma_load_4d(A, &tmA, &full[stage], kc * 64, 0, 0, nt, pol_w);
-        } else if (g.a_mode == 3) {
-          tma_load_5d(A, &tmA, &full[stage], kc * 64, 0, 0, 0, nt, pol_w);
+        const int at = nt * kPair + (int)rank;    // this CTA's 128-row A tile
+        if constexpr (kPair == 1) {
+          mbar_arrive_expect_tx(&full[stage], g.stage_bytes);
+          if (g.a_mode == 1) {
+            tma_load_2d(A, &tmA, &full[stage], kc * 64, at * 64, pol_w);
+            tma_load_2d(A + kATileBytes / 2, &tmA2, &full[stage], kc * 64, at * 64, pol_w);
+          } else if (g.a_mode == 2) {
+            tma_load_4d(A, &tmA, &full[stage], kc * 64, 0, 0, at, pol_w);
+          } else if (g.a_mode == 3) {
+            tma_load_5d(A, &tmA, &full[stage], kc * 64, 0, 0, 0, at, pol_w);
+          } else {
+            tma_load_2d(A, &tmA, &full[stage], kc * 64, at * 128, pol_w);
+          }
+          for (int p = 0; p < nparts; ++p)
+            tma_load_2d(B + p * b_rows * 128, &tmB, &full[stage], kc * 64,
+                        g.row0 + rb * g.RT + p * part_rows, pol_x);
         } else {
-          tma_load_2d(A, &tmA, &full[stage], kc * 64, nt * 128, pol_w);
+          // both CTAs' bytes complete on the first CTA's barrier, which expects them all
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * g.stage_bytes);
+          const uint32_t fb = lead_addr(&full[stage]);
+          if (g.a_mode == 1) {
+            tma_load_2d_pair(A, &tmA, fb, kc * 64, at * 64, pol_w);
+            tma_load_2d_pair(A + kATileBytes / 2, &tmA2, fb, kc * 64, at * 64, pol_w);
+          } else if (g.a_mode == 2) {
+            tma_load_4d_pair(A, &tmA, fb, kc * 64, 0, 0, at, pol_w);
+          } else if (g.a_mode == 3) {
+            tma_load_5d_pair(A, &tmA, fb, kc * 64, 0, 0, 0, at, pol_w);
+          } else {
+            tma_load_2d_pair(A, &tmA, fb, kc * 64, at * 128, pol_w);
+          }
+          for (int p = 0; p < nparts; ++p)
+            tma_load_2d_pair(B + p * b_rows * 128, &tmB, fb, kc * 64,
+                             g.row0 + rb * g.RT + p * part_rows + (int)rank * b_rows, pol_x);
         }
-        for (int p = 0; p < nparts; ++p)
-          tma_load_2d(B + p * part_rows * 128, &tmB, &full[stage], kc * 64,
-                      g.row0 + rb * g.RT + p * part_rows, pol_x);
-        if (++stage == g.nstages) { stage = 0; phase ^= 1; }
-        if (++kc == KC) {
-          kc = 0;
+        stage += np;
+        while (stage >= NS) { stage -= NS; phase ^= 1; }
+        kc += np;
+        while (kc >= KC) {
+          kc -= KC;
           if (++rb == g.row_blocks) { rb = 0; ++nt; }
+        }
+      }
+      if constexpr (kPair == 2) {
+        // The pair's MMA completions arrive on these barriers from the first CTA: wait for the
+        // release of every stage so that no arrival lands after this CTA has exited.
+        if (pidx == 0) {
+          const long long n = u_end - u_begin;
+          for (long long i = n; i < n + NS && !*abort_flag; ++i)
+            if (!mbar_wait(&empty[i % NS], (uint32_t)(((i / NS) & 1) ^ 1), abort_flag, g.status)) break;
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(128, part_rows, 0, 0);
+    if (lane == 0 && leader) {
+      const uint32_t idesc = idesc_bf16(128 * kPair, part_rows, 0, 0);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -179,20 +238,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * g.stage_bytes);
           const uint32_t b_addr = a_addr + kATileBytes;
+          // Straight-line issue (k-steps and parts fully unrolled): control flow between
+          // consecutive tcgen05.mma instructions stalls the issue by tens of cycles each.
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t adesc = sdesc_sw128(a_addr + kk * 32, 16, 1024);
-            for (int p = 0; p < nparts; ++p) {
-              const uint64_t bdesc = sdesc_sw128(b_addr + p * part_rows * 128 + kk * 32, 16, 1024);
-              umma_f16(dcol + p * part_rows, adesc, bdesc, idesc, (first && kk == 0) ? 0u : 1u);
+            const uint32_t accum = (first && kk == 0) ? 0u : 1u;
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+              const uint64_t bdesc = sdesc_sw128(b_addr + p * b_rows * 128 + kk * 32, 16, 1024);
+              const uint32_t d = dcol + p * part_rows;
+              if constexpr (kPair == 2) umma_f16_pair(d, adesc, bdesc, idesc, accum);
+              else umma_f16(d, adesc, bdesc, idesc, accum);
             }
           }
-          umma_commit(&empty[stage]);
+          if constexpr (kPair == 2) umma_commit_pair(&empty[stage]);
+          else umma_commit(&empty[stage]);
           first = false;
           if (++stage == g.nstages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        umma_commit(&acc_full[acc]);
+        if constexpr (kPair == 2) umma_commit_pair(&acc_full[acc]);
+        else umma_commit(&acc_full[acc]);
         if (g.n_acc == 2) {
           acc ^= 1;
           if (acc == 0) acc_phase ^= 1;
@@ -201,11 +268,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
     }
-  } else {
+  } else if (warp >= 2 && warp <= 5) {
     // Epilogue warps 2..5: TMEM lane quarter = warp % 4 -> A-tile row m.
     const int q = warp & 3;
     const int m = q * 32 + lane;
     const int et = threadIdx.x - 64;   // 0..127
+    // the accumulator is free again once all epilogue warps of the pair (or CTA) are done
+    auto acc_release = [&](int a) {
+      if constexpr (kPair == 2) mbar_arrive_cluster(lead_addr(&acc_empty[a]));
+      else mbar_arrive(&acc_empty[a]);
+    };
     int acc = 0;
     uint32_t acc_phase = 0;
     int sbuf = 0;
@@ -217,6 +289,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const long long seg_end = min(u_end, tend);
       const bool full_tile = (u == tstart) && (seg_end == tend);
       const int nt = (int)(tile / g.row_blocks), rb = (int)(tile % g.row_blocks);
+      const int at = nt * kPair + (int)rank;             // this CTA's 128-row weight tile
+      const long long ctile = tile * kPair + rank;       // its fixup counter
       const int rbase = rb * g.RT;                       // first activation row of the block
       const int nvalid_rows = min(g.RT, g.rows - rbase);
       const int nblk = (nvalid_rows + 31) >> 5;
@@ -226,6 +300,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_wait_sleep(&acc_full[acc], acc_phase, abort_flag, g.status);
       tc_fence_after();
       const uint32_t tacc = tbase + (uint32_t(q * 32) << 16) + acc * g.RT;
+      // 32 accumulator columns (activation rows b*32..) of this lane
+      auto ld_acc = [&](int b, float* v) { tmem_ld32(tacc + b * 32, v); };
       // Residual epilogues are additive: split segments add straight into x (fp32 atomics).
       const bool additive = (ep.kind == kEpiResid);
       const bool from_tmem = full_tile || additive;
@@ -243,7 +319,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         g_last = cta_of(tend - 1, U, G);
         const unsigned nseg_u = (unsigned)(g_last - g_first + 1);
         if (et == 0) {
-          const unsigned done = atomicAdd(&g.counters[tile], 0u);
+          const unsigned done = atomicAdd(&g.counters[ctile], 0u);
           *last_flag = (done == nseg_u - 1) ? 2 : 0;
         }
         named_bar_sync(1, 128);
@@ -252,18 +328,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (et == 0) {
             __threadfence();
             asm volatile("fence.proxy.async;" ::: "memory");   // partials are read by bulk copies
-            g.counters[tile] = 0u;                // nobody else touches it in this launch
+            g.counters[ctile] = 0u;               // nobody else touches it in this launch
           }
         } else {
-          const long long me = blockIdx.x;
-          const int slot = (cta_start(me, U, G) < tstart) ? 1 : 0;
-          float* P = g.partial + ((size_t)me * 2 + slot) * (size_t)g.RTp * 128;
+          const int slot = (cta_start(gp, U, G) < tstart) ? 1 : 0;
+          float* P = g.partial + ((size_t)blockIdx.x * 2 + slot) * (size_t)g.RTp * 128;
           for (int b = 0; b < nblk; ++b) {
             float* buf = &staging[b & 1][0][0];
             if (et == 0) bulk_wait_read<1>();    // the store issued from this buffer 2 blocks ago
             named_bar_sync(1, 128);
             float v[32];
-            tmem_ld32(tacc + b * 32, v);
+            ld_acc(b, v);
 #pragma unroll
             for (int j = 0; j < 32; ++j) buf[j * 128 + m] = v[j];
             fence_proxy_async_smem();
@@ -275,14 +350,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          if (lane == 0) acc_release(acc);
           if (et == 0) {
             bulk_wait_all();                      // partial writes performed
             asm volatile("fence.proxy.async;" ::: "memory");
             __threadfence();
-            const unsigned prev = atomicAdd(&g.counters[tile], 1u);
+            const unsigned prev = atomicAdd(&g.counters[ctile], 1u);
             const int is_last = (prev == nseg_u - 1) ? 1 : 0;
-            if (is_last) g.counters[tile] = 0u;   // ready for the next launch
+            if (is_last) g.counters[ctile] = 0u;  // ready for the next launch
             __threadfence();
             asm volatile("fence.proxy.async;" ::: "memory");
             *last_flag = is_last;
@@ -302,11 +377,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           named_bar_sync(1, 128);
         }
         const int nseg = (int)(g_last - g_first + 1);
-        const int own_idx = (int)(blockIdx.x - g_first);
+        const int own_idx = (int)(gp - g_first);
         auto src = [&](int sidx, int b) {
           const long long gg = g_first + sidx;
           const int sl = (cta_start(gg, U, G) < tstart) ? 1 : 0;
-          return g.partial + ((size_t)gg * 2 + sl) * (size_t)g.RTp * 128 + (size_t)b * 32 * 128;
+          const size_t cta = (size_t)gg * kPair + rank;
+          return g.partial + (cta * 2 + sl) * (size_t)g.RTp * 128 + (size_t)b * 32 * 128;
         };
         // Segments to fetch from memory (all but our own when it is still in TMEM).
         const int nfetch = (from_tmem) ? 0 : (own_in_tmem ? nseg - 1 : nseg);
@@ -338,7 +414,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int b = 0; b < nblk; ++b) {
           float v[32];
           if (from_tmem) {
-            tmem_ld32(tacc + b * 32, v);
+            ld_acc(b, v);
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.f;
@@ -347,7 +423,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               for (int sidx = 0; sidx < nseg; ++sidx) {
                 if (own_in_tmem && sidx == own_idx) {
                   float w[32];
-                  tmem_ld32(tacc + b * 32, w);
+                  ld_acc(b, w);
 #pragma unroll
                   for (int j = 0; j < 32; ++j) v[j] += w[j];
                 } else {
@@ -385,7 +461,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               for (int sidx = 0; sidx < nseg; ++sidx) {
                 if (own_in_tmem && sidx == own_idx) {
                   float w[32];
-                  tmem_ld32(tacc + b * 32, w);
+                  ld_acc(b, w);
 #pragma unroll
                   for (int j = 0; j < 32; ++j) v[j] += w[j];
                   continue;
@@ -404,7 +480,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
             }
           }
-          epilogue_block<T>(ep, v, staging[sbuf], nt * 128, rbase + b * 32, m,
+          epilogue_block<T>(ep, v, staging[sbuf], at * 128, rbase + b * 32, m,
                             min(32, nvalid_rows - b * 32), !full_tile, meta_pos, meta_kv, rbase);
           sbuf ^= 1;
           // every thread passed the barrier inside the epilogue, so block b's slots are free
@@ -419,15 +495,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         named_bar_sync(1, 128);   // meta / staging / stages are reused afterwards
       }
-      if (own_in_tmem) {
+      if (own_in_tmem || from_tmem) {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
-      }
-      if (from_tmem) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        if (lane == 0) acc_release(acc);
       }
       if (g.n_acc == 2) {
         acc ^= 1;
@@ -439,9 +510,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair == 2) cluster_sync_all();   // the peer is done with our TMEM and barriers
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tbase, g.tmem_cols);
+    if constexpr (kPair == 2) tmem_dealloc_pair(tbase, g.tmem_cols);
+    else tmem_dealloc(tbase, g.tmem_cols);
   }
 }
 
@@ -506,9 +579,25 @@ int gemm_tc_row_tile(int rows) {
   return 256;
 }
 
-int gemm_tc_box_rows(int rows) {
+int gemm_tc_box_rows(int rows, int pair) {
   const int RT = gemm_tc_row_tile(rows);
-  return RT > 256 ? RT / 2 : RT;
+  return (RT > 256 ? RT / 2 : RT) / pair;
+}
+
+// Process-wide switch for the CTA-pair path: SMDM_GEMM_PAIR=0 forces single CTAs.
+static int pair_enabled() {
+  static int v = [] {
+    const char* e = getenv("SMDM_GEMM_PAIR");
+    return (e && e[0] == '0') ? 0 : 1;
+  }();
+  return v;
+}
+
+int gemm_tc_pair(int n_out, int swiglu, int rows) {
+  (void)rows;
+  const int n_tiles = swiglu ? (n_out + 63) / 64 : (n_out + 127) / 128;
+  // the pair covers two adjacent 128-row weight tiles, so their count must be even
+  return (pair_enabled() && n_tiles % 2 == 0) ? 2 : 1;
 }
 
 static int pow2_ceil(int x) {
@@ -518,9 +607,44 @@ static int pow2_ceil(int x) {
 }
 
 cudaError_t gemm_tc_set_smem_attr() {
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<__nv_bfloat16>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-  return e;
+  const void* fns[4] = {(const void*)gemm_tc_kernel<__nv_bfloat16, 1, 1>,
+                        (const void*)gemm_tc_kernel<__nv_bfloat16, 1, 2>,
+                        (const void*)gemm_tc_kernel<__nv_bfloat16, 2, 1>,
+                        (const void*)gemm_tc_kernel<__nv_bfloat16, 2, 2>};
+  for (const void* f : fns) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+// Co-resident 2-CTA clusters of the pair kernel on the current device (cached per device).
+static int max_pair_clusters(int smem_bytes) {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem_bytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<__nv_bfloat16, 2, 1>, &cfg) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      n = -1;
+    }
+    cached[dev] = n;
+  }
+  return cached[dev];
 }
 
 cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream) {
@@ -534,33 +658,70 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream) {
   g.row_blocks = (c.rows + g.RT - 1) / g.RT;
   g.rows = c.rows;
   g.row0 = c.row0;
-  g.units = (long long)g.n_tiles * g.row_blocks * g.KC;
-  const SmemLayout L = gemm_smem_layout(g.RT, c.max_stages > 0 ? c.max_stages : 8);
+  const int pair = (c.pair == 2) ? 2 : 1;
+  if (pair == 2 && (g.n_tiles & 1)) return cudaErrorInvalidValue;
+  const int pair_tiles = g.n_tiles / pair;     // tiles of pair * 128 weight rows
+  g.units = (long long)pair_tiles * g.row_blocks * g.KC;
+  const SmemLayout L = gemm_smem_layout(g.RT / pair, c.max_stages > 0 ? c.max_stages : 8);
   g.RTp = (g.RT + 31) & ~31;
   g.nstages = L.nstages;
   g.stage_bytes = L.stage_bytes;
   g.staging_off = L.staging_off;
   g.meta_off = L.meta_off;
   g.bar_off = L.bar_off;
-  g.n_acc = (g.RT <= 256) ? 2 : 1;
+  g.np = (c.producers == 1) ? 1 : 2;
+  g.n_acc = (g.RT <= 256) ? 2 : 1;   // double-buffered accumulators where TMEM allows
   g.tmem_cols = pow2_ceil(g.n_acc * g.RT);
   g.partial = c.partial;
   g.counters = c.counters;
   g.status = c.status;
   // Grid: one CTA per SM, units split stream-K style.  When the tile count is close to the SM
   // count, one whole tile per CTA (no split-K fixups, tight tail) beats splitting.
-  long long G = c.num_ctas;
-  const long long tiles_total = (long long)g.n_tiles * g.row_blocks;
-  if (tiles_total <= G && tiles_total * 10 >= G * 6) G = tiles_total;
+  // G counts work groups: CTAs, or CTA pairs in pair mode (no more pairs than can be resident
+  // at once: some GPCs have an odd number of usable SMs).
+  long long G = c.num_ctas / pair;
+  if (pair == 2) {
+    const int mc = max_pair_clusters(L.total);
+    if (mc > 0 && G > mc) G = mc;
+  }
+  const long long tiles_total = (long long)pair_tiles * g.row_blocks;
+  if (c.sched == 1 ? tiles_total <= G
+                   : c.sched == 0 && tiles_total <= G && tiles_total * 10 >= G * 6)
+    G = tiles_total;
   if (G > g.units) G = g.units;
   if (G < 1) G = 1;
   if (g.n_tiles * g.row_blocks > c.max_tiles) return cudaErrorInvalidValue;
-  if ((long long)g.RTp * 128 * 2 * G * 4 > (long long)c.partial_bytes)
+  if ((long long)g.RTp * 128 * 2 * G * pair * 4 > (long long)c.partial_bytes)
     return cudaErrorInvalidValue;  // split-K scratch too small for this row tile
-  gemm_tc_kernel<__nv_bfloat16><<<(unsigned)G, kGemmThreads, L.total, stream>>>(
-      *c.tmA, c.swiglu ? *c.tmA2 : *c.tmA, *c.tmB, g, c.epi);
   // (kEpiQKV requires a rotary-interleaved A map: a_interleave == d_head)
-  return cudaGetLastError();
+  const CUtensorMap& tA2 = c.swiglu ? *c.tmA2 : *c.tmA;
+  const bool two_parts = g.RT > 256;
+  if (pair == 1) {
+    if (two_parts)
+      gemm_tc_kernel<__nv_bfloat16, 1, 2><<<(unsigned)G, kGemmThreads, L.total, stream>>>(
+          *c.tmA, tA2, *c.tmB, g, c.epi);
+    else
+      gemm_tc_kernel<__nv_bfloat16, 1, 1><<<(unsigned)G, kGemmThreads, L.total, stream>>>(
+          *c.tmA, tA2, *c.tmB, g, c.epi);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)(G * 2));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = L.total;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (two_parts)
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<__nv_bfloat16, 2, 2>, *c.tmA, tA2, *c.tmB, g,
+                              c.epi);
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<__nv_bfloat16, 2, 1>, *c.tmA, tA2, *c.tmB, g,
+                            c.epi);
 }
 
 cudaError_t launch_gemm_simt(const float* W, const float* W2, const float* X, int ldx, int K,

@@ -7,7 +7,7 @@ namespace smdm {
 struct GemmCall {
   const CUtensorMap* tmA;   // weights [n_out][K] bf16, box {64, 128} (SwiGLU: gate, box {64, 64})
   const CUtensorMap* tmA2;  // SwiGLU: up weights, box {64, 64}
-  const CUtensorMap* tmB;   // activations [*][K] bf16, box {64, gemm_tc_box_rows(rows)}
+  const CUtensorMap* tmB;   // activations [*][K] bf16, box {64, gemm_tc_box_rows(rows, pair)}
   int K;
   int n_out;                // output features (SwiGLU: ffn)
   int rows;                 // activation rows
@@ -15,7 +15,12 @@ struct GemmCall {
   int swiglu;
   int a_interleave;         // 0, or d_head: tmA is the rotary-interleaved 4-D/5-D QKV map
   int num_ctas;             // persistent grid size (one CTA per SM)
+  int pair;                 // 1: one CTA per tile; 2: CTA pairs (M=256 MMAs, half the
+                            // activation rows per CTA); gemm_tc_pair() picks it
   int max_stages;           // 0 = as many as fit
+  int producers;            // TMA-issuing threads, 1 or 2 (0 = default)
+  int sched;                // 0: whole tiles per CTA when the tile count is 60-100% of the grid,
+                            // else stream-K; 1: whole tiles whenever they fit; 2: stream-K
   float* partial;           // split-K scratch: [num_ctas][2][128][row_tile rounded to 32] fp32
   size_t partial_bytes;
   unsigned* counters;       // [max_tiles], zero-initialised; restored to zero by the kernel
@@ -25,7 +30,9 @@ struct GemmCall {
 };
 
 int gemm_tc_row_tile(int rows);
-int gemm_tc_box_rows(int rows);
+int gemm_tc_box_rows(int rows, int pair);
+// CTA-pair mode (2) or single-CTA mode (1) for a bf16 GEMM of this shape.
+int gemm_tc_pair(int n_out, int swiglu, int rows);
 cudaError_t gemm_tc_set_smem_attr();
 cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream);
 cudaError_t launch_gemm_simt(const float* W, const float* W2, const float* X, int ldx, int K,
