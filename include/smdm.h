@@ -64,7 +64,9 @@ enum { SMDM_PLAN_ORDER = 0, SMDM_PLAN_SEMIAR = 1 };
 /* Model and capacity.  The pages do not describe the base network; the library implements a
  * pre-RMSNorm transformer (multi-head attention with 1-D rotate-half RoPE on the original
  * position ids, SwiGLU MLP, untied LM head).
- * bf16 models need d_model % 128 == 0, d_head in {64, 128}, d_ffn % 64 == 0. */
+ * bf16 models need d_model % 128 == 0, d_head in {64, 128}, d_ffn % 64 == 0 and vocab % 4 == 0
+ * (logit rows are written with 16-byte-aligned bulk copies; logit buffers passed to the
+ * library must be 16-byte aligned). */
 typedef struct {
   int n_layers, d_model, n_heads, d_head, d_ffn;
   int vocab;         /* content vocabulary V */

@@ -51,6 +51,49 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
   return r == CUDA_SUCCESS;
 }
 
+// Interleaved gate/up view for the SwiGLU GEMM's A tiles: one 3-D map {d, 2, ffn} over both
+// weight tensors (the second dimension steps from the lower of the two base addresses to the
+// higher), box {64, 2, 64}, so that a 16 KB tile holds gate row f0 + i and up row f0 + i on
+// adjacent rows 2i, 2i + 1.  Returns 0 when the address gap is unusable as a TMA stride (then
+// the two-box layout is used), 1 when gate comes first, 2 when up comes first.
+int encode_gateup_interleaved(CUtensorMap* m, const void* gate, const void* up, uint64_t d,
+                              uint64_t f) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return 0;
+  const uintptr_t g = reinterpret_cast<uintptr_t>(gate), u = reinterpret_cast<uintptr_t>(up);
+  const bool up_first = u < g;
+  const uint64_t delta = up_first ? g - u : u - g;
+  if (delta == 0 || delta % 16 || delta >= (1ull << 40)) return 0;
+  cuuint64_t dims[3] = {d, 2, f};
+  cuuint64_t strides[2] = {delta, d * 2};
+  cuuint32_t box[3] = {64, 2, 64};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(up_first ? up : gate), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return 0;
+  return up_first ? 2 : 1;
+}
+
+// 2-D output map for the GEMM epilogue's TMA stores: `cols` x `rows` elements (bf16 or fp32),
+// row pitch `ld` elements, box {box_cols, 32}, no swizzle.
+bool encode_out(CUtensorMap* m, const void* base, bool f32, uint64_t cols, uint64_t rows,
+                uint64_t ld, uint32_t box_cols) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn || !base || rows == 0) return false;
+  const uint64_t es = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * es};
+  cuuint32_t box[2] = {box_cols, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Rotary-interleaved view of W_qkv [3d][d] for the GEMM's A tiles: a 128-row tile is loaded so
 // that A-tile row 2i holds weight row i of the first half of a head and row 2i + 1 the matching
 // row of the second half (the RoPE partner), putting the two on adjacent TMEM lanes.
@@ -109,6 +152,7 @@ bool config_ok(const smdm_config* c, std::string* why) {
     if (c->d_model % 128) return fail("bf16 models need d_model % 128 == 0");
     if (c->d_head != 64 && c->d_head != 128) return fail("bf16 models need d_head 64 or 128");
     if (c->d_ffn % 64) return fail("bf16 models need d_ffn % 64 == 0");
+    if (c->vocab % 4) return fail("bf16 models need vocab % 4 == 0");
   } else if (c->dtype == SMDM_F32) {
     if (c->d_head % 32 || c->d_head > 128) return fail("fp32 models need d_head % 32 == 0, <= 128");
   } else {
@@ -207,7 +251,8 @@ struct smdm_handle {
   std::vector<const void*> attn_norm, w_qkv, w_o, mlp_norm, w_gate, w_up, w_down;
   uint8_t* ws;
   Rows rows, aux;
-  std::vector<CUtensorMap> tm_qkv, tm_o, tm_gate, tm_up, tm_down;
+  std::vector<CUtensorMap> tm_qkv, tm_o, tm_gate, tm_up, tm_down, tm_gu;
+  std::vector<int> gu_il;   // per layer: 0 two-box gate/up tiles, 1/2 interleaved (tm_gu)
   CUtensorMap tm_lm, tm_kc, tm_vc, tm_kscr, tm_vscr, tm_q;
   std::string err;
   SeqState seq[SMDM_MAX_BATCH];
@@ -332,7 +377,22 @@ smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensor
     const int pair = gemm_tc_pair(n_out, swiglu, rows);
     if (!encode_2d(&tmB, X, K, MR, (uint64_t)K * 2, 64, gemm_tc_box_rows(rows, pair)))
       return fail(h, SMDM_ECUDA, "cuTensorMapEncodeTiled failed for an activation operand");
+    CUtensorMap tmOut;
+    bool ok_out = false;
+    switch (ep.kind) {
+      case kEpiStore: ok_out = encode_out(&tmOut, ep.out, false, ep.n_valid, rows, ep.ld_out, 128); break;
+      case kEpiQKV: ok_out = encode_out(&tmOut, ep.q_out, false, ep.d_model, rows, ep.d_model, 128); break;
+      case kEpiSwiGLU: ok_out = encode_out(&tmOut, ep.act, false, ep.n_valid, rows, ep.ld_act, 64); break;
+      case kEpiResid: ok_out = encode_out(&tmOut, ep.x, true, ep.n_valid, rows, ep.ld_x, 128); break;
+      case kEpiLMHead:
+        // without logits the map is never used: any valid fp32 map will do
+        ok_out = ep.logits ? encode_out(&tmOut, ep.logits, true, ep.n_valid, rows, ep.ld_logits, 128)
+                           : encode_out(&tmOut, ep.pmax, true, 128, 32, 128, 128);
+        break;
+    }
+    if (!ok_out) return fail(h, SMDM_ECUDA, "cuTensorMapEncodeTiled failed for a GEMM output");
     GemmCall c{};
+    c.tmOut = &tmOut;
     c.pair = pair;
     c.tmA = tmA;
     c.tmA2 = tmA2;
@@ -342,6 +402,7 @@ smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensor
     c.rows = rows;
     c.row0 = 0;
     c.swiglu = swiglu;
+    c.swiglu_il = swiglu && ep.swiglu_il;
     c.a_interleave = a_interleave;
     c.num_ctas = h->L.n_sms;
     c.partial = h->at<float>(h->L.partial);
@@ -469,7 +530,11 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
     eg.n_valid = c.d_ffn;
     eg.act = act;
     eg.ld_act = c.d_ffn;
-    if ((s = gemm(h, SMDM_K_GEMM_GATEUP, h->bf16 ? &h->tm_gate[l] : nullptr, h->bf16 ? &h->tm_up[l] : nullptr,
+    const bool il = h->bf16 && h->gu_il[l] != 0;
+    eg.swiglu_il = il ? 1 : 0;
+    eg.swiglu_up_first = (il && h->gu_il[l] == 2) ? 1 : 0;
+    if ((s = gemm(h, SMDM_K_GEMM_GATEUP, h->bf16 ? (il ? &h->tm_gu[l] : &h->tm_gate[l]) : nullptr,
+                  h->bf16 ? &h->tm_up[l] : nullptr,
                   h->w_gate[l], h->w_up[l], hb, d, c.d_ffn, R, 1, eg, st)))
       return s;
     // down + residual
@@ -619,12 +684,15 @@ smdm_status smdm_create(const smdm_config* cfg, const smdm_weights* w, void* d_w
     h->tm_o.resize(nl);
     h->tm_gate.resize(nl);
     h->tm_up.resize(nl);
+    h->tm_gu.resize(nl);
+    h->gu_il.assign(nl, 0);
     h->tm_down.resize(nl);
     for (int l = 0; l < nl; ++l) {
       ok &= encode_qkv_interleaved(&h->tm_qkv[l], w->w_qkv[l], d, dh);
       ok &= encode_2d(&h->tm_o[l], w->w_o[l], d, d, (uint64_t)d * 2, 64, 128);
       ok &= encode_2d(&h->tm_gate[l], w->w_gate[l], d, f, (uint64_t)d * 2, 64, 64);
       ok &= encode_2d(&h->tm_up[l], w->w_up[l], d, f, (uint64_t)d * 2, 64, 64);
+      h->gu_il[l] = encode_gateup_interleaved(&h->tm_gu[l], w->w_gate[l], w->w_up[l], d, f);
       ok &= encode_2d(&h->tm_down[l], w->w_down[l], f, d, (uint64_t)f * 2, 64, 128);
     }
     ok &= encode_2d(&h->tm_lm, w->lm_head, d, cfg->vocab, (uint64_t)d * 2, 64, 128);
@@ -1147,12 +1215,15 @@ extern "C" smdm_status smdm_forward_stepcausal_noalloc(
     h->tm_o.resize(nl);
     h->tm_gate.resize(nl);
     h->tm_up.resize(nl);
+    h->tm_gu.resize(nl);
+    h->gu_il.assign(nl, 0);
     h->tm_down.resize(nl);
     for (int l = 0; l < nl; ++l) {
       ok &= encode_qkv_interleaved(&h->tm_qkv[l], w->w_qkv[l], d, dh);
       ok &= encode_2d(&h->tm_o[l], w->w_o[l], d, d, (uint64_t)d * 2, 64, 128);
       ok &= encode_2d(&h->tm_gate[l], w->w_gate[l], d, f, (uint64_t)d * 2, 64, 64);
       ok &= encode_2d(&h->tm_up[l], w->w_up[l], d, f, (uint64_t)d * 2, 64, 64);
+      h->gu_il[l] = encode_gateup_interleaved(&h->tm_gu[l], w->w_gate[l], w->w_up[l], d, f);
       ok &= encode_2d(&h->tm_down[l], w->w_down[l], f, d, (uint64_t)f * 2, 64, 128);
     }
     ok &= encode_2d(&h->tm_lm, w->lm_head, d, vc.vocab, (uint64_t)d * 2, 64, 128);

@@ -56,7 +56,8 @@ struct GemmDev {
   int row0;        // first activation row (TMA y offset)
   long long units; // n_tiles * row_blocks * KC
   int swiglu;
-  int a_mode;      // 0: 2-D box {64,128}; 1: SwiGLU gate+up boxes {64,64};
+  int a_mode;      // 0: 2-D box {64,128}; 1: SwiGLU gate+up boxes {64,64}; 4: SwiGLU
+                   // interleaved 3-D box {64,2,64};
                    // 2: 4-D rotary interleave (d_head 128); 3: 5-D rotary interleave (d_head 64)
   int RTp;         // partial-sum row stride (RT rounded up to 32)
   int np;          // TMA producer threads (1 or 2; stages alternate between them)
@@ -79,7 +80,8 @@ SMDM_DEV long long cta_of(long long u, long long U, long long G) { return ((u + 
 template <typename T, int kPair, int NP>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
-                   const __grid_constant__ CUtensorMap tmB, const GemmDev g, const EpiParams ep) {
+                   const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmOut,
+                   const GemmDev g, const EpiParams ep) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -115,7 +117,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (g.swiglu) tma_prefetch_desc(&tmA2);
+    tma_prefetch_desc(&tmOut);
+    if (g.a_mode == 1) tma_prefetch_desc(&tmA2);
   }
   // Pair: both CTAs are running and their barriers initialised before any cross-CTA signal or
   // the pair's joint TMEM allocation (one warp in each CTA allocates collectively).
@@ -168,7 +171,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int at = nt * kPair + (int)rank;    // this CTA's 128-row A tile
         if constexpr (kPair == 1) {
           mbar_arrive_expect_tx(&full[stage], g.stage_bytes);
-          if (g.a_mode == 1) {
+          if (g.a_mode == 4) {
+            tma_load_3d(A, &tmA, &full[stage], kc * 64, 0, at * 64, pol_w);
+          } else if (g.a_mode == 1) {
             tma_load_2d(A, &tmA, &full[stage], kc * 64, at * 64, pol_w);
             tma_load_2d(A + kATileBytes / 2, &tmA2, &full[stage], kc * 64, at * 64, pol_w);
           } else if (g.a_mode == 2) {
@@ -185,7 +190,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           // both CTAs' bytes complete on the first CTA's barrier, which expects them all
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * g.stage_bytes);
           const uint32_t fb = lead_addr(&full[stage]);
-          if (g.a_mode == 1) {
+          if (g.a_mode == 4) {
+            tma_load_3d_pair(A, &tmA, fb, kc * 64, 0, at * 64, pol_w);
+          } else if (g.a_mode == 1) {
             tma_load_2d_pair(A, &tmA, fb, kc * 64, at * 64, pol_w);
             tma_load_2d_pair(A + kATileBytes / 2, &tmA2, fb, kc * 64, at * 64, pol_w);
           } else if (g.a_mode == 2) {
@@ -333,28 +340,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         } else {
           const int slot = (cta_start(gp, U, G) < tstart) ? 1 : 0;
           float* P = g.partial + ((size_t)blockIdx.x * 2 + slot) * (size_t)g.RTp * 128;
+          // Direct stores from registers: for accumulator column j the 128 lanes write 512
+          // contiguous bytes ([column][row] blocks, the layout the summing CTA loads in bulk).
+          // This keeps the SM's copy engine, busy with the next segment's loads, out of it.
           for (int b = 0; b < nblk; ++b) {
-            float* buf = &staging[b & 1][0][0];
-            if (et == 0) bulk_wait_read<1>();    // the store issued from this buffer 2 blocks ago
-            named_bar_sync(1, 128);
             float v[32];
             ld_acc(b, v);
+            float* Pb = P + (size_t)b * 32 * 128 + m;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) buf[j * 128 + m] = v[j];
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (et == 0) {
-              bulk_store(P + (size_t)b * 32 * 128, buf, 32 * 128 * 4);
-              bulk_commit();
-            }
+            for (int j = 0; j < 32; ++j) Pb[j * 128] = v[j];
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) acc_release(acc);
+          __threadfence();                        // this thread's partial stores are visible
+          named_bar_sync(1, 128);
           if (et == 0) {
-            bulk_wait_all();                      // partial writes performed
             asm volatile("fence.proxy.async;" ::: "memory");
-            __threadfence();
             const unsigned prev = atomicAdd(&g.counters[ctile], 1u);
             const int is_last = (prev == nseg_u - 1) ? 1 : 0;
             if (is_last) g.counters[ctile] = 0u;  // ready for the next launch
@@ -450,6 +452,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 return -1;
               };
               if (et == 0) {
+                bulk_wait_read<0>();   // output copies issued from these buffers are done reading
                 for (int k = 0; k < min(2, nfetch); ++k) {
                   mbar_arrive_expect_tx(&io_bar[k], 16384);
                   bulk_load(&staging[k][0][0], src(fetch_index(k), b), 16384, &io_bar[k]);
@@ -480,8 +483,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
             }
           }
-          epilogue_block<T>(ep, v, staging[sbuf], at * 128, rbase + b * 32, m,
-                            min(32, nvalid_rows - b * 32), !full_tile, meta_pos, meta_kv, rbase);
+          epilogue_block<T>(ep, &tmOut, v, reinterpret_cast<uint8_t*>(&staging[sbuf][0][0]),
+                            at * 128, rbase + b * 32, m, et, min(32, nvalid_rows - b * 32),
+                            meta_pos, meta_kv, rbase);
           sbuf ^= 1;
           // every thread passed the barrier inside the epilogue, so block b's slots are free
           if (use_ring && et == 0) {
@@ -493,6 +497,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         }
+        if (et == 0) bulk_wait_read<0>();   // staging buffers are free once the copies read them
         named_bar_sync(1, 128);   // meta / staging / stages are reused afterwards
       }
       if (own_in_tmem || from_tmem) {
@@ -507,6 +512,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         acc_phase ^= 1;
       }
     }
+    if (et == 0) bulk_wait_all();   // output copies complete before the CTA exits
   }
   tc_fence_before();
   __syncthreads();
@@ -652,7 +658,7 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream) {
   GemmDev g{};
   g.KC = c.K / 64;
   g.swiglu = c.swiglu;
-  g.a_mode = c.swiglu ? 1 : c.a_interleave == 128 ? 2 : c.a_interleave == 64 ? 3 : 0;
+  g.a_mode = c.swiglu ? (c.swiglu_il ? 4 : 1) : c.a_interleave == 128 ? 2 : c.a_interleave == 64 ? 3 : 0;
   g.n_tiles = c.swiglu ? (c.n_out + 63) / 64 : (c.n_out + 127) / 128;
   g.RT = gemm_tc_row_tile(c.rows);
   g.row_blocks = (c.rows + g.RT - 1) / g.RT;
@@ -691,18 +697,21 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream) {
   if (G > g.units) G = g.units;
   if (G < 1) G = 1;
   if (g.n_tiles * g.row_blocks > c.max_tiles) return cudaErrorInvalidValue;
+  // 32-row output blocks of a row tile must not reach into the next row tile
+  if (g.row_blocks > 1 && (g.RT & 31)) return cudaErrorInvalidValue;
+  if (!c.tmOut) return cudaErrorInvalidValue;
   if ((long long)g.RTp * 128 * 2 * G * pair * 4 > (long long)c.partial_bytes)
     return cudaErrorInvalidValue;  // split-K scratch too small for this row tile
   // (kEpiQKV requires a rotary-interleaved A map: a_interleave == d_head)
-  const CUtensorMap& tA2 = c.swiglu ? *c.tmA2 : *c.tmA;
+  const CUtensorMap& tA2 = (c.swiglu && !c.swiglu_il) ? *c.tmA2 : *c.tmA;
   const bool two_parts = g.RT > 256;
   if (pair == 1) {
     if (two_parts)
       gemm_tc_kernel<__nv_bfloat16, 1, 2><<<(unsigned)G, kGemmThreads, L.total, stream>>>(
-          *c.tmA, tA2, *c.tmB, g, c.epi);
+          *c.tmA, tA2, *c.tmB, *c.tmOut, g, c.epi);
     else
       gemm_tc_kernel<__nv_bfloat16, 1, 1><<<(unsigned)G, kGemmThreads, L.total, stream>>>(
-          *c.tmA, tA2, *c.tmB, g, c.epi);
+          *c.tmA, tA2, *c.tmB, *c.tmOut, g, c.epi);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg{};
@@ -718,10 +727,10 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (two_parts)
-    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<__nv_bfloat16, 2, 2>, *c.tmA, tA2, *c.tmB, g,
-                              c.epi);
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<__nv_bfloat16, 2, 1>, *c.tmA, tA2, *c.tmB, g,
-                            c.epi);
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<__nv_bfloat16, 2, 2>, *c.tmA, tA2, *c.tmB,
+                              *c.tmOut, g, c.epi);
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<__nv_bfloat16, 2, 1>, *c.tmA, tA2, *c.tmB,
+                            *c.tmOut, g, c.epi);
 }
 
 cudaError_t launch_gemm_simt(const float* W, const float* W2, const float* X, int ldx, int K,

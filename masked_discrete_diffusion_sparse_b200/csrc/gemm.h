@@ -6,13 +6,21 @@ namespace smdm {
 
 struct GemmCall {
   const CUtensorMap* tmA;   // weights [n_out][K] bf16, box {64, 128} (SwiGLU: gate, box {64, 64})
-  const CUtensorMap* tmA2;  // SwiGLU: up weights, box {64, 64}
+  const CUtensorMap* tmA2;  // SwiGLU: up weights, box {64, 64} (split layout)
+                            // interleaved layout: tmA = 3-D map {d, 2 (gate/up), ffn}, box
+                            // {64, 2, 64}: A-tile row 2i / 2i+1 = gate / up row f0 + i
   const CUtensorMap* tmB;   // activations [*][K] bf16, box {64, gemm_tc_box_rows(rows, pair)}
+  const CUtensorMap* tmOut; // epilogue output, rows = `rows` (no swizzle), box {w, 32}:
+                            //   store: out bf16 [rows][n_out], w 128;  QKV: q bf16 [rows][d], w 128;
+                            //   SwiGLU: act bf16 [rows][ffn], w 64;  residual: x fp32 [rows][d],
+                            //   w 128 (reduce-add);  LM head: logits fp32 [rows][V], w 128 (or any
+                            //   valid map when no logits are written)
   int K;
   int n_out;                // output features (SwiGLU: ffn)
   int rows;                 // activation rows
   int row0;                 // first activation row in tmB
-  int swiglu;
+  int swiglu;               // 1: gate/up tiles with the SwiGLU epilogue
+  int swiglu_il;            // SwiGLU: tmA is the interleaved gate/up map (tmA2 unused)
   int a_interleave;         // 0, or d_head: tmA is the rotary-interleaved 4-D/5-D QKV map
   int num_ctas;             // persistent grid size (one CTA per SM)
   int pair;                 // 1: one CTA per tile; 2: CTA pairs (M=256 MMAs, half the

@@ -77,9 +77,12 @@ struct EpiParams {
   // kEpiResid: x[r][n] += acc (fp32 residual stream)
   float* x;
   int ld_x;
-  // kEpiSwiGLU: act[r][f] = silu(gate) * up; tile = 64 gate rows then 64 up rows
+  // kEpiSwiGLU: act[r][f] = silu(gate) * up; tile = 64 gate rows then 64 up rows, or with
+  // swiglu_il the gate and up rows of feature f0 + i on lanes 2i and 2i + 1 (swapped when
+  // swiglu_up_first)
   void* act;
   int ld_act;
+  int swiglu_il, swiglu_up_first;
   // kEpiLMHead
   float* logits;     // optional [rows][ld_logits]
   int ld_logits;
@@ -89,7 +92,16 @@ struct EpiParams {
   int n_vt;
 };
 
-SMDM_DEV float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+// silu(g) = g * sigmoid(g) with the fast division (a full-precision division takes a slow
+// software path)
+SMDM_DEV float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+// silu for bf16 outputs: sigmoid(g) = (1 + tanh(g / 2)) / 2 with the hardware tanh
+// approximation (one special-function op instead of two; its error is far below bf16 rounding)
+SMDM_DEV float silu_bf16out(float g) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * g));
+  return g * fmaf(0.5f, t, 0.5f);
+}
 
 // Apply the epilogue to a staged tile S[16][128] (S[j][m] = accumulator for activation row
 // r0 + j and output feature n0 + m; for SwiGLU m < 64 are gate rows f0 + m and m >= 64 the up
@@ -234,13 +246,11 @@ SMDM_DEV void epilogue_tile(const EpiParams& p, const float (*S)[128], int n0, i
 }
 
 // ------------------------------------------------------------------------------------------
-// Register epilogue of the tcgen05 GEMM: one block of 32 activation rows (TMEM columns) for the
-// A-tile row held by TMEM lane m; v[j] = accumulator of activation row r0 + j.
+// Epilogue of the tcgen05 GEMM: TMEM lane m holds A-tile row m (an output feature) and TMEM
+// columns are activation rows.
 //   - QKV tiles are loaded with rotary partners interleaved (A-tile row 2i <- weight row i of
 //     the first half of a head, row 2i + 1 <- row i of the second half), so the rotation needs
 //     only a lane exchange with lane m ^ 1.
-//   - SwiGLU and the LM-head statistics combine values of different lanes through `stage`
-//     ([32][128] fp32 shared memory, one barrier per block, callers alternate two buffers).
 //   - meta_pos / meta_kv: per-row position and K/V cache offset of the tile's rows (shared
 //     memory, filled once per tile), indexed by row - meta_r0.
 // ------------------------------------------------------------------------------------------
@@ -249,141 +259,155 @@ SMDM_DEV int qkv_lane_feature(int m, int d_head) {
   return (m >> 6) * 64 + (m & 1) * 32 + ((m >> 1) & 31);     // d_head == 64
 }
 
-SMDM_DEV void store8(__nv_bfloat16* dst, const float* f) {
-  __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]), b = __floats2bfloat162_rn(f[2], f[3]),
-                 c = __floats2bfloat162_rn(f[4], f[5]), d = __floats2bfloat162_rn(f[6], f[7]);
-  uint4 u;
-  u.x = *reinterpret_cast<uint32_t*>(&a);
-  u.y = *reinterpret_cast<uint32_t*>(&b);
-  u.z = *reinterpret_cast<uint32_t*>(&c);
-  u.w = *reinterpret_cast<uint32_t*>(&d);
-  *reinterpret_cast<uint4*>(dst) = u;
-}
-
-// Epilogue of one block of 32 activation rows.  v[j]: accumulator of row r0 + j for A-tile row
-// m (TMEM lane).  Register step: rotary on q/k (lane pairs m, m ^ 1 hold x_i, x_{i+d/2}).
-// Then the block is staged in shared memory as S[32 rows][128 features] and written row-major
-// with 16-byte vectors (scattered 2-byte stores would stall on outstanding-request slots).
-// One named barrier (128 epilogue threads); callers alternate two staging buffers.
+// Epilogue of one block of 32 activation rows, written out through shared memory with TMA
+// stores (one copy per block instead of hundreds of per-thread stores).  v[j]: accumulator of
+// activation row r0 + j for A-tile row m (TMEM lane m).  buf: the block's 16 KB staging buffer;
+// callers alternate two, and since et == 0 waits for its earlier copies to finish reading
+// shared memory before the block's barrier, a buffer is free again two blocks later.  All 128
+// epilogue threads call this (et = 0..127); et == 0 issues the copies.  tm_out: the call's
+// output tensor map (bf16 out / q / act boxes of 32 rows, fp32 x / logits boxes of 32 rows);
+// K/V cache rows of QKV tiles go out as 1-D bulk copies, one per run of consecutive slots.
+// Output rows at or beyond the map's row count are clipped by the TMA unit.
 template <typename T>
-SMDM_DEV void epilogue_block(const EpiParams& p, float* v, float (*S)[128], int n0, int r0, int m,
-                             int nrows, bool atomic_resid, const int* meta_pos,
+SMDM_DEV void epilogue_block(const EpiParams& p, const CUtensorMap* tm_out, float* v, uint8_t* buf,
+                             int n0, int r0, int m, int et, int nrows, const int* meta_pos,
                              const long long* meta_kv, int meta_r0) {
-  int f = m;   // feature (0..127 within the tile) held by this lane
-  if (p.kind == kEpiQKV) {
-    const int dh = p.d_head, half = dh >> 1;
-    f = qkv_lane_feature(m, dh);
-    const int region = n0 / p.d_model;
-    if (region < 2) {
-      const int ih = (f % dh) % half;
-      const bool second = (m & 1) != 0;
+  auto publish = [&]() {   // staged data visible to the async proxy; earlier copies done reading
+    fence_proxy_async_smem();
+    if (et == 0) bulk_wait_read<0>();
+    named_bar_sync(1, 128);
+  };
+  switch (p.kind) {
+    case kEpiQKV: {
+      const int dh = p.d_head, half = dh >> 1;
+      const int f = qkv_lane_feature(m, dh);
+      const int region = n0 / p.d_model;
+      const int nn0 = n0 - region * p.d_model;
+      if (region < 2) {
+        const int ih = (f % dh) % half;
+        const bool second = (m & 1) != 0;
 #pragma unroll
-      for (int g = 0; g < 32; g += 8) {
-        float2 cs[8];
+        for (int g = 0; g < 32; g += 8) {
+          float2 cs[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int jj = min(g + j, nrows - 1);
-          cs[j] = __ldg(p.rope + (size_t)meta_pos[r0 + jj - meta_r0] * half + ih);
-        }
+          for (int j = 0; j < 8; ++j) {
+            const int jj = min(g + j, nrows - 1);
+            cs[j] = __ldg(p.rope + (size_t)meta_pos[r0 + jj - meta_r0] * half + ih);
+          }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float a = v[g + j];
-          const float b = __shfl_xor_sync(0xffffffffu, a, 1);
-          v[g + j] = second ? (b * cs[j].y + a * cs[j].x) : (a * cs[j].x - b * cs[j].y);
+          for (int j = 0; j < 8; ++j) {
+            const float a = v[g + j];
+            const float b = __shfl_xor_sync(0xffffffffu, a, 1);
+            v[g + j] = second ? (b * cs[j].y + a * cs[j].x) : (a * cs[j].x - b * cs[j].y);
+          }
         }
       }
-    }
-  }
+      // q: [32 rows][128 features]; k / v: [head within the tile][32 rows][d_head]
+      __nv_bfloat16* Sb = reinterpret_cast<__nv_bfloat16*>(buf);
+      const int hh = f / dh;
+      __nv_bfloat16* dst = (region == 0) ? Sb + f : Sb + hh * 32 * dh + (f - hh * dh);
+      const int stride = (region == 0) ? 128 : dh;
 #pragma unroll
-  for (int j = 0; j < 32; ++j) S[j][f] = v[j];
-  named_bar_sync(1, 128);
-  const int t = m;   // 0..127 consumer index
-  switch (p.kind) {
-    case kEpiStore: {
-      T* out = reinterpret_cast<T*>(p.out);
-      if constexpr (sizeof(T) == 2) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int idx = t + 128 * q, j = idx >> 4, c = (idx & 15) * 8;
-          if (j < nrows && n0 + c < p.n_valid)
-            store8(reinterpret_cast<__nv_bfloat16*>(out) + (size_t)(r0 + j) * p.ld_out + n0 + c, &S[j][c]);
+      for (int j = 0; j < 32; ++j) dst[j * stride] = __float2bfloat16_rn(v[j]);
+      publish();
+      if (et == 0) {
+        if (region == 0) {
+          tma_store_2d(tm_out, Sb, nn0, r0);
+        } else {
+          const long long base = (long long)p.layer * p.kv.layer_stride +
+                                 (long long)(nn0 / dh) * p.kv.head_stride;
+          __nv_bfloat16* cache =
+              reinterpret_cast<__nv_bfloat16*>(region == 1 ? p.kv.k : p.kv.v) + base;
+          int j0 = 0;
+          while (j0 < nrows) {
+            const long long o0 = meta_kv[r0 + j0 - meta_r0];
+            int j1 = j0 + 1;
+            while (j1 < nrows && meta_kv[r0 + j1 - meta_r0] == o0 + (long long)(j1 - j0) * dh) ++j1;
+            for (int h = 0; h < 128 / dh; ++h)
+              bulk_store(cache + (long long)h * p.kv.head_stride + o0, Sb + (h * 32 + j0) * dh,
+                         (uint32_t)((j1 - j0) * dh * 2));
+            j0 = j1;
+          }
         }
+        bulk_commit();
       }
       break;
     }
-    case kEpiQKV: {
-      const int dh = p.d_head;
-      const int region = n0 / p.d_model;
-      const int nn0 = n0 - region * p.d_model;
+    case kEpiStore: {
+      __nv_bfloat16* Sb = reinterpret_cast<__nv_bfloat16*>(buf);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int idx = t + 128 * q, j = idx >> 4, c = (idx & 15) * 8;
-        if (j >= nrows) continue;
-        __nv_bfloat16* dst;
-        if (region == 0) {
-          dst = reinterpret_cast<__nv_bfloat16*>(p.q_out) + (size_t)(r0 + j) * p.d_model + nn0 + c;
-        } else {
-          const int h = (nn0 + c) / dh, i = (nn0 + c) % dh;
-          dst = reinterpret_cast<__nv_bfloat16*>(region == 1 ? p.kv.k : p.kv.v) +
-                (long long)p.layer * p.kv.layer_stride + (long long)h * p.kv.head_stride +
-                meta_kv[r0 + j - meta_r0] + i;
-        }
-        store8(dst, &S[j][c]);
+      for (int j = 0; j < 32; ++j) Sb[j * 128 + m] = __float2bfloat16_rn(v[j]);
+      publish();
+      if (et == 0) {
+        tma_store_2d(tm_out, Sb, n0, r0);
+        bulk_commit();
       }
       break;
     }
     case kEpiResid: {
+      float* S = reinterpret_cast<float*>(buf);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int idx = t + 128 * q, j = idx >> 5, c = (idx & 31) * 4;
-        if (j >= nrows || n0 + c >= p.n_valid) continue;
-        float* x = p.x + (size_t)(r0 + j) * p.ld_x + n0 + c;
-        const float4 a = *reinterpret_cast<const float4*>(&S[j][c]);
-        if (atomic_resid) {
-          asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(x), "f"(a.x),
-                       "f"(a.y), "f"(a.z), "f"(a.w)
-                       : "memory");
-        } else {
-          float4 o = *reinterpret_cast<const float4*>(x);
-          o.x += a.x;
-          o.y += a.y;
-          o.z += a.z;
-          o.w += a.w;
-          *reinterpret_cast<float4*>(x) = o;
-        }
+      for (int j = 0; j < 32; ++j) S[j * 128 + m] = v[j];
+      publish();
+      if (et == 0) {
+        tma_reduce_add_2d(tm_out, S, n0, r0);   // x += block (fp32, element-wise atomic)
+        bulk_commit();
       }
       break;
     }
     case kEpiSwiGLU: {
-      // features 0..63 = gate rows f0 + i, 64..127 = up rows f0 + i
+      if (p.swiglu_il) {
+        // the partner lane m ^ 1 holds the other half of the pair; lane parity picks the rows
+        // (even lanes even rows) so that the work splits evenly, with no shared-memory exchange
+        __nv_bfloat16* Ob = reinterpret_cast<__nv_bfloat16*>(buf);   // [32][64] bf16
+        const int i = m >> 1, h = m & 1;
+        const bool mine_is_gate = (h == (p.swiglu_up_first ? 1 : 0));
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int idx = t + 128 * q, j = idx >> 3, c = (idx & 7) * 8;
-        if (j >= nrows || (n0 >> 1) + c >= p.n_valid) continue;
-        float o[8];
+        for (int j = 0; j < 32; j += 2) {   // even lanes take row j, odd lanes row j + 1
+          const float o0 = __shfl_xor_sync(0xffffffffu, v[j], 1);
+          const float o1 = __shfl_xor_sync(0xffffffffu, v[j + 1], 1);
+          const float mine = h ? v[j + 1] : v[j];
+          const float other = h ? o1 : o0;
+          const float gate = mine_is_gate ? mine : other;
+          const float up = mine_is_gate ? other : mine;
+          Ob[(j + h) * 64 + i] = __float2bfloat16_rn(silu_bf16out(gate) * up);
+        }
+        publish();
+        if (et == 0) {
+          tma_store_2d(tm_out, Ob, n0 >> 1, r0);
+          bulk_commit();
+        }
+        break;
+      }
+      // lanes 0..63: gate rows f0 + m; lanes 64..127: up rows f0 + m - 64 (f0 = n0 / 2)
+      float* U = reinterpret_cast<float*>(buf);                               // [32][64] fp32
+      __nv_bfloat16* Ob = reinterpret_cast<__nv_bfloat16*>(buf + 32 * 64 * 4);  // [32][64] bf16
+      if (m >= 64) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = silu_f(S[j][c + e]) * S[j][64 + c + e];
-        if constexpr (sizeof(T) == 2)
-          store8(reinterpret_cast<__nv_bfloat16*>(p.act) + (size_t)(r0 + j) * p.ld_act + (n0 >> 1) + c, o);
+        for (int j = 0; j < 32; ++j) U[j * 64 + (m - 64)] = v[j];
+      }
+      named_bar_sync(1, 128);
+      if (m < 64) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) Ob[j * 64 + m] = __float2bfloat16_rn(silu_bf16out(v[j]) * U[j * 64 + m]);
+      }
+      publish();
+      if (et == 0) {
+        tma_store_2d(tm_out, Ob, n0 >> 1, r0);
+        bulk_commit();
       }
       break;
     }
     case kEpiLMHead: {
-      if (p.logits) {
+      float* S = reinterpret_cast<float*>(buf);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int idx = t + 128 * q, j = idx >> 5, c = (idx & 31) * 4;
-          if (j >= nrows) continue;
-          float* dst = p.logits + (size_t)(r0 + j) * p.ld_logits + n0 + c;
-          if (n0 + c + 4 <= p.n_valid && (p.ld_logits & 3) == 0) {
-            *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(&S[j][c]);
-          } else {
-            for (int e = 0; e < 4; ++e)
-              if (n0 + c + e < p.n_valid) dst[e] = S[j][c + e];
-          }
-        }
+      for (int j = 0; j < 32; ++j) S[j * 128 + m] = v[j];
+      publish();
+      if (p.logits && et == 0) {
+        tma_store_2d(tm_out, S, n0, r0);
+        bulk_commit();
       }
-      const int warp = t >> 5, lane = t & 31;
+      const int warp = et >> 5, lane = et & 31;
       const int vt = n0 >> 7;
       for (int j = warp * 8; j < min(warp * 8 + 8, nrows); ++j) {
         float best = -INFINITY;
@@ -391,7 +415,7 @@ SMDM_DEV void epilogue_block(const EpiParams& p, float* v, float (*S)[128], int 
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int ff = lane + 32 * u;
-          const float x = (n0 + ff < p.n_valid) ? S[j][ff] : -INFINITY;
+          const float x = (n0 + ff < p.n_valid) ? S[j * 128 + ff] : -INFINITY;
           if (x > best) { best = x; arg = n0 + ff; }
         }
 #pragma unroll
@@ -404,7 +428,7 @@ SMDM_DEV void epilogue_block(const EpiParams& p, float* v, float (*S)[128], int 
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int ff = lane + 32 * u;
-          if (n0 + ff < p.n_valid) sum += __expf(S[j][ff] - best);
+          if (n0 + ff < p.n_valid) sum += __expf(S[j * 128 + ff] - best);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);

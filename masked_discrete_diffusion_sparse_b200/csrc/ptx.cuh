@@ -112,6 +112,15 @@ SMDM_DEV void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int x,
       : "memory");
 }
 
+SMDM_DEV void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1, int c2,
+                          uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+      : "memory");
+}
+
 SMDM_DEV void tma_load_4d(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1, int c2,
                           int c3, uint64_t policy) {
   asm volatile(
@@ -145,6 +154,21 @@ SMDM_DEV void bulk_store(void* dst, const void* src_smem, uint32_t bytes) {
                    reinterpret_cast<uint64_t>(dst)),
                "r"(smem_u32(src_smem)), "r"(bytes)
                : "memory");
+}
+// TMA tiled store / fp32 reduce-add of a shared-memory box into global memory (bulk group);
+// coordinates outside the tensor are not written.
+SMDM_DEV void tma_store_2d(const CUtensorMap* m, const void* src_smem, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(smem_u32(src_smem)), "r"(x), "r"(y)
+               : "memory");
+}
+SMDM_DEV void tma_reduce_add_2d(const CUtensorMap* m, const void* src_smem, int x, int y) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(src_smem)), "r"(x), "r"(y)
+      : "memory");
 }
 SMDM_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N committed bulk groups are still reading their shared-memory source.
@@ -187,6 +211,14 @@ SMDM_DEV void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t bar_clu
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
       " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+SMDM_DEV void tma_load_3d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster, int c0, int c1,
+                               int c2, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
       : "memory");
 }
 SMDM_DEV void tma_load_4d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster, int c0, int c1,
