@@ -63,6 +63,9 @@ SMDM_DEV uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// DH: head dim (64 or 128) as a compile-time constant so that every MMA issue sequence is
+// straight-line code (control flow between tcgen05.mma instructions stalls the issue).
+template <int DH>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnDev a) {
@@ -96,8 +99,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int nkv_all = (nkeys + 127) / 128;
   const int j0 = split * nkv_all / a.nsplit, j1 = (split + 1) * nkv_all / a.nsplit;
   const int nkv = j1 - j0;                           // key tiles of this split
-  const int dh = a.dh;
+  constexpr int dh = DH;
   if (nkv == 0) {
+    griddep_launch();
+    griddep_wait();
     // empty split: contribute nothing to the combine
     for (int r = threadIdx.x; r < nq; r += blockDim.x) {
       float* ml = a.part_ml + (((size_t)split * a.rows_total + qrow0 + r) * a.H + h) * 2;
@@ -106,7 +111,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     return;
   }
-  const int nsub = dh / 64;                          // 64-wide chunks of the head dim
+  constexpr int nsub = dh / 64;                      // 64-wide chunks of the head dim
   const long long cache_base = (long long)sg.seq * a.cache_rows_per_seq +
                                ((long long)a.layer * a.H + h) * a.cap;
 
@@ -135,6 +140,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
   const uint32_t t_o = tbase + 256;   // O accumulator columns [256, 256 + dh)
+  griddep_launch();
+  griddep_wait();   // q, the KV cache and the row metadata come from earlier kernels
 
   if (warp == 0) {
     if (lane == 0) {
@@ -173,6 +180,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (!mbar_wait(&s_free[b], ((j >> 1) & 1) ^ 1, abort_flag, a.status)) break;
           tc_fence_after();
           const uint32_t k_addr = smem_u32(smem + a.k_off + stage * a.stage_bytes);
+#pragma unroll
           for (int kk = 0; kk < dh / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
             umma_f16(tbase + b * 128, sdesc_sw128(q_addr + off, 16, 1024),
@@ -188,6 +196,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (!mbar_wait(&v_full[pstage], pphase, abort_flag, a.status)) break;
           tc_fence_after();
           const uint32_t v_addr = smem_u32(smem + a.v_off + pstage * a.stage_bytes);
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
             umma_f16(t_o, sdesc_sw128(p_addr + aoff, 16, 1024),
@@ -366,6 +375,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 __global__ void attn_combine_kernel(const float* __restrict__ part_o,
                                     const float* __restrict__ part_ml, int nsplit, int rows,
                                     int H, int dh, int d_model, __nv_bfloat16* __restrict__ out) {
+  griddep_launch();
+  griddep_wait();
   const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (w >= rows * H) return;
@@ -455,7 +466,10 @@ static int attn_layout(int dh, AttnDev& d) {
 }
 
 cudaError_t attn_tc_set_smem_attr() {
-  return cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const cudaError_t e = cudaFuncSetAttribute(
+      attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               227 * 1024);
 }
 
@@ -514,14 +528,20 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t stream) {
   d.part_ml = c.part_o ? c.part_o + (size_t)d.nsplit * c.rows_total * c.d_model : nullptr;
   const int smem = attn_layout(c.dh, d);
   dim3 grid(nb * d.nsplit, c.H);
-  attn_tc_kernel<<<grid, kAttnThreads, smem, stream>>>(*c.tmQ, *c.tmK, *c.tmV, d);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (c.dh == 128)
+    e = launch_pdl(attn_tc_kernel<128>, grid, dim3(kAttnThreads), smem, stream, 1, *c.tmQ, *c.tmK,
+                   *c.tmV, d);
+  else if (c.dh == 64)
+    e = launch_pdl(attn_tc_kernel<64>, grid, dim3(kAttnThreads), smem, stream, 1, *c.tmQ, *c.tmK,
+                   *c.tmV, d);
+  else
+    return cudaErrorInvalidValue;
   if (e != cudaSuccess || d.nsplit == 1) return e;
   const long long warps = (long long)c.rows_total * c.H;
-  attn_combine_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, stream>>>(
-      d.part_o, d.part_ml, d.nsplit, c.rows_total, c.H, c.dh, c.d_model,
-      reinterpret_cast<__nv_bfloat16*>(c.out));
-  return cudaGetLastError();
+  return launch_pdl(attn_combine_kernel, dim3((unsigned)((warps * 32 + 255) / 256)), dim3(256), 0,
+                    stream, 1, (const float*)d.part_o, (const float*)d.part_ml, d.nsplit,
+                    c.rows_total, c.H, c.dh, c.d_model, reinterpret_cast<__nv_bfloat16*>(c.out));
 }
 
 template <typename T>

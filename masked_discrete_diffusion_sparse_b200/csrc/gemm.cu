@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
+  griddep_launch();   // the next kernel may start its prologue
 
   // Work is split over pairs (kPair == 2) or CTAs; a tile is kPair * 128 weight rows.
   const long long U = g.units, G = gridDim.x / kPair;
@@ -164,10 +165,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const long long u_first = u_begin + pidx;
       int tile_i = (int)(u_first / KC), kc = (int)(u_first % KC);
       int nt = tile_i / g.row_blocks, rb = tile_i % g.row_blocks;
+      // Activation (B) loads of one stage; the weights (A) do not depend on earlier kernels.
+      auto load_b = [&](int st, int rb_, int kc_) {
+        uint8_t* B = smem + st * g.stage_bytes + kATileBytes;
+        for (int p = 0; p < nparts; ++p) {
+          const int y = g.row0 + rb_ * g.RT + p * part_rows + (int)rank * b_rows;
+          if constexpr (kPair == 1)
+            tma_load_2d(B + p * b_rows * 128, &tmB, &full[st], kc_ * 64, y, pol_x);
+          else
+            tma_load_2d_pair(B + p * b_rows * 128, &tmB, lead_addr(&full[st]), kc_ * 64, y, pol_x);
+        }
+      };
+      // First round of stages: issue the weight loads before waiting for the previous kernel
+      // (programmatic dependent launch) and the activation loads after it.
+      int pend_st[8], pend_rb[8], pend_kc[8];
+      int npend = 0;
+      bool dep_done = false;
+      auto finish_dep = [&]() {
+        griddep_wait();
+        for (int i = 0; i < npend; ++i) load_b(pend_st[i], pend_rb[i], pend_kc[i]);
+        npend = 0;
+        dep_done = true;
+      };
       for (long long u = u_first; u < u_end; u += np) {
+        if (!dep_done && (u - u_begin >= NS || npend == 8)) finish_dep();
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, g.status)) break;
         uint8_t* A = smem + stage * g.stage_bytes;
-        uint8_t* B = A + kATileBytes;
         const int at = nt * kPair + (int)rank;    // this CTA's 128-row A tile
         if constexpr (kPair == 1) {
           mbar_arrive_expect_tx(&full[stage], g.stage_bytes);
@@ -183,9 +206,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           } else {
             tma_load_2d(A, &tmA, &full[stage], kc * 64, at * 128, pol_w);
           }
-          for (int p = 0; p < nparts; ++p)
-            tma_load_2d(B + p * b_rows * 128, &tmB, &full[stage], kc * 64,
-                        g.row0 + rb * g.RT + p * part_rows, pol_x);
         } else {
           // both CTAs' bytes complete on the first CTA's barrier, which expects them all
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * g.stage_bytes);
@@ -202,9 +222,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           } else {
             tma_load_2d_pair(A, &tmA, fb, kc * 64, at * 128, pol_w);
           }
-          for (int p = 0; p < nparts; ++p)
-            tma_load_2d_pair(B + p * b_rows * 128, &tmB, fb, kc * 64,
-                             g.row0 + rb * g.RT + p * part_rows + (int)rank * b_rows, pol_x);
+        }
+        if (dep_done) {
+          load_b(stage, rb, kc);
+        } else {
+          pend_st[npend] = stage;
+          pend_rb[npend] = rb;
+          pend_kc[npend] = kc;
+          ++npend;
         }
         stage += np;
         while (stage >= NS) { stage -= NS; phase ^= 1; }
@@ -214,6 +239,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (++rb == g.row_blocks) { rb = 0; ++nt; }
         }
       }
+      if (!dep_done) finish_dep();
       if constexpr (kPair == 2) {
         // The pair's MMA completions arrive on these barriers from the first CTA: wait for the
         // release of every stage so that no arrival lands after this CTA has exited.
@@ -277,6 +303,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp >= 2 && warp <= 5) {
     // Epilogue warps 2..5: TMEM lane quarter = warp % 4 -> A-tile row m.
+    griddep_wait();   // row metadata, outputs, partial slots and counters follow earlier kernels
     const int q = warp & 3;
     const int m = q * 32 + lane;
     const int et = threadIdx.x - 64;   // 0..127
@@ -707,30 +734,18 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream) {
   const bool two_parts = g.RT > 256;
   if (pair == 1) {
     if (two_parts)
-      gemm_tc_kernel<__nv_bfloat16, 1, 2><<<(unsigned)G, kGemmThreads, L.total, stream>>>(
-          *c.tmA, tA2, *c.tmB, *c.tmOut, g, c.epi);
-    else
-      gemm_tc_kernel<__nv_bfloat16, 1, 1><<<(unsigned)G, kGemmThreads, L.total, stream>>>(
-          *c.tmA, tA2, *c.tmB, *c.tmOut, g, c.epi);
-    return cudaGetLastError();
+      return launch_pdl(gemm_tc_kernel<__nv_bfloat16, 1, 2>, dim3((unsigned)G), dim3(kGemmThreads),
+                        L.total, stream, 1, *c.tmA, tA2, *c.tmB, *c.tmOut, g, c.epi);
+    return launch_pdl(gemm_tc_kernel<__nv_bfloat16, 1, 1>, dim3((unsigned)G), dim3(kGemmThreads),
+                      L.total, stream, 1, *c.tmA, tA2, *c.tmB, *c.tmOut, g, c.epi);
   }
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)(G * 2));
-  cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = L.total;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   if (two_parts)
-    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<__nv_bfloat16, 2, 2>, *c.tmA, tA2, *c.tmB,
-                              *c.tmOut, g, c.epi);
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<__nv_bfloat16, 2, 1>, *c.tmA, tA2, *c.tmB,
-                            *c.tmOut, g, c.epi);
+    return launch_pdl(gemm_tc_kernel<__nv_bfloat16, 2, 2>, dim3((unsigned)(G * 2)),
+                      dim3(kGemmThreads), L.total, stream, 2, *c.tmA, tA2, *c.tmB, *c.tmOut, g,
+                      c.epi);
+  return launch_pdl(gemm_tc_kernel<__nv_bfloat16, 2, 1>, dim3((unsigned)(G * 2)),
+                    dim3(kGemmThreads), L.total, stream, 2, *c.tmA, tA2, *c.tmB, *c.tmOut, g,
+                    c.epi);
 }
 
 cudaError_t launch_gemm_simt(const float* W, const float* W2, const float* X, int ldx, int K,

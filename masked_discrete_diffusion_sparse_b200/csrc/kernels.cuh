@@ -6,10 +6,49 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
+#include <utility>
 
 #include "ptx.cuh"
 
 namespace smdm {
+
+// Programmatic dependent launch for the library's kernels (SMDM_PDL=0 turns it off).
+inline bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("SMDM_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+// Launch `kern` with programmatic stream serialization (and a cluster of cluster_x CTAs when
+// > 1).  Every kernel launched this way calls griddep_wait() before it touches data that an
+// earlier kernel produces or consumes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = (unsigned)cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 constexpr int kMaxBatch = 8;
 constexpr int kTypePrompt = 0, kTypeClean = 1, kTypeMask = 2, kTypeReg = 3;

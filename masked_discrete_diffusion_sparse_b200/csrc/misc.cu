@@ -19,6 +19,8 @@ namespace smdm {
 // every row of the step.  slot: K/V of row i go to cache slot ctx + i.
 // ------------------------------------------------------------------------------------------
 __global__ void pack_step_kernel(PackArgs a) {
+  griddep_launch();
+  griddep_wait();   // launched with programmatic dependent launch
   const PackSeq& s = a.s[blockIdx.x];
   __shared__ int qbuf_count;
   __shared__ int warp_counts[32];
@@ -110,6 +112,8 @@ __global__ void pack_step_kernel(PackArgs a) {
 
 // Prefill / dense / training-form rows: one thread per row.
 __global__ void pack_linear_kernel(LinearPackArgs a) {
+  griddep_launch();
+  griddep_wait();   // launched with programmatic dependent launch
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= a.n) return;
   int id, pos, type, label;
@@ -152,6 +156,8 @@ __global__ void pack_linear_kernel(LinearPackArgs a) {
 }
 
 __global__ void gather_rows_kernel(const int* __restrict__ src_rows, int n, int* __restrict__ qrow) {
+  griddep_launch();
+  griddep_wait();   // launched with programmatic dependent launch
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) qrow[i] = src_rows[i];
 }
@@ -186,6 +192,8 @@ template <> struct Vec4<__nv_bfloat16> {
 // One CTA of 256 threads per row; the row stays in registers (d <= 8192, d % 4 == 0).
 template <typename T>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(NormArgs a) {
+  griddep_launch();
+  griddep_wait();   // launched with programmatic dependent launch
   constexpr int kMaxV = 8;
   const int r = blockIdx.x;
   const int src = a.gather ? a.gather[r] : r;
@@ -233,6 +241,8 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(NormArgs a) {
 // unmask: one CTA per sequence.
 // ------------------------------------------------------------------------------------------
 __global__ void unmask_kernel(UnmaskArgs a) {
+  griddep_launch();
+  griddep_wait();   // launched with programmatic dependent launch
   const UnmaskSeq& s = a.s[blockIdx.x];
   extern __shared__ float sh[];
   float* conf = sh;                                     // [n_q]
@@ -335,32 +345,27 @@ __global__ void fill_i32_kernel(int* p, int n, int v) {
 // launchers
 // ------------------------------------------------------------------------------------------
 cudaError_t launch_pack_step(const PackArgs& a, cudaStream_t st) {
-  pack_step_kernel<<<a.n_seq, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(pack_step_kernel, dim3(a.n_seq), dim3(256), 0, st, 1, a);
 }
 cudaError_t launch_pack_linear(const LinearPackArgs& a, cudaStream_t st) {
   if (a.n <= 0) return cudaSuccess;
-  pack_linear_kernel<<<(a.n + 255) / 256, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(pack_linear_kernel, dim3((a.n + 255) / 256), dim3(256), 0, st, 1, a);
 }
 cudaError_t launch_gather_rows(const int* src, int n, int* qrow, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  gather_rows_kernel<<<(n + 255) / 256, 256, 0, st>>>(src, n, qrow);
-  return cudaGetLastError();
+  return launch_pdl(gather_rows_kernel, dim3((n + 255) / 256), dim3(256), 0, st, 1, src, n, qrow);
 }
 template <typename T>
 cudaError_t launch_rmsnorm(const NormArgs& a, int rows, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  rmsnorm_kernel<T><<<rows, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(rmsnorm_kernel<T>, dim3(rows), dim3(256), 0, st, 1, a);
 }
 template cudaError_t launch_rmsnorm<float>(const NormArgs&, int, cudaStream_t);
 template cudaError_t launch_rmsnorm<__nv_bfloat16>(const NormArgs&, int, cudaStream_t);
 
 cudaError_t launch_unmask(const UnmaskArgs& a, int max_nq, cudaStream_t st) {
   const size_t smem = (size_t)max_nq * 12;
-  unmask_kernel<<<a.n_seq, 512, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(unmask_kernel, dim3(a.n_seq), dim3(512), smem, st, 1, a);
 }
 cudaError_t launch_debug_mask(const int* type, const int* label, int n, uint32_t* bitmap,
                               cudaStream_t st) {

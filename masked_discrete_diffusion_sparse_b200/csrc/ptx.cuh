@@ -182,6 +182,16 @@ SMDM_DEV void fence_proxy_async_smem() {
 }
 
 // ------------------------------------------------------------------------------------------
+// Programmatic dependent launch: a kernel launched with it may start while the previous kernel
+// in the stream is still running.  griddep_wait() blocks the calling thread until the previous
+// grids have completed and their memory is visible; it must precede every access to data that
+// earlier kernels produce or consume (a no-op when the launch did not use the attribute).
+// griddep_launch() lets the next kernel start its own prologue early.
+// ------------------------------------------------------------------------------------------
+SMDM_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+SMDM_DEV void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ------------------------------------------------------------------------------------------
 // CTA pairs (cluster of 2, tcgen05 cta_group::2)
 // ------------------------------------------------------------------------------------------
 SMDM_DEV uint32_t cluster_ctarank() {
