@@ -82,9 +82,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* kv_empty = v_full + NS;
   uint64_t* s_full = kv_empty + NS;   // [2]
   uint64_t* s_free = s_full + 2;      // [2]
-  uint64_t* p_full = s_free + 2;
-  uint64_t* pv_done = p_full + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pv_done + 1);
+  uint64_t* p_full = s_free + 2;      // [2] per P buffer: softmax warps wrote P(j), j & 1 == b
+  uint64_t* pv_done = p_full + 2;     // [2] per P buffer: the P(j) V(j) product completed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pv_done + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -126,8 +126,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&s_full[b], 1);
       mbar_init(&s_free[b], 4);
     }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&p_full[b], 4);
+      mbar_init(&pv_done[b], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -192,19 +194,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (j >= 1) {
           // O += P_{j-1} V_{j-1}
           const int jj = j - 1;
-          if (!mbar_wait(p_full, jj & 1, abort_flag, a.status)) break;
+          const int pb = jj & 1;   // P buffer of tile jj; its k-th use has phase k & 1
+          if (!mbar_wait(&p_full[pb], (jj >> 1) & 1, abort_flag, a.status)) break;
           if (!mbar_wait(&v_full[pstage], pphase, abort_flag, a.status)) break;
           tc_fence_after();
           const uint32_t v_addr = smem_u32(smem + a.v_off + pstage * a.stage_bytes);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_f16(t_o, sdesc_sw128(p_addr + aoff, 16, 1024),
+            umma_f16(t_o, sdesc_sw128(p_addr + pb * (128 * 128 * 2) + aoff, 16, 1024),
                      sdesc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
                      (jj > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&kv_empty[pstage]);
-          umma_commit(pv_done);
+          umma_commit(&pv_done[pb]);
           if (++pstage == NS) { pstage = 0; pphase ^= 1; }
         }
       }
@@ -232,9 +235,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[b]);
-        if (j >= 1 && !mbar_wait(pv_done, (j - 1) & 1, abort_flag, a.status)) break;
+        // keep in step with the other warps: signal P(j) only once P buffer j & 1 is free, so
+        // that no arrival can land in a later phase of p_full (its P rows are never read back)
+        if (j >= 2 && !mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, a.status)) break;
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(&p_full[j & 1]);
         continue;
       }
       const int key0 = (j0 + j) * 128;
@@ -274,10 +279,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         m_ref = mx;
       }
       float rs = 0.f;
-      // O and P are still in use by the previous P V product.
-      if (j >= 1 && !mbar_wait(pv_done, (j - 1) & 1, abort_flag, a.status)) break;
+      // P buffer j & 1 was last read by the P V product of tile j - 2
+      if (j >= 2 && !mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, a.status)) break;
+      const bool rescale = __any_sync(0xffffffffu, alpha != 1.f) && j >= 1;
+      // rescaling O needs the product of tile j - 1 accumulated first
+      if (rescale && !mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status))
+        break;
       tc_fence_after();
-      if (__any_sync(0xffffffffu, alpha != 1.f) && j >= 1) {
+      if (rescale) {
         for (int c = 0; c < dh / 16; ++c) {
           float o[16];
           tmem_ld16(t_o + lane_off + c * 16, o);
@@ -307,7 +316,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           pk.y = pack_bf16x2(p[2], p[3]);
           pk.z = pack_bf16x2(p[4], p[5]);
           pk.w = pack_bf16x2(p[6], p[7]);
-          p_store_swizzled(Ps, em, hh * 8 + c8, pk);
+          p_store_swizzled(Ps + (j & 1) * (128 * 128 * 2), em, hh * 8 + c8, pk);
         }
       }
       tc_fence_before();
@@ -317,10 +326,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[j & 1]);
     }
     // Final: O / l (one split), or the unnormalised partial for the combine pass.
-    if (nkv > 0 && mbar_wait(pv_done, (nkv - 1) & 1, abort_flag, a.status)) {
+    if (nkv > 0 && mbar_wait(&pv_done[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1, abort_flag, a.status)) {
       tc_fence_after();
       if (a.nsplit == 1) {
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
@@ -451,7 +460,7 @@ __global__ void attn_simt_kernel(const T* __restrict__ q, T* __restrict__ out, K
 static int attn_layout(int dh, AttnDev& d) {
   const int q_bytes = 128 * dh * 2;
   const int kv_bytes = 128 * dh * 2;
-  const int p_bytes = 128 * 128 * 2;
+  const int p_bytes = 2 * 128 * 128 * 2;   // two P buffers (tile j uses buffer j & 1)
   d.q_off = 0;
   d.p_off = q_bytes;
   d.stage_bytes = kv_bytes;
