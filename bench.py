@@ -115,6 +115,12 @@ def run_cost(wl: synth.Workload, plan: synth.Plan):
     return costs
 
 
+# DRAM bytes (read + write) over algorithmic bytes of gemm_tc_kernel, from one ncu capture of
+# three launches (QKV, O, gate/up) of the 1024-token workload:
+# profiles/gemm_attn_t2i1024_ncu_full.md.  Re-measure whenever the GEMM kernel changes.
+GEMM_TRAFFIC_RATIO = 327.8 / 321.4
+
+
 def gemm_bytes_per_run(wl: synth.Workload, plan: synth.Plan, es=2):
     """Algorithmic bytes of the GEMM launches of one full run: weights once per launch plus
     activation operand reads and output writes."""
@@ -478,7 +484,10 @@ def main():
         "gpu_launches": launches_per_run * args.steps,
         "roofline": {"bound": "hbm", "kernel": "gemm_tc_kernel (all weight GEMMs)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": (achieved / hbm) if achieved else None, "traffic": None,
+                     "frac": (achieved / hbm) if achieved else None,
+                     "traffic": (GEMM_TRAFFIC_RATIO * gb / gemm_n) if gemm_n else None,
+                     "traffic_unit": "bytes per launch (measured DRAM/algorithmic ratio x "
+                                     "algorithmic bytes per launch)",
                      "peak_source": peak_src,
                      "gemm_ms_per_run": gemm_ms, "gemm_launches_per_run": gemm_n,
                      "gemm_algorithmic_gb_per_run": gb / 1e9},
