@@ -312,6 +312,9 @@ def main():
     import torch
     import torch.distributed as dist
     import masked_discrete_diffusion_sparse_b200 as smdm
+    from masked_discrete_diffusion_sparse_b200.replicas import (aggregate_throughput,
+                                                                replica_sequence_ids,
+                                                                slowest_time_ms)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -325,8 +328,9 @@ def main():
 
     m = wl.model
     B = wl.batch
-    plans = [synth.make_plan(wl, rank * B + s) for s in range(B)]
-    prompts_np = np.stack([synth.make_prompt(wl, rank * B + s) for s in range(B)])
+    seq_ids = replica_sequence_ids(rank, B)   # disjoint sequence sets across ranks
+    plans = [synth.make_plan(wl, i) for i in seq_ids]
+    prompts_np = np.stack([synth.make_prompt(wl, i) for i in seq_ids])
     msr, max_rows = capacities(wl, plans)
     cfg = smdm.make_config(m.n_layers, m.d_model, m.n_heads, m.d_head, m.d_ffn, m.vocab,
                            n_reg=m.n_reg,
@@ -334,7 +338,7 @@ def main():
                            rope_theta=m.rope_theta, rms_eps=m.rms_eps, max_batch=B,
                            max_len=wl.prompt_len + wl.gen_len, max_step_rows=msr,
                            max_rows=max_rows)
-    weights = device_weights(wl, wl.seed + 7919 * rank, dev)
+    weights = device_weights(wl, wl.seed + 7919, dev)   # the same model on every replica
     model = smdm.Model(cfg, weights)
     stream = torch.cuda.Stream(device=dev)
 
@@ -401,12 +405,9 @@ def main():
     with torch.cuda.stream(stream):
         ms = timed(graph.replay, args.steps)
     clocks = sampler.stop()
-    ms_t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = slowest_time_ms(ms, world, dist, dev)
     tokens_per_run = Lg * B
-    value = tokens_per_run * world / (ms_max / 1e3)
+    value = aggregate_throughput(tokens_per_run, world, ms_max)
     assert model.smdm_device_status(stream) == 0
 
     # e2e: public API, pinned host inputs -> device, grid -> host, every run
@@ -438,12 +439,10 @@ def main():
             for _ in range(max(1, args.warmup)):
                 e2e_run()
             e_ms = timed(e2e_run, max(3, args.steps // 2))
-        et = torch.tensor([e_ms], device=dev)
-        if world > 1:
-            dist.all_reduce(et, op=dist.ReduceOp.MAX)
-        e2e = {"value": tokens_per_run * world / (float(et.item()) / 1e3), "unit": UNIT,
+        e_max = slowest_time_ms(e_ms, world, dist, dev)
+        e2e = {"value": aggregate_throughput(tokens_per_run, world, e_max), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": float(et.item()), "path": "smdm_generate (eager launches)"}
+               "ms_per_step": e_max, "path": "smdm_generate (eager launches)"}
 
     # dense comparator: the same library's dense full-sequence MDM step, full run
     dense = None
