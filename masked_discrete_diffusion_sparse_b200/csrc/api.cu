@@ -374,7 +374,7 @@ smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensor
   if (h->bf16) {
     CUtensorMap tmB;
     const size_t MR = align_up((size_t)h->cfg.max_rows, 256);
-    const int pair = gemm_tc_pair(n_out, swiglu, rows);
+    const int pair = gemm_tc_pair(n_out, swiglu, rows, ep.kind);
     if (!encode_2d(&tmB, X, K, MR, (uint64_t)K * 2, 64, gemm_tc_box_rows(rows, pair)))
       return fail(h, SMDM_ECUDA, "cuTensorMapEncodeTiled failed for an activation operand");
     CUtensorMap tmOut;

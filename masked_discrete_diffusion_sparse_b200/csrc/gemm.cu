@@ -626,11 +626,27 @@ static int pair_enabled() {
   return v;
 }
 
-int gemm_tc_pair(int n_out, int swiglu, int rows) {
+// Whole tiles (one CTA per tile, no split-K fix-up) when the tile count is at least this
+// percentage of the grid (measured on the 4096-token run: 40 puts the QKV GEMM (96 tiles) and
+// the LM head (64 tiles) on whole tiles, the O / down GEMMs (32 tiles) on stream-K);
+// SMDM_WHOLE_TILE_MIN overrides it.
+static int whole_tile_min_pct() {
+  static int v = [] {
+    const char* e = getenv("SMDM_WHOLE_TILE_MIN");
+    const int x = e ? atoi(e) : 40;
+    return (x >= 1 && x <= 100) ? x : 40;
+  }();
+  return v;
+}
+
+int gemm_tc_pair(int n_out, int swiglu, int rows, int epi_kind) {
   (void)rows;
   const int n_tiles = swiglu ? (n_out + 63) / 64 : (n_out + 127) / 128;
-  // the pair covers two adjacent 128-row weight tiles, so their count must be even
-  return (pair_enabled() && n_tiles % 2 == 0) ? 2 : 1;
+  // Measured on the 4096-token run: pairs help the QKV and gate/up GEMMs and cost the residual
+  // (O, down) and LM-head GEMMs a little.  The pair covers two adjacent 128-row weight tiles, so
+  // their count must be even.
+  const bool wants = epi_kind == kEpiQKV || epi_kind == kEpiSwiGLU;
+  return (pair_enabled() && wants && n_tiles % 2 == 0) ? 2 : 1;
 }
 
 static int pow2_ceil(int x) {
@@ -718,8 +734,9 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream) {
     if (mc > 0 && G > mc) G = mc;
   }
   const long long tiles_total = (long long)pair_tiles * g.row_blocks;
+  const int whole_pct = whole_tile_min_pct();
   if (c.sched == 1 ? tiles_total <= G
-                   : c.sched == 0 && tiles_total <= G && tiles_total * 10 >= G * 6)
+                   : c.sched == 0 && tiles_total <= G && tiles_total * 100 >= G * whole_pct)
     G = tiles_total;
   if (G > g.units) G = g.units;
   if (G < 1) G = 1;

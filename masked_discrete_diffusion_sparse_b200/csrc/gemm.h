@@ -40,7 +40,7 @@ struct GemmCall {
 int gemm_tc_row_tile(int rows);
 int gemm_tc_box_rows(int rows, int pair);
 // CTA-pair mode (2) or single-CTA mode (1) for a bf16 GEMM of this shape.
-int gemm_tc_pair(int n_out, int swiglu, int rows);
+int gemm_tc_pair(int n_out, int swiglu, int rows, int epi_kind);
 cudaError_t gemm_tc_set_smem_attr();
 cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream);
 cudaError_t launch_gemm_simt(const float* W, const float* W2, const float* X, int ldx, int K,
