@@ -76,6 +76,23 @@ int encode_gateup_interleaved(CUtensorMap* m, const void* gate, const void* up, 
   return up_first ? 2 : 1;
 }
 
+// Head-tile view for the attention kernel: rows of `row_elems` bf16 split into 64-element
+// (128-byte) chunks, dims {64, rows, row_elems / 64}, box {64, 128, nsub}: one copy brings a
+// 128-row tile of nsub chunks, landing as nsub swizzled [128][64] sub-tiles.
+bool encode_head_tiles(CUtensorMap* m, const void* base, uint64_t row_elems, uint64_t rows,
+                       uint32_t nsub) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn || row_elems % 64) return false;
+  cuuint64_t dims[3] = {64, rows, row_elems / 64};
+  cuuint64_t strides[2] = {row_elems * 2, 128};
+  cuuint32_t box[3] = {64, 128, nsub};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // 2-D output map for the GEMM epilogue's TMA stores: `cols` x `rows` elements (bf16 or fp32),
 // row pitch `ld` elements, box {box_cols, 32}, no swizzle.
 bool encode_out(CUtensorMap* m, const void* base, bool f32, uint64_t cols, uint64_t rows,
@@ -698,13 +715,11 @@ smdm_status smdm_create(const smdm_config* cfg, const smdm_weights* w, void* d_w
     ok &= encode_2d(&h->tm_lm, w->lm_head, d, cfg->vocab, (uint64_t)d * 2, 64, 128);
     const size_t MR = align_up((size_t)cfg->max_rows, 256);
     const uint64_t cache_rows = (uint64_t)cfg->max_batch * nl * H * h->L.cap;
-    ok &= encode_2d(&h->tm_kc, h->at<uint8_t>(h->L.kc), dh, cache_rows, (uint64_t)dh * 2, 64, 128);
-    ok &= encode_2d(&h->tm_vc, h->at<uint8_t>(h->L.vc), dh, cache_rows, (uint64_t)dh * 2, 64, 128);
-    ok &= encode_2d(&h->tm_kscr, h->at<uint8_t>(h->L.kscr), dh, (uint64_t)H * MR, (uint64_t)dh * 2,
-                    64, 128);
-    ok &= encode_2d(&h->tm_vscr, h->at<uint8_t>(h->L.vscr), dh, (uint64_t)H * MR, (uint64_t)dh * 2,
-                    64, 128);
-    ok &= encode_2d(&h->tm_q, h->at<uint8_t>(h->L.q), d, MR, (uint64_t)d * 2, 64, 128);
+    ok &= encode_head_tiles(&h->tm_kc, h->at<uint8_t>(h->L.kc), dh, cache_rows, dh / 64);
+    ok &= encode_head_tiles(&h->tm_vc, h->at<uint8_t>(h->L.vc), dh, cache_rows, dh / 64);
+    ok &= encode_head_tiles(&h->tm_kscr, h->at<uint8_t>(h->L.kscr), dh, (uint64_t)H * MR, dh / 64);
+    ok &= encode_head_tiles(&h->tm_vscr, h->at<uint8_t>(h->L.vscr), dh, (uint64_t)H * MR, dh / 64);
+    ok &= encode_head_tiles(&h->tm_q, h->at<uint8_t>(h->L.q), d, MR, dh / 64);
     if (!ok) {
       delete h;
       return SMDM_ECUDA;
@@ -1228,11 +1243,9 @@ extern "C" smdm_status smdm_forward_stepcausal_noalloc(
     }
     ok &= encode_2d(&h->tm_lm, w->lm_head, d, vc.vocab, (uint64_t)d * 2, 64, 128);
     const size_t MR = align_up((size_t)vc.max_rows, 256);
-    ok &= encode_2d(&h->tm_kscr, h->at<uint8_t>(L.kscr), dh, (uint64_t)H * MR, (uint64_t)dh * 2,
-                    64, 128);
-    ok &= encode_2d(&h->tm_vscr, h->at<uint8_t>(L.vscr), dh, (uint64_t)H * MR, (uint64_t)dh * 2,
-                    64, 128);
-    ok &= encode_2d(&h->tm_q, h->at<uint8_t>(L.q), d, MR, (uint64_t)d * 2, 64, 128);
+    ok &= encode_head_tiles(&h->tm_kscr, h->at<uint8_t>(L.kscr), dh, (uint64_t)H * MR, dh / 64);
+    ok &= encode_head_tiles(&h->tm_vscr, h->at<uint8_t>(L.vscr), dh, (uint64_t)H * MR, dh / 64);
+    ok &= encode_head_tiles(&h->tm_q, h->at<uint8_t>(L.q), d, MR, dh / 64);
     if (!ok) return SMDM_ECUDA;
   }
   return smdm_forward_stepcausal(h, d_ids, d_pos, d_type, d_label, n, d_logit_rows, n_rows,

@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t pol_q = policy_evict_normal();
       const uint64_t pol_kv = policy_evict_last();
       mbar_arrive_expect_tx(q_full, 128 * dh * 2);
-      for (int c = 0; c < nsub; ++c) tma_load_2d(Qs + c * 16384, &tmQ, q_full, h * dh + c * 64, qrow0, pol_q);
+      tma_load_3d(Qs, &tmQ, q_full, 0, qrow0, h * nsub, pol_q);   // nsub [128][64] sub-tiles
       int stage = 0;
       uint32_t phase = 0;
       for (int j = 0; j < nkv; ++j) {
@@ -159,9 +159,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         uint8_t* Vs = smem + a.v_off + stage * a.stage_bytes;
         const int y = (int)(cache_base + (long long)(j0 + j) * 128);
         mbar_arrive_expect_tx(&k_full[stage], 128 * dh * 2);
-        for (int c = 0; c < nsub; ++c) tma_load_2d(Ks + c * 16384, &tmK, &k_full[stage], c * 64, y, pol_kv);
+        tma_load_3d(Ks, &tmK, &k_full[stage], 0, y, 0, pol_kv);
         mbar_arrive_expect_tx(&v_full[stage], 128 * dh * 2);
-        for (int c = 0; c < nsub; ++c) tma_load_2d(Vs + c * 16384, &tmV, &v_full[stage], c * 64, y, pol_kv);
+        tma_load_3d(Vs, &tmV, &v_full[stage], 0, y, 0, pol_kv);
         if (++stage == NS) { stage = 0; phase ^= 1; }
       }
     }

@@ -21,8 +21,10 @@ struct AttnCall {
   const int* kvlen;
   const int* type;
   const int* label;
-  const CUtensorMap* tmQ;   // q [rows][d_model] bf16, box {64, 128}
-  const CUtensorMap* tmK;   // K cache as 2-D [cache rows][d_head] bf16, box {64, 128}
+  // 3-D head-tile maps {64, rows, row elements / 64}, box {64, 128, d_head / 64} (one copy per
+  // 128-row tile):
+  const CUtensorMap* tmQ;   // q [rows][d_model] bf16 (chunk coordinate = head * d_head / 64)
+  const CUtensorMap* tmK;   // K cache [cache rows][d_head] bf16
   const CUtensorMap* tmV;   // V cache, same layout
   long long cache_rows_per_seq;
   int cap;
