@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--n-reg", type=int, default=None,
+                    help="register rows per step (the method's 64 by default); for the "
+                         "register-count sensitivity study")
     return ap.parse_args()
 
 
@@ -306,6 +309,12 @@ def capacities(wl, plans):
 def main():
     args = parse()
     wl = synth.WORKLOADS[args.workload]
+    if args.n_reg is not None and args.n_reg != wl.model.n_reg:
+        if args.n_reg < 1:
+            raise SystemExit("--n-reg must be >= 1")
+        import dataclasses
+        wl = dataclasses.replace(wl, name=f"{wl.name}-reg{args.n_reg}",
+                                 model=dataclasses.replace(wl.model, n_reg=args.n_reg))
     if args.impl == "reference":
         return run_reference(args, wl)
 

@@ -6,6 +6,7 @@ fp32 weights; sampled tokens equal the oracle's argmax except where the oracle's
 below that tolerance.  Trajectories are teacher-forced: after every step the oracle adopts the
 device's committed tokens when they are admissible.
 """
+import dataclasses
 import os
 
 import numpy as np
@@ -85,6 +86,22 @@ def test_device_mask_predicate_matches_oracle():
 @pytest.mark.parametrize("name", ["tiny-f32-cos", "tiny-bf16-cos", "tiny-bf16-semiar"])
 def test_sparse_run_tiny(name):
     wl = synth.WORKLOADS[name]
+    r = Runner(wl)
+    try:
+        checks, grids, states = run_teacher_forced(r)
+        _check_all(checks, r.tol)
+        assert (grids.cpu().numpy() >= 0).all()
+    finally:
+        r.close()
+
+
+@pytest.mark.parametrize("n_reg", [1, 32])
+def test_sparse_run_register_count(n_reg):
+    """Register-count variants of the sparse row set (the method uses 64 registers): n_reg
+    register rows with ids REG_0.. at positions L+1..L+n_reg; same kernels, parity per step."""
+    base = synth.WORKLOADS["tiny-bf16-cos"]
+    wl = dataclasses.replace(base, name=f"{base.name}-reg{n_reg}",
+                             model=dataclasses.replace(base.model, n_reg=n_reg))
     r = Runner(wl)
     try:
         checks, grids, states = run_teacher_forced(r)
