@@ -43,6 +43,25 @@ def test_invalid_config_is_rejected_without_gpu():
     assert lib.smdm_workspace_bytes(ctypes.byref(bad2)) == 0
 
 
+def test_config_rules_for_bf16_models():
+    """bf16 shape rules of the header: d_model % 128, d_head in {64, 128}, d_ffn % 64 and
+    vocab % 4 (16-byte logit rows); a valid shape gets a positive workspace size."""
+    lib = smdm.lib()
+    ok = dict(dtype=smdm.SMDM_BF16, max_batch=1, max_len=300, max_step_rows=200, max_rows=300)
+    good = smdm.make_config(2, 256, 2, 128, 704, 1000, **ok)
+    assert lib.smdm_workspace_bytes(ctypes.byref(good)) > 0
+    for shape in [(2, 192, 3, 64, 704, 1000),    # d_model % 128
+                  (2, 256, 8, 32, 704, 1000),    # d_head 32
+                  (2, 256, 2, 128, 700, 1000),   # d_ffn % 64
+                  (2, 256, 2, 128, 704, 1002)]:  # vocab % 4
+        bad = smdm.make_config(*shape, **ok)
+        assert lib.smdm_workspace_bytes(ctypes.byref(bad)) == 0, shape
+    # the fp32 path has none of the tile rules
+    f32 = smdm.make_config(2, 128, 2, 64, 320, 301, dtype=smdm.SMDM_F32, max_batch=1,
+                           max_len=100, max_step_rows=100, max_rows=100)
+    assert lib.smdm_workspace_bytes(ctypes.byref(f32)) > 0
+
+
 def test_model_refuses_to_run_without_cuda():
     import torch
     if torch.cuda.is_available():
