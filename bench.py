@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--form", default="sampling", choices=["sampling", "training"],
+                    help="sampling: full sparse sampling runs (the headline); training: one "
+                         "training-form forward over a whole step-labelled trajectory")
     ap.add_argument("--n-reg", type=int, default=None,
                     help="register rows per step (the method's 64 by default); for the "
                          "register-count sensitivity study")
@@ -296,6 +299,88 @@ def device_weights(wl: synth.Workload, seed: int, device):
     return w
 
 
+def trajectory_rows(wl: synth.Workload, plan: synth.Plan, prompt: np.ndarray, seed: int):
+    """Rows of a whole sampling trajectory in the step-labelled training form (order plans):
+    the prompt (label 0), then for every step k the clean copies of the tokens decoded at step
+    k, the mask copies of the same positions (the decode set C_k) and the registers, all
+    labelled k.  Token values are random (structure and sizes are what the forward's cost
+    depends on).  Returns ids, pos, types, labels and the logit rows (the mask copies)."""
+    m = wl.model
+    P, Lg = wl.prompt_len, wl.gen_len
+    L = P + Lg
+    g = np.random.Generator(np.random.PCG64([wl.seed, 7000 + seed]))
+    ids, pos, types, labels, logit_rows = list(prompt), list(range(1, P + 1)), [0] * P, [0] * P, []
+    for k in range(1, plan.n_steps + 1):
+        q = plan.query_positions(k)
+        n = len(q)
+        ids += list(g.integers(0, m.vocab, n))
+        pos += list(q)
+        types += [1] * n                      # clean copies
+        labels += [k] * n
+        logit_rows += list(range(len(ids), len(ids) + n))
+        ids += [m.vocab] * n                  # [MASK] copies
+        pos += list(q)
+        types += [2] * n
+        labels += [k] * n
+        ids += [m.vocab + 2 + j for j in range(m.n_reg)]
+        pos += [L + 1 + j for j in range(m.n_reg)]
+        types += [3] * m.n_reg
+        labels += [k] * m.n_reg
+    as32 = lambda a: np.asarray(a, dtype=np.int32)
+    return as32(ids), as32(pos), as32(types), as32(labels), as32(logit_rows)
+
+
+def run_training_form(args, wl):
+    """Times one training-form forward (smdm_forward_stepcausal) over the whole trajectory of
+    the workload's plan: every row of every step in one forward under the label predicate."""
+    import torch
+    import masked_discrete_diffusion_sparse_b200 as smdm
+    if wl.plan == "semiar" or wl.batch != 1:
+        raise SystemExit("--form training supports single-sequence order plans")
+    m = wl.model
+    dev = torch.device("cuda", 0)
+    plan = synth.make_plan(wl, 0)
+    prompt = synth.make_prompt(wl, 0)
+    ids, pos, types, labels, lrows = trajectory_rows(wl, plan, prompt, 0)
+    n = len(ids)
+    cfg = smdm.make_config(m.n_layers, m.d_model, m.n_heads, m.d_head, m.d_ffn, m.vocab,
+                           n_reg=m.n_reg,
+                           dtype=smdm.SMDM_BF16 if m.dtype == synth.BF16 else smdm.SMDM_F32,
+                           rope_theta=m.rope_theta, rms_eps=m.rms_eps, max_batch=1,
+                           max_len=wl.prompt_len + wl.gen_len, max_step_rows=1, max_rows=n)
+    model = smdm.Model(cfg, device_weights(wl, wl.seed + 7919, dev))
+    t = lambda a: torch.as_tensor(a, device=dev)
+    d_ids, d_pos, d_types, d_labels, d_rows = t(ids), t(pos), t(types), t(labels), t(lrows)
+    logits = torch.empty((len(lrows), m.vocab), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def fwd():
+        model.smdm_forward_stepcausal(d_ids, d_pos, d_types, d_labels, d_rows, logits,
+                                      stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            fwd()
+        torch.cuda.synchronize()
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            fwd()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    assert model.smdm_device_status(stream) == 0
+    print(json.dumps({"metric": "training-form forward rows/s", "value": n / (ms / 1e3),
+                      "unit": "rows/s", "n_gpus": 1, "steps": args.steps,
+                      "warmup": max(3, args.warmup), "ms_per_step": ms,
+                      "higher_is_better": True, "form": "training", "rows": n,
+                      "logit_rows": int(len(lrows)), "dtype": "bf16" if m.dtype == synth.BF16
+                      else "f32", "data": "synthetic", "config": describe(wl)}), flush=True)
+    model.close()
+    return 0
+
+
 def capacities(wl, plans):
     m = wl.model
     msr = 1
@@ -317,6 +402,9 @@ def main():
                                  model=dataclasses.replace(wl.model, n_reg=args.n_reg))
     if args.impl == "reference":
         return run_reference(args, wl)
+
+    if args.form == "training":
+        return run_training_form(args, wl)
 
     import torch
     import torch.distributed as dist
