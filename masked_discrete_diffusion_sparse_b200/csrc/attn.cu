@@ -8,10 +8,11 @@
 //   label mode — the training-form rule evaluated per (query, key) from row types and step
 //     labels; keys are the rows of the same forward.
 //
-// bf16 path: one CTA per (sequence, 128-row query tile, head).  Warp 0 streams Q and K/V tiles
-// with TMA, warp 1 issues tcgen05.mma (S = Q K^T into one of two TMEM buffers, O += P V into a
-// TMEM accumulator), warps 2-5 own one query row per thread: masking, online softmax in the
-// exp2 domain, P (bf16) into swizzled shared memory, final 1/l scaling.  The running maximum is
+// bf16 path: one CTA per (sequence, 128-row query tile, head, key split).  Warp 0 streams Q and
+// K/V tiles with TMA (one copy per 128-row head tile), warp 1 issues tcgen05.mma (S = Q K^T
+// into one of two TMEM buffers, O += P V into a TMEM accumulator), warps 2-5 own one query row
+// per thread: masking, online softmax in the exp2 domain, P (bf16) into one of two swizzled
+// shared-memory buffers, final 1/l scaling (or the unnormalised partial for the combine).  The running maximum is
 // only moved (and O rescaled) when it grows by more than 2^8, so most tiles skip the rescale;
 // the result is exact because numerator and denominator share the reference maximum.
 // fp32 path: one warp per (row, head), SIMT.

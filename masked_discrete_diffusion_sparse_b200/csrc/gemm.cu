@@ -4,10 +4,13 @@
 // the MMA's A operand and the activation rows (up to 512 of them) are its N dimension, so the
 // per-step row count of a sparse step (|A| + |C| + registers, usually < 300) never pads the
 // 128-row MMA M dimension.  Work is split stream-K style: the (tile, 64-wide K chunk) units are
-// divided evenly over one CTA per SM; tiles cut between CTAs are finished by whichever CTA
-// contributes last (fp32 partials in L2-resident scratch, summed in a fixed order so results
-// are deterministic).  Warp roles: warp 0 issues TMA loads, warp 1 owns TMEM and issues
-// tcgen05.mma, warps 2-5 drain the accumulator through the fused epilogue.
+// divided evenly over one CTA (or 2-CTA cluster) per SM (pair); tiles cut between CTAs are
+// finished by whichever CTA contributes last (fp32 partials in L2-resident scratch, summed in a
+// fixed order so results are deterministic).  When the tile count is a large enough share of
+// the grid, every CTA takes one whole tile instead.  Warp roles: warps 0 and 6 issue TMA loads
+// (alternate pipeline stages), warp 1 owns TMEM and issues tcgen05.mma (straight-line per
+// 64-wide K chunk), warps 2-5 drain the accumulator through the fused epilogue, which writes
+// its 32-row blocks with TMA / bulk copies.
 //
 // fp32 path (SIMT FFMA): the same tiles and epilogues for fp32 models, where a tf32 MMA would
 // not hold the 1e-4 tolerance.

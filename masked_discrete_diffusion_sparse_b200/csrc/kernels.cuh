@@ -1,5 +1,6 @@
 // Device-side structures shared by the kernels of the sparse sampling step, the step-causal
-// predicate, and the GEMM epilogues (applied to a staged 16-row x 128-feature fp32 tile).
+// predicate, the launch helper (programmatic dependent launch) and the GEMM epilogues (a staged
+// 16-row tile for the fp32 SIMT GEMM; 32-row TMEM blocks written with TMA copies for tcgen05).
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
