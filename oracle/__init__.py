@@ -271,7 +271,12 @@ class Incremental:
     registers; the K/V they get then are kept for every later step (Figure 3; Sec. 3.2).
     """
 
-    def __init__(self, m: Model, prompt: np.ndarray, gen_len: int):
+    def __init__(self, m: Model, prompt: np.ndarray, gen_len: int,
+                 preset_pos: Optional[Sequence[int]] = None,
+                 preset_tok: Optional[Sequence[int]] = None):
+        """preset_pos / preset_tok: generation positions given from the start (bidirectional
+        tasks: inpainting, outpainting, infilling).  They are clean tokens of block 0, computed
+        with the prompt and cached; the sampler decodes only the other positions."""
         self.m = m
         s = m.shape
         self.P = len(prompt)
@@ -284,15 +289,24 @@ class Incremental:
         self.c_labels = np.zeros(0, dtype=np.int64)
         self.new_pos = np.zeros(0, dtype=np.int64)   # decoded at the previous step
         self.step_k = 0
-        if self.P:
-            self._prefill(np.asarray(prompt, dtype=np.int64))
+        pp = np.zeros(0, dtype=np.int64) if preset_pos is None else np.asarray(preset_pos, np.int64)
+        pt = np.zeros(0, dtype=np.int64) if preset_tok is None else np.asarray(preset_tok, np.int64)
+        if len(pp) != len(pt) or (len(pp) and ((pp <= self.P).any() or (pp > self.L).any()
+                                               or len(np.unique(pp)) != len(pp))):
+            raise ValueError("preset positions must be distinct generation positions")
+        self.grid[pp - self.P - 1] = pt
+        if self.P or len(pp):
+            self._prefill(np.asarray(prompt, dtype=np.int64), pp, pt)
 
-    def _prefill(self, prompt: np.ndarray):
-        """The prompt (block 0) is computed once and its K/V stored (Sec. 3.2)."""
-        pos = np.arange(1, self.P + 1)
-        types = np.full(self.P, PROMPT)
-        labels = np.zeros(self.P, dtype=np.int64)
-        self._run_rows(self.m.emb[prompt], pos, types, labels, keep=np.ones(self.P, bool))
+    def _prefill(self, prompt: np.ndarray, preset_pos: np.ndarray, preset_tok: np.ndarray):
+        """Block 0 — the prompt and any given generation tokens — is computed once and its K/V
+        stored (Sec. 3.2); its rows see each other (label 0)."""
+        n = self.P + len(preset_pos)
+        ids = np.concatenate([prompt, preset_tok]).astype(np.int64)
+        pos = np.concatenate([np.arange(1, self.P + 1), preset_pos])
+        types = np.concatenate([np.full(self.P, PROMPT), np.full(len(preset_pos), CLEAN)])
+        labels = np.zeros(n, dtype=np.int64)
+        self._run_rows(self.m.emb[ids], pos, types, labels, keep=np.ones(n, bool))
 
     def _run_rows(self, x, pos, types, labels, keep) -> np.ndarray:
         """Run all layers for the given rows against the cache; append the `keep` rows' K/V."""
@@ -391,10 +405,13 @@ def query_set(plan: synth.Plan, state: Incremental, k: int) -> np.ndarray:
 
 
 def generate(m: Model, prompt: np.ndarray, gen_len: int, plan: synth.Plan,
-             max_steps: Optional[int] = None, teacher=None) -> Tuple[Incremental, List[StepRecord]]:
+             max_steps: Optional[int] = None, teacher=None,
+             preset_pos: Optional[Sequence[int]] = None,
+             preset_tok: Optional[Sequence[int]] = None) -> Tuple[Incremental, List[StepRecord]]:
     """Full sparse sampling run.  `teacher(k, query_pos, logits, tok, rows)` may return
-    (positions, tokens) to adopt instead of the oracle's own choice (used by parity tests)."""
-    st = Incremental(m, prompt, gen_len)
+    (positions, tokens) to adopt instead of the oracle's own choice (used by parity tests).
+    preset_pos / preset_tok: given generation tokens (bidirectional tasks; see Incremental)."""
+    st = Incremental(m, prompt, gen_len, preset_pos, preset_tok)
     recs = []
     K = plan.n_steps if max_steps is None else min(max_steps, plan.n_steps)
     for k in range(1, K + 1):
@@ -414,12 +431,15 @@ def generate(m: Model, prompt: np.ndarray, gen_len: int, plan: synth.Plan,
 
 
 def trajectory(prompt: np.ndarray, shape: synth.ModelShape, gen_len: int,
-               recs: List[StepRecord], steps: Optional[Sequence[int]] = None):
+               recs: List[StepRecord], steps: Optional[Sequence[int]] = None,
+               preset_pos: Optional[Sequence[int]] = None,
+               preset_tok: Optional[Sequence[int]] = None):
     """Training-form sequence that reproduces the queried steps of a finished run in ONE forward.
 
-    Rows: the prompt (block 0); for every step j the tokens committed at j (clean block j);
-    for every queried step k the decode set C_k as mask rows plus n_reg registers, all labelled
-    k.  Returns (ids, pos, types, labels, {k: row indices of C_k}).
+    Rows: the prompt and any given generation tokens (block 0); for every step j the tokens
+    committed at j (clean block j); for every queried step k the decode set C_k as mask rows
+    plus n_reg registers, all labelled k.  Returns (ids, pos, types, labels,
+    {k: row indices of C_k}).
     """
     P = len(prompt)
     L = P + gen_len
@@ -427,6 +447,11 @@ def trajectory(prompt: np.ndarray, shape: synth.ModelShape, gen_len: int,
     pos = list(range(1, P + 1))
     types = [PROMPT] * P
     labels = [0] * P
+    if preset_pos is not None:
+        ids += list(np.asarray(preset_tok, dtype=np.int64))
+        pos += list(np.asarray(preset_pos, dtype=np.int64))
+        types += [CLEAN] * len(preset_pos)
+        labels += [0] * len(preset_pos)
     for r in recs:
         ids += list(r.committed_tok)
         pos += list(r.committed_pos)

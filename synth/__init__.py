@@ -320,6 +320,46 @@ def make_plan(wl: Workload, seq: int = 0) -> Plan:
     raise ValueError(wl.plan)
 
 
+@dataclass
+class BidirTask:
+    """A bidirectional generation task: some generation positions are given (clean from the
+    start, computed with the prompt) and the plan decodes only the others.
+
+    kind "inpaint": a centred square hole of half the grid side is masked, the rest given;
+    "outpaint": a centred square of half the grid side is given, the rest masked;
+    "infill": a seeded half of the positions (1-D, any workload) is given.
+    preset_pos: 1-based absolute positions (ascending); preset_tok: their token ids."""
+    kind: str
+    preset_pos: np.ndarray
+    preset_tok: np.ndarray
+    plan: Plan
+
+
+def make_bidir_task(wl: Workload, kind: str, seq: int = 0, n_steps: Optional[int] = None) -> BidirTask:
+    g = np.random.Generator(np.random.PCG64([wl.seed, 3000 + seq]))
+    P, Lg = wl.prompt_len, wl.gen_len
+    given = np.zeros(Lg, dtype=bool)
+    if kind in ("inpaint", "outpaint"):
+        side = wl.grid_side
+        if not side or side * side != Lg:
+            raise ValueError("inpaint / outpaint need a square grid workload")
+        lo, hi = side // 4, side // 4 + side // 2
+        centre = np.zeros((side, side), dtype=bool)
+        centre[lo:hi, lo:hi] = True
+        given = (~centre if kind == "inpaint" else centre).reshape(-1)
+    elif kind == "infill":
+        given[g.permutation(Lg)[:Lg // 2]] = True
+    else:
+        raise ValueError(kind)
+    preset_idx = np.flatnonzero(given)
+    masked_idx = np.flatnonzero(~given)
+    preset_tok = g.integers(0, wl.model.vocab, size=len(preset_idx)).astype(np.int32)
+    order = masked_idx[g.permutation(len(masked_idx))]
+    K = min(n_steps if n_steps is not None else wl.n_steps, len(order))
+    plan = Plan("order", K, (order + P + 1).astype(np.int32), cosine_schedule(len(order), K))
+    return BidirTask(kind, (preset_idx + P + 1).astype(np.int32), preset_tok, plan)
+
+
 def semiar_block(plan: Plan, prompt_len: int, k: int):
     """1-based absolute position range [lo, hi) of the block processed at step k (semi-AR)."""
     b = (k - 1) // plan.steps_per_block

@@ -463,3 +463,74 @@ def test_planted_missing_register_visibility_is_caught(monkeypatch):
     ids, pos, types, labels, qrows = oracle.trajectory(prompt, m.shape, st.Lg, recs, steps=[2])
     lg = oracle.forward_stepcausal(m, ids, pos, types, labels, qrows[2])
     assert np.max(np.abs(lg - recs[1].logits)) > 1e-6
+
+
+# ------------------------------------------------------------------------------------------
+# Bidirectional tasks: generation positions given from the start (inpainting, outpainting,
+# infilling).  Given tokens are clean rows of block 0, cached with the prompt.
+# ------------------------------------------------------------------------------------------
+
+def _bidir_run(m, P=6, Lg=24, n_given=10, steps=4, seed=5):
+    g = np.random.Generator(np.random.PCG64(seed))
+    prompt = g.integers(0, m.shape.vocab, P)
+    idx = g.permutation(Lg)
+    given = np.sort(idx[:n_given]) + P + 1
+    given_tok = g.integers(0, m.shape.vocab, n_given)
+    rest = idx[n_given:] + P + 1
+    plan = synth.Plan("order", steps, rest.astype(np.int32),
+                      synth.cosine_schedule(Lg - n_given, steps))
+    st, recs = oracle.generate(m, prompt, Lg, plan, preset_pos=given, preset_tok=given_tok)
+    return prompt, given, given_tok, plan, st, recs
+
+
+def test_bidir_training_form_equals_incremental():
+    """(b) with given generation tokens: the one-forward training form (given tokens as
+    label-0 clean rows) reproduces every cached step of the bidirectional run exactly."""
+    m = tiny_model()
+    prompt, given, given_tok, plan, st, recs = _bidir_run(m)
+    ids, pos, types, labels, qrows = oracle.trajectory(prompt, m.shape, st.Lg, recs,
+                                                       preset_pos=given, preset_tok=given_tok)
+    rows = np.concatenate([qrows[r.k] for r in recs])
+    lg = oracle.forward_stepcausal(m, ids, pos, types, labels, rows)
+    inc = np.concatenate([r.logits for r in recs])
+    assert float(np.max(np.abs(lg - inc))) < 1e-10
+
+
+def test_bidir_given_tokens_stay_and_condition():
+    m = tiny_model()
+    prompt, given, given_tok, plan, st, recs = _bidir_run(m)
+    P = len(prompt)
+    # the given tokens are in the grid from the start and are never overwritten
+    assert (st.grid[given - P - 1] == given_tok).all()
+    assert (st.grid >= 0).all()
+    with pytest.raises(ValueError):
+        st.commit(given[:1], [0])
+    # they condition the generation: another given token changes the first step's logits
+    other = given_tok.copy()
+    other[0] = (other[0] + 1) % m.shape.vocab
+    st2 = oracle.Incremental(m, prompt, st.Lg, given, other)
+    q = plan.query_positions(1)
+    assert np.max(np.abs(st2.step_logits(q) - recs[0].logits)) > 1e-6
+    # and an empty given set is the plain prompt-only run
+    st3 = oracle.Incremental(m, prompt, st.Lg, [], [])
+    st4 = oracle.Incremental(m, prompt, st.Lg)
+    assert np.array_equal(st3.step_logits(q), st4.step_logits(q))
+
+
+def test_bidir_tasks_split_the_generation_region():
+    for name, kinds in (("tiny-bf16-cos", ("inpaint", "outpaint", "infill")),
+                        ("tiny-bf16-semiar", ("infill",))):
+        wl = synth.WORKLOADS[name]
+        for kind in kinds:
+            t = synth.make_bidir_task(wl, kind)
+            gen = set(range(wl.prompt_len + 1, wl.prompt_len + wl.gen_len + 1))
+            given = set(t.preset_pos.tolist())
+            todo = set(t.plan.order.tolist())
+            assert given | todo == gen and not (given & todo)
+            assert int(t.plan.n_per_step.sum()) == len(todo)
+            if kind == "inpaint":     # a centred hole: the masked positions form one square
+                side = wl.grid_side
+                hole = sorted(p - wl.prompt_len - 1 for p in todo)
+                rows = {i // side for i in hole}
+                cols = {i % side for i in hole}
+                assert len(hole) == len(rows) * len(cols) == (side // 2) ** 2
