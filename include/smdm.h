@@ -120,6 +120,18 @@ const char* smdm_last_error(const smdm_handle* h);
 smdm_status smdm_prefill(smdm_handle* h, int seq, const int32_t* d_prompt, int P, int Lgen,
                          int32_t* d_grid, cudaStream_t stream);
 
+/* Prefill with given generation tokens, for bidirectional-context tasks (inpainting,
+ * outpainting, infilling: the paper page's sec. 4.5, Figure 6).  As smdm_prefill, and the
+ * n_given tokens d_given_tok[i] at 1-based absolute positions d_given_pos[i] (distinct, in
+ * P+1..P+Lgen) are clean rows of block 0: computed with the prompt (label 0, bidirectional with
+ * it), cached, and written into d_grid.  Later steps must query only the other positions.
+ * d_given_pos / d_given_tok: device int32 [n_given], read during the call.  A position outside
+ * the generation region or a token id outside the vocabulary sets the device status word
+ * (SMDM_EDEVICE at the next synchronising call); duplicate positions are not detected. */
+smdm_status smdm_prefill_given(smdm_handle* h, int seq, const int32_t* d_prompt, int P, int Lgen,
+                               const int32_t* d_given_pos, const int32_t* d_given_tok,
+                               int n_given, int32_t* d_grid, cudaStream_t stream);
+
 /* One sampling step for one sequence (Figure-3 example; Sec. 3.2; Appendix 7.2).
  * Rows, in this order: the tokens decoded at the previous step of this sequence (new cache:
  * their ids from the grid, label k-1), the decode set C (id [MASK], label k), n_reg registers.

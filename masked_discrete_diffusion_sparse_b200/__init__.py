@@ -30,7 +30,7 @@ STATUS_NAMES = {0: "SMDM_OK", 1: "SMDM_EINVAL", 2: "SMDM_ESHAPE", 3: "SMDM_ENOME
                 4: "SMDM_ECUDA", 5: "SMDM_ESTATE", 6: "SMDM_ETIMEOUT", 7: "SMDM_EDEVICE"}
 
 EXPORTED = ["smdm_workspace_bytes", "smdm_create", "smdm_destroy", "smdm_last_error",
-            "smdm_prefill", "smdm_step", "smdm_dense_step", "smdm_generate",
+            "smdm_prefill", "smdm_prefill_given", "smdm_step", "smdm_dense_step", "smdm_generate",
             "smdm_forward_stepcausal", "smdm_debug_mask", "smdm_debug_rows",
             "smdm_context_length", "smdm_device_status", "smdm_profile_begin",
             "smdm_profile_end", "smdm_forward_stepcausal_noalloc"]
@@ -105,6 +105,8 @@ def lib() -> ctypes.CDLL:
     L.smdm_last_error.restype = ctypes.c_char_p
     L.smdm_prefill.argtypes = [vp, i32, vp, i32, i32, vp, vp]
     L.smdm_prefill.restype = st
+    L.smdm_prefill_given.argtypes = [vp, i32, vp, i32, i32, vp, vp, i32, vp, vp]
+    L.smdm_prefill_given.restype = st
     L.smdm_step.argtypes = [vp, i32, ctypes.POINTER(smdm_step_desc), vp, vp, vp, vp]
     L.smdm_step.restype = st
     L.smdm_dense_step.argtypes = [vp, ctypes.POINTER(smdm_step_desc), vp, vp, vp, vp]
@@ -211,6 +213,19 @@ class Model:
                      stream=None):
         self._check(lib().smdm_prefill(self.h, seq, _ptr(_i32(prompt)) if prompt.numel() else None,
                                        prompt.numel(), gen_len, _ptr(_i32(grid)), _stream(stream)))
+
+    def smdm_prefill_given(self, seq: int, prompt: torch.Tensor, gen_len: int,
+                           given_pos: torch.Tensor, given_tok: torch.Tensor, grid: torch.Tensor,
+                           stream=None):
+        """Prefill with given generation tokens (bidirectional tasks): 1-based absolute
+        positions and their token ids, device int32 tensors of equal length."""
+        if given_pos.numel() != given_tok.numel():
+            raise ValueError("given_pos and given_tok differ in length")
+        n = given_pos.numel()
+        self._check(lib().smdm_prefill_given(
+            self.h, seq, _ptr(_i32(prompt)) if prompt.numel() else None, prompt.numel(), gen_len,
+            _ptr(_i32(given_pos)) if n else None, _ptr(_i32(given_tok)) if n else None, n,
+            _ptr(_i32(grid)), _stream(stream)))
 
     def smdm_step(self, descs: Sequence[dict], logits: Optional[torch.Tensor] = None,
                   tok: Optional[torch.Tensor] = None, conf: Optional[torch.Tensor] = None,

@@ -748,15 +748,23 @@ int smdm_context_length(const smdm_handle* h, int seq) {
   return h->seq[seq].ctx;
 }
 
-smdm_status smdm_prefill(smdm_handle* h, int seq, const int32_t* d_prompt, int P, int Lgen,
-                         int32_t* d_grid, cudaStream_t st) {
+// Block 0 of a sequence: the prompt and (bidirectional tasks) any given generation tokens.
+static smdm_status prefill_block0(smdm_handle* h, int seq, const int32_t* d_prompt, int P,
+                                  int Lgen, const int32_t* d_given_pos,
+                                  const int32_t* d_given_tok, int n_given, int32_t* d_grid,
+                                  cudaStream_t st) {
   if (!h) return SMDM_EINVAL;
   smdm_status s;
   if ((s = check_seq(h, seq))) return s;
   if (P < 0 || Lgen < 1 || P + Lgen > h->cfg.max_len)
     return fail(h, SMDM_ESHAPE, "P=%d, Lgen=%d outside max_len %d", P, Lgen, h->cfg.max_len);
-  if (P > h->cfg.max_rows) return fail(h, SMDM_ESHAPE, "prompt longer than max_rows");
+  if (n_given < 0 || n_given >= Lgen)
+    return fail(h, SMDM_EINVAL, "n_given=%d must leave generation positions to decode", n_given);
+  if (P + n_given > h->cfg.max_rows)
+    return fail(h, SMDM_ESHAPE, "prompt and given tokens longer than max_rows");
   if (!d_grid || (P > 0 && !d_prompt)) return fail(h, SMDM_EINVAL, "null prompt or grid");
+  if (n_given > 0 && (!d_given_pos || !d_given_tok))
+    return fail(h, SMDM_EINVAL, "null given positions or tokens");
   { Launch lg_(h, SMDM_K_OTHER, st); CK(launch_fill_i32(d_grid, Lgen, -1, st)); }
   if (P > 0)
     CK(cudaMemcpyAsync(h->prompt(seq), d_prompt, (size_t)P * 4, cudaMemcpyDeviceToDevice, st));
@@ -765,29 +773,46 @@ smdm_status smdm_prefill(smdm_handle* h, int seq, const int32_t* d_prompt, int P
   q.P = P;
   q.Lg = Lgen;
   q.grid = d_grid;
-  if (P > 0) {
+  const int n0 = P + n_given;   // rows of block 0
+  if (n0 > 0) {
     LinearPackArgs a{};
-    a.mode = kPackPrefill;
-    a.n = P;
+    a.mode = n_given > 0 ? kPackPrefillGiven : kPackPrefill;
+    a.n = n0;
     a.seq = seq;
     a.P = P;
+    a.Lg = Lgen;
     a.vocab = h->cfg.vocab;
     a.emb_rows = h->cfg.vocab + 2 + h->cfg.n_reg;
     a.max_pos = h->L.max_pos;
     a.prompt = h->prompt(seq);
+    a.given_pos = d_given_pos;
+    a.given_tok = d_given_tok;
+    a.grid_out = d_grid;
     a.rows = h->rows;
     a.status = h->status();
     { Launch lg_(h, SMDM_K_PACK, st); CK(launch_pack_linear(a, st)); }
     FwdSpec f{};
-    f.R = P;
+    f.R = n0;
     f.attn_mode = 0;
     f.n_seg = 1;
-    f.seg[0] = AttnSeg{seq, 0, P, P, 0};
+    f.seg[0] = AttnSeg{seq, 0, n0, n0, 0};
     if ((s = forward(h, f, st))) return s;
   }
   q.active = true;
-  q.ctx = P;
+  q.ctx = n0;
   return SMDM_OK;
+}
+
+smdm_status smdm_prefill(smdm_handle* h, int seq, const int32_t* d_prompt, int P, int Lgen,
+                         int32_t* d_grid, cudaStream_t st) {
+  return prefill_block0(h, seq, d_prompt, P, Lgen, nullptr, nullptr, 0, d_grid, st);
+}
+
+smdm_status smdm_prefill_given(smdm_handle* h, int seq, const int32_t* d_prompt, int P, int Lgen,
+                               const int32_t* d_given_pos, const int32_t* d_given_tok,
+                               int n_given, int32_t* d_grid, cudaStream_t st) {
+  return prefill_block0(h, seq, d_prompt, P, Lgen, d_given_pos, d_given_tok, n_given, d_grid,
+                        st);
 }
 
 smdm_status smdm_step(smdm_handle* h, int n_seq, const smdm_step_desc* hd, float* d_logits,

@@ -117,11 +117,22 @@ __global__ void pack_linear_kernel(LinearPackArgs a) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= a.n) return;
   int id, pos, type, label;
-  if (a.mode == kPackPrefill) {
+  if (a.mode == kPackPrefill || (a.mode == kPackPrefillGiven && i < a.P)) {
     id = a.prompt[i];
     pos = i + 1;
     type = kTypePrompt;
     label = 0;
+  } else if (a.mode == kPackPrefillGiven) {
+    // a given generation token: clean, block 0, computed and cached with the prompt
+    id = a.given_tok[i - a.P];
+    pos = a.given_pos[i - a.P];
+    type = kTypeClean;
+    label = 0;
+    if (pos <= a.P || pos > a.P + a.Lg || id < 0 || id >= a.vocab) {
+      atomicOr(a.status, kStatusBounds);
+    } else {
+      a.grid_out[pos - a.P - 1] = id;
+    }
   } else if (a.mode == kPackDense) {
     pos = i + 1;
     if (i < a.P) {

@@ -26,16 +26,20 @@ struct PackArgs {
   uint32_t* status;
 };
 
-enum { kPackPrefill = 0, kPackDense = 1, kPackTrain = 2 };
+enum { kPackPrefill = 0, kPackDense = 1, kPackTrain = 2, kPackPrefillGiven = 3 };
 
 struct LinearPackArgs {
   int mode;
   int n;            // rows
   int seq;
   int P;
+  int Lg;           // prefill with given tokens: generation length
   int vocab, emb_rows, max_pos;
   const int* prompt;    // prefill / dense
   const int* grid;      // dense
+  const int* given_pos; // prefill with given generation tokens: rows P.. are these
+  const int* given_tok;
+  int* grid_out;        // ... and their tokens are written into this grid
   const int* ids;       // training form
   const int* pos;
   const int* type;

@@ -84,12 +84,17 @@ class Runner:
     """Drives one workload on the device and the oracle side by side."""
 
     def __init__(self, wl: synth.Workload, batch: int = 1, gain_std: float = 0.02,
-                 train_rows: int = 0, weights: Optional[synth.Weights] = None):
+                 train_rows: int = 0, weights: Optional[synth.Weights] = None,
+                 tasks: Optional[List[synth.BidirTask]] = None):
+        """tasks: one bidirectional task per sequence (given generation tokens + the plan over
+        the other positions) instead of the workload's own plan."""
         self.wl = wl
         self.batch = batch
         self.w = weights or synth.make_weights(wl.model, wl.seed, gain_std=gain_std)
         self.om = oracle.Model(self.w)
-        self.plans = [synth.make_plan(wl, s) for s in range(batch)]
+        self.tasks = tasks
+        self.plans = ([t.plan for t in tasks] if tasks else
+                      [synth.make_plan(wl, s) for s in range(batch)])
         self.prompts = [synth.make_prompt(wl, s) for s in range(batch)]
         self.cfg = config_for(wl, batch, train_rows, self.plans)
         self.dev_w = upload_weights(self.w)
@@ -114,9 +119,16 @@ def run_teacher_forced(r: Runner, max_steps: Optional[int] = None, check_rows: b
     grids = torch.full((B, Lg), -7, dtype=torch.int32, device="cuda")
     states = []
     for s in range(B):
-        r.model.smdm_prefill(s, i32(r.prompts[s]), Lg, grids[s])
-        states.append(oracle.Incremental(r.om, r.prompts[s], Lg))
-    K = wl.n_steps if max_steps is None else min(max_steps, wl.n_steps)
+        if r.tasks:
+            t = r.tasks[s]
+            r.model.smdm_prefill_given(s, i32(r.prompts[s]), Lg, i32(t.preset_pos),
+                                       i32(t.preset_tok), grids[s])
+            states.append(oracle.Incremental(r.om, r.prompts[s], Lg, t.preset_pos, t.preset_tok))
+        else:
+            r.model.smdm_prefill(s, i32(r.prompts[s]), Lg, grids[s])
+            states.append(oracle.Incremental(r.om, r.prompts[s], Lg))
+    n_steps = min(p.n_steps for p in r.plans)
+    K = n_steps if max_steps is None else min(max_steps, n_steps)
     checks = []
     for k in range(1, K + 1):
         descs, qsets, packs = [], [], []

@@ -111,6 +111,23 @@ def test_sparse_run_register_count(n_reg):
         r.close()
 
 
+@pytest.mark.parametrize("kind", ["inpaint", "infill"])
+def test_bidirectional_task_run(kind):
+    """Bidirectional tasks (given generation tokens as block-0 clean rows, cached with the
+    prompt): teacher-forced sampling of the remaining positions against the oracle."""
+    wl = synth.WORKLOADS["tiny-bf16-cos"]
+    task = synth.make_bidir_task(wl, kind)
+    r = Runner(wl, tasks=[task])
+    try:
+        checks, grids, states = run_teacher_forced(r)
+        _check_all(checks, r.tol)
+        g = grids[0].cpu().numpy()
+        assert (g >= 0).all()
+        assert (g[task.preset_pos - wl.prompt_len - 1] == task.preset_tok).all()
+    finally:
+        r.close()
+
+
 def test_sparse_run_batched_sequences():
     """Three sequences with different prompts and orders in one forward per step."""
     wl = synth.WORKLOADS["tiny-bf16-batch"]
