@@ -404,6 +404,71 @@ def query_set(plan: synth.Plan, state: Incremental, k: int) -> np.ndarray:
     return semiar_queries(state.grid, state.P, lo, hi)
 
 
+class Switched(Incremental):
+    """Sampler state under the speed switches of the pages' Table 6 (the paper notes' ablation
+    section: cache the prompt, cache decoded responses, truncate the masked responses).
+
+    Every switch on is the sparse step of `Incremental`.  Off switches put rows back into each
+    step: cache_prompt=False recomputes the prompt (label 0) every step; cache_res=False
+    recomputes every decoded token (label = the step it was decoded at) every step instead of
+    caching it; truncate=False adds every other still-masked position as a mask row of the step
+    (label k, so the decode set sees it).  The step's rows are ordered by label: prompt,
+    decoded tokens by decode step (then position), the decode set, the other masks, registers.
+    Logits are taken for the decode set only.
+    """
+
+    def __init__(self, m: Model, prompt: np.ndarray, gen_len: int, cache_prompt: bool = True,
+                 cache_res: bool = True, truncate: bool = True):
+        self.cache_prompt, self.cache_res, self.truncate = cache_prompt, cache_res, truncate
+        self.prompt_ids = np.asarray(prompt, dtype=np.int64)
+        self.decoded_at = np.full(gen_len, -1, dtype=np.int64)
+        super().__init__(m, prompt if cache_prompt else np.zeros(0, dtype=np.int64), gen_len)
+        self.P = len(prompt)            # positions stay absolute whether or not the prompt is cached
+        self.L = self.P + gen_len
+
+    def rows(self, query_pos):
+        """(Packed rows of the next step in label order, index of the decode set's first row,
+        keep mask of the rows whose K/V enter the cache)."""
+        s = self.m.shape
+        k = self.step_k + 1
+        P, L = self.P, self.L
+        query_pos = np.asarray(query_pos, dtype=np.int64)
+        ids, pos, types, labels, keep = [], [], [], [], []
+        if not self.cache_prompt:
+            ids += list(self.prompt_ids); pos += list(range(1, P + 1))
+            types += [PROMPT] * P; labels += [0] * P; keep += [False] * P
+        if self.cache_res:
+            dec = np.asarray(self.new_pos, dtype=np.int64)
+        else:
+            done = np.flatnonzero(self.grid >= 0)
+            done = done[np.lexsort((done, self.decoded_at[done]))]   # by decode step, position
+            dec = done + P + 1
+        ids += list(self.grid[dec - P - 1]); pos += list(dec); types += [CLEAN] * len(dec)
+        labels += list(self.decoded_at[dec - P - 1]); keep += [self.cache_res] * len(dec)
+        c0 = len(ids)
+        ids += [s.mask_id] * len(query_pos); pos += list(query_pos)
+        types += [MASK] * len(query_pos); labels += [k] * len(query_pos); keep += [False] * len(query_pos)
+        if not self.truncate:
+            inq = set(query_pos.tolist())
+            rest = [p for p in range(P + 1, L + 1) if self.grid[p - P - 1] < 0 and p not in inq]
+            ids += [s.mask_id] * len(rest); pos += rest; types += [MASK] * len(rest)
+            labels += [k] * len(rest); keep += [False] * len(rest)
+        ids += [s.vocab + 2 + j for j in range(s.n_reg)]; pos += [L + 1 + j for j in range(s.n_reg)]
+        types += [REG] * s.n_reg; labels += [k] * s.n_reg; keep += [False] * s.n_reg
+        a = lambda v: np.asarray(v, dtype=np.int64)
+        return Packed(a(ids), a(pos), a(types), a(labels)), c0, np.asarray(keep, dtype=bool)
+
+    def step_logits(self, query_pos) -> np.ndarray:
+        rows, c0, keep = self.rows(query_pos)
+        self.step_k += 1
+        x = self._run_rows(self.m.emb[rows.ids], rows.pos, rows.types, rows.labels, keep)
+        return self.m.logits(x[c0:c0 + len(query_pos)])
+
+    def commit(self, positions, tokens):
+        super().commit(positions, tokens)
+        self.decoded_at[np.asarray(positions, dtype=np.int64) - self.P - 1] = self.step_k
+
+
 def generate(m: Model, prompt: np.ndarray, gen_len: int, plan: synth.Plan,
              max_steps: Optional[int] = None, teacher=None,
              preset_pos: Optional[Sequence[int]] = None,

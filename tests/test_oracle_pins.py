@@ -534,3 +534,91 @@ def test_bidir_tasks_split_the_generation_region():
                 rows = {i // side for i in hole}
                 cols = {i % side for i in hole}
                 assert len(hole) == len(rows) * len(cols) == (side // 2) ** 2
+
+
+# ------------------------------------------------------------------------------------------
+# Table-6 speed switches (cache prompt / cache responses / truncate)
+# ------------------------------------------------------------------------------------------
+
+SWITCHES = [(cp, cr, tr) for cp in (True, False) for cr in (True, False) for tr in (True, False)]
+
+
+def _replay_switched(m, prompt, Lg, recs, cp, cr, tr):
+    st = oracle.Switched(m, prompt, Lg, cache_prompt=cp, cache_res=cr, truncate=tr)
+    out = []
+    for r in recs:
+        out.append(st.step_logits(r.query_pos))
+        st.commit(r.committed_pos, r.committed_tok)
+    return st, out
+
+
+def test_switches_cache_are_exact():
+    """Caching the prompt and the decoded responses changes only the cost: with truncation on,
+    all four cache settings give the sparse step's decode-set logits (fp64, 1e-10)."""
+    m = tiny_model()
+    prompt, plan, st, recs = _tiny_run(m)
+    for cp, cr, tr in SWITCHES:
+        if not tr:
+            continue
+        _, out = _replay_switched(m, prompt, st.Lg, recs, cp, cr, tr)
+        err = max(float(np.max(np.abs(o - r.logits))) for o, r in zip(out, recs))
+        assert err < 1e-10, (cp, cr, tr, err)
+
+
+def test_switches_without_truncation_match_the_one_forward_form():
+    """Without truncation the step's other masks are mask rows of the step (the decode set sees
+    them), so the logits change; every cache setting still reproduces the one-forward
+    step-labelled form of the same rows exactly."""
+    m = tiny_model()
+    prompt, plan, st, recs = _tiny_run(m)
+    P, Lg = len(prompt), st.Lg
+    ref = None
+    for cp, cr, tr in SWITCHES:
+        if tr:
+            continue
+        _, out = _replay_switched(m, prompt, Lg, recs, cp, cr, tr)
+        if ref is None:
+            ref = out
+            # differs from the truncated step on some step (the other masks are visible)
+            assert max(float(np.max(np.abs(o - r.logits))) for o, r in zip(out, recs)) > 1e-6
+        assert max(float(np.max(np.abs(o - q))) for o, q in zip(out, ref)) < 1e-10
+    # one forward per step: all clean rows so far + this step's masks (C first) + registers
+    sw = oracle.Switched(m, prompt, Lg, cache_prompt=False, cache_res=False, truncate=False)
+    for r, o in zip(recs, ref):
+        rows, c0, _ = sw.rows(r.query_pos)
+        lg = oracle.forward_stepcausal(m, rows.ids, rows.pos, rows.types, rows.labels,
+                                       np.arange(c0, c0 + len(r.query_pos)))
+        assert float(np.max(np.abs(lg - o))) < 1e-10
+        sw.step_k += 1
+        sw.commit(r.committed_pos, r.committed_tok)
+
+
+def test_switches_visible_keys_are_one_range_per_row():
+    """With the step rows ordered by label, every row's visible keys over [cache | step rows]
+    form one contiguous range [lo, hi): lo = cache length for prompt rows recomputed next to a
+    cache of decoded tokens, else 0; hi = cache length + (the step rows with label <= the row's
+    label for clean rows, all step rows for mask and register rows).  Checked against the
+    predicate for every switch setting and step."""
+    m = tiny_model()
+    prompt, plan, st, recs = _tiny_run(m)
+    for cp, cr, tr in SWITCHES:
+        sw = oracle.Switched(m, prompt, st.Lg, cache_prompt=cp, cache_res=cr, truncate=tr)
+        for r in recs:
+            rows, c0, keep = sw.rows(r.query_pos)
+            ctx = sw.ctx
+            kt = np.concatenate([sw.c_types, rows.types])
+            kl = np.concatenate([sw.c_labels, rows.labels])
+            vis = oracle.cross_mask(rows.types, rows.labels, kt, kl)
+            clean = (rows.types == oracle.PROMPT) | (rows.types == oracle.CLEAN)
+            for i in range(rows.n):
+                idx = np.flatnonzero(vis[i])
+                lo, hi = int(idx[0]), int(idx[-1]) + 1
+                assert hi - lo == len(idx), (cp, cr, tr, i)          # contiguous
+                exp_lo = ctx if (clean[i] and rows.labels[i] == 0 and not cp and ctx > 0) else 0
+                if clean[i]:
+                    exp_hi = ctx + int(np.sum(clean & (rows.labels <= rows.labels[i])))
+                else:
+                    exp_hi = ctx + rows.n
+                assert (lo, hi) == (exp_lo, exp_hi), (cp, cr, tr, i, lo, hi, exp_lo, exp_hi)
+            sw.step_logits(r.query_pos)
+            sw.commit(r.committed_pos, r.committed_tok)
