@@ -71,6 +71,21 @@ def token_admissible(tok_dev: np.ndarray, ref_logits: np.ndarray, tol: float) ->
     return ok
 
 
+def topn_commit_admissible(ref_logits: np.ndarray, rows, n_commit: int, tol: float) -> bool:
+    """A TOP-n commit set is admissible when it has min(n, rows) rows and every row in it has an
+    oracle confidence within the tolerance of the oracle's n-th highest confidence: a swapped
+    row is a near-tie.  The tolerance acts on the logit scale, so the confidence (a softmax
+    maximum) may fall by a factor exp(-2 tol scale)."""
+    _, oconf, _ = oracle.unmask(ref_logits, oracle.POLICY_TOPN, n_commit)
+    n = min(n_commit, len(oconf))
+    if len(rows) != n:
+        return False
+    nth = np.sort(oconf)[::-1][n - 1]
+    scale = max(1.0, float(np.max(np.abs(ref_logits))))
+    bound = nth * math.exp(-2 * tol * scale)
+    return all(oconf[int(r)] >= bound for r in rows)
+
+
 @dataclass
 class StepCheck:
     k: int
@@ -199,12 +214,8 @@ def run_teacher_forced(r: Runner, max_steps: Optional[int] = None, check_rows: b
             elif ref is None:
                 commit_ok &= len(cpos) == min(r.plans[s].commit, n_q)
             else:
-                _, oconf, orows = oracle.unmask(ref, oracle.POLICY_TOPN, r.plans[s].commit)
-                nth = np.sort(oconf)[::-1][min(r.plans[s].commit, n_q) - 1]
-                scale = max(1.0, float(np.max(np.abs(ref))))
-                bound = nth * math.exp(-2 * r.tol * scale)
-                commit_ok &= len(cpos) == min(r.plans[s].commit, n_q)
-                commit_ok &= all(oconf[qidx[int(p)]] >= bound for p in cpos)
+                commit_ok &= topn_commit_admissible(ref, [qidx[int(p)] for p in cpos],
+                                                    r.plans[s].commit, r.tol)
             # device grid tokens are the device argmax of the committed rows
             commit_ok &= all(int(ctok[i]) == int(tks[qidx[int(p)]]) for i, p in enumerate(cpos))
             # device grid untouched elsewhere
