@@ -106,7 +106,10 @@ size_t smdm_workspace_bytes(const smdm_config* cfg);
 
 /* Create a handle.  d_workspace: caller-allocated device memory of >= smdm_workspace_bytes,
  * 256-byte aligned; it is initialised here (synchronously, on the legacy default stream).
- * Fails with SMDM_ENOMEM if `bytes` is too small, SMDM_ESHAPE for unsupported shapes. */
+ * Fails with SMDM_ENOMEM if `bytes` is too small, SMDM_ESHAPE for unsupported shapes,
+ * SMDM_EINVAL for a null `out`, null weights or a misaligned workspace (checked on the host,
+ * before any CUDA call), SMDM_ECUDA if a CUDA call fails.  *out is null after any failure.
+ * Every other call returns SMDM_EINVAL for a null handle; smdm_destroy(NULL) does nothing. */
 smdm_status smdm_create(const smdm_config* cfg, const smdm_weights* w, void* d_workspace,
                         size_t bytes, smdm_handle** out);
 void smdm_destroy(smdm_handle* h);

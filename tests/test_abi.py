@@ -70,3 +70,44 @@ def test_model_refuses_to_run_without_cuda():
                            max_step_rows=200, max_rows=300)
     with pytest.raises(RuntimeError):
         smdm.Model(cfg, {})
+
+
+def test_argument_errors_return_before_any_device_work():
+    """The header's error rule: argument errors are reported on the host, before any launch.
+    A null handle or null weights give SMDM_EINVAL, an invalid shape SMDM_ESHAPE, with no CUDA
+    call (this runs without a GPU)."""
+    lib = smdm.lib()
+    E = smdm.SMDM_EINVAL
+    assert lib.smdm_prefill(None, 0, None, 4, 8, None, None) == E
+    assert lib.smdm_prefill_given(None, 0, None, 4, 8, None, None, 0, None, None) == E
+    assert lib.smdm_step(None, 1, None, None, None, None, None) == E
+    assert lib.smdm_dense_step(None, None, None, None, None, None) == E
+    assert lib.smdm_generate(None, 1, None, 4, 8, None, 0, None, None) == E
+    assert lib.smdm_forward_stepcausal(None, None, None, None, None, 1, None, 1, None, None) == E
+    assert lib.smdm_debug_mask(None, None, None, 1, None, None) == E
+    n = ctypes.c_int(0)
+    assert lib.smdm_debug_rows(None, None, None, None, None, ctypes.byref(n), None) == E
+    assert lib.smdm_profile_begin(None, 1) == E
+    assert lib.smdm_profile_end(None, None, None) == E
+    bits = ctypes.c_uint(0)
+    assert lib.smdm_device_status(None, ctypes.byref(bits), None) == E
+    assert lib.smdm_context_length(None, 0) == -1
+    assert lib.smdm_last_error(None) == b"null handle"
+    lib.smdm_destroy(None)
+
+    good = smdm.make_config(2, 256, 2, 128, 704, 1000, dtype=smdm.SMDM_BF16, max_batch=1,
+                            max_len=300, max_step_rows=200, max_rows=300)
+    bad = smdm.make_config(2, 192, 3, 64, 704, 1000, dtype=smdm.SMDM_BF16, max_batch=1,
+                           max_len=300, max_step_rows=200, max_rows=300)
+    out = ctypes.c_void_p(1)
+    assert lib.smdm_create(ctypes.byref(bad), None, None, 0, ctypes.byref(out)) == \
+        smdm.SMDM_ESHAPE
+    assert out.value is None                       # *out is cleared on every failure
+    assert lib.smdm_create(ctypes.byref(good), None, None, 0, ctypes.byref(out)) == E
+    assert lib.smdm_create(ctypes.byref(good), None, None, 0, None) == E
+    w = smdm.smdm_weights()                        # every pointer null
+    assert lib.smdm_forward_stepcausal_noalloc(ctypes.byref(good), ctypes.byref(w), None, None,
+                                               None, None, 4, None, 1, None, None) == E
+    assert lib.smdm_forward_stepcausal_noalloc(ctypes.byref(bad), ctypes.byref(w), None, None,
+                                               None, None, 4, None, 1, None, None) == \
+        smdm.SMDM_ESHAPE
