@@ -1,4 +1,4 @@
-"""The host side of the parity protocol (the judgement the GPU parity tests make): the logit error
+"""The host side of the parity protocol (the decision the GPU parity tests take): the logit error
 relative to the logit scale, token admissibility at near-ties and the TOP-n commit rule.  These
 run on CPU with hand-made logits whose answers are known."""
 import numpy as np
