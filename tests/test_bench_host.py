@@ -52,3 +52,52 @@ def test_step_shapes_cover_every_generated_token():
         assert sum(q for (_, q, _, _) in shapes) == wl.gen_len
         for (R, q, ctx, n_new) in shapes:
             assert R == n_new + q + wl.model.n_reg
+
+
+def test_streamed_parameters_per_step():
+    """Weights streamed by one sampling step (every layer plus the LM head) for the five model
+    shapes: 1.84 M, 135.5 M, 843.1 M (both text-to-image sizes) and 1652.6 M parameters."""
+    b = _bench()
+    # (millions, half a unit of the last digit given)
+    expect = {"A": (1.84, 0.005), "B": (135.5, 0.05), "C": (843.1, 0.05), "D": (843.1, 0.05),
+              "E": (1652.6, 0.05)}
+    for name, (n, half) in expect.items():
+        m = synth.WORKLOADS[name].model
+        got = (m.n_layers * b.layer_params(m) + m.vocab * m.d_model) / 1e6
+        assert abs(got - n) <= half, (name, got)
+
+
+def _cache_before(P, recs, k):
+    """(types, labels) of the oracle's KV cache before step k: the prompt, then the tokens
+    committed at steps 1..k-2 (the ones of step k-1 are step k's new-cache rows)."""
+    types = [oracle.PROMPT] * P
+    labels = [0] * P
+    for r in recs[:max(k - 2, 0)]:
+        types += [oracle.CLEAN] * len(r.committed_pos)
+        labels += [r.k] * len(r.committed_pos)
+    return np.array(types), np.array(labels)
+
+
+def test_step_shapes_and_attention_work_match_the_oracle_run():
+    """The bench's per-step shapes (rows, decode rows, cache length, new-cache rows) and its
+    attention work (sum over rows of visible keys) equal what the oracle's sampling run packs
+    and what its step-causal predicate allows, for an order plan and a semi-AR plan."""
+    b = _bench()
+    for name in ("tiny-f32-cos", "tiny-bf16-semiar"):
+        wl = synth.WORKLOADS[name]
+        plan = synth.make_plan(wl, 0)
+        prompt = synth.make_prompt(wl, 0)
+        om = oracle.Model(synth.make_weights(wl.model, wl.seed))
+        st, recs = oracle.generate(om, prompt, wl.gen_len, plan)
+        shapes = b.step_shapes(wl, plan)
+        assert len(shapes) == len(recs)
+        for (R, q, ctx, n_new), r in zip(shapes, recs):
+            pk = r.packed
+            assert R == pk.n and q == len(r.query_pos), (name, r.k)
+            assert n_new == int(np.sum(pk.types == oracle.CLEAN)), (name, r.k)
+            ct, cl = _cache_before(wl.prompt_len, recs, r.k)
+            assert ctx == len(ct), (name, r.k)
+            vis = oracle.cross_mask(pk.types, pk.labels, np.concatenate([ct, pk.types]),
+                                    np.concatenate([cl, pk.labels]))
+            kv_sum = n_new * (ctx + n_new) + (R - n_new) * (ctx + R)
+            assert kv_sum == int(vis.sum()), (name, r.k)
