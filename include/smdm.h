@@ -185,7 +185,11 @@ typedef struct {
 /* Full generation of `batch` sequences (slots 0..batch-1) with the same P, Lgen and step
  * count: prefill, then K steps.  d_prompts: int32 [batch][P]; plans: host [batch];
  * d_grids: int32 [batch][Lgen] (output).  mode SMDM_MODE_SPARSE batches the sequences into
- * one forward per step; SMDM_MODE_DENSE runs the dense comparator step per sequence. */
+ * one forward per step; SMDM_MODE_DENSE runs the dense comparator step per sequence.
+ * The whole plan is checked on the host before any work (step sizes, their sum, P + Lgen
+ * against max_len and, in sparse mode, every step's rows against max_step_rows and the
+ * batched rows against max_rows): a bad plan returns SMDM_EINVAL / SMDM_ESHAPE with no
+ * sequence changed. */
 smdm_status smdm_generate(smdm_handle* h, int batch, const int32_t* d_prompts, int P, int Lgen,
                           const smdm_plan* plans, int mode, int32_t* d_grids,
                           cudaStream_t stream);

@@ -165,6 +165,10 @@ bool config_ok(const smdm_config* c, std::string* why) {
   if (c->d_model > 8192) return fail("d_model > 8192 is not supported");
   if (c->max_batch < 1 || c->max_batch > SMDM_MAX_BATCH) return fail("max_batch out of range");
   if (c->max_len < 1 || c->max_step_rows < 1 || c->max_rows < 1) return fail("bad capacity");
+  // positions, cache slots and row indices are 32-bit on the device
+  if ((long long)c->max_len + c->max_step_rows + c->n_reg + 8 > (1LL << 30) ||
+      c->max_rows > (1 << 24) || c->n_reg > (1 << 16))
+    return fail("capacity too large");
   if (c->dtype == SMDM_BF16) {
     if (c->d_model % 128) return fail("bf16 models need d_model % 128 == 0");
     if (c->d_head != 64 && c->d_head != 128) return fail("bf16 models need d_head 64 or 128");
@@ -987,6 +991,14 @@ smdm_status smdm_generate(smdm_handle* h, int batch, const int32_t* d_prompts, i
   if (mode != SMDM_MODE_SPARSE && mode != SMDM_MODE_DENSE)
     return fail(h, SMDM_EINVAL, "unknown mode %d", mode);
   const int K = plans[0].n_steps;
+  if (P < 0 || Lgen < 1 || (long long)P + Lgen > h->cfg.max_len)
+    return fail(h, SMDM_ESHAPE, "P=%d, Lgen=%d outside max_len %d", P, Lgen, h->cfg.max_len);
+  if (K < 1 || K > Lgen) return fail(h, SMDM_EINVAL, "step count %d outside [1, Lgen]", K);
+  // Whole-plan checks before any work, so that a bad plan leaves every sequence untouched.
+  // Rows of sparse step k for one sequence: the tokens committed at step k-1 (new-cache rows),
+  // the decode set and the registers; they must fit max_step_rows, and a batched step's rows
+  // summed over the sequences must fit max_rows (the checks smdm_step makes per step).
+  std::vector<long long> batch_rows(K, 0);
   for (int b = 0; b < batch; ++b) {
     const smdm_plan& p = plans[b];
     if (p.n_steps != K || K < 1) return fail(h, SMDM_EINVAL, "plans need the same step count");
@@ -1005,7 +1017,27 @@ smdm_status smdm_generate(smdm_handle* h, int batch, const int32_t* d_prompts, i
     } else {
       return fail(h, SMDM_EINVAL, "unknown plan kind");
     }
+    for (int k = 0; k < K; ++k) {
+      long long n_new, n_q;
+      if (p.kind == SMDM_PLAN_ORDER) {
+        n_new = k ? p.h_n_per_step[k - 1] : 0;
+        n_q = p.h_n_per_step[k];
+      } else {
+        n_new = k ? p.commit : 0;
+        n_q = p.block - (long long)(k % p.steps_per_block) * p.commit;
+      }
+      const long long rows = n_new + n_q + h->cfg.n_reg;
+      if (mode == SMDM_MODE_SPARSE && rows > h->cfg.max_step_rows)
+        return fail(h, SMDM_ESHAPE, "plan %d step %d needs %lld rows, max_step_rows is %d", b,
+                    k + 1, rows, h->cfg.max_step_rows);
+      batch_rows[k] += rows;
+    }
   }
+  if (mode == SMDM_MODE_SPARSE)
+    for (int k = 0; k < K; ++k)
+      if (batch_rows[k] > h->cfg.max_rows)
+        return fail(h, SMDM_ESHAPE, "batched step %d needs %lld rows, max_rows is %d", k + 1,
+                    batch_rows[k], h->cfg.max_rows);
   smdm_status s;
   for (int b = 0; b < batch; ++b)
     if ((s = smdm_prefill(h, b, d_prompts + (size_t)b * P, P, Lgen, d_grids + (size_t)b * Lgen, st)))

@@ -111,3 +111,14 @@ def test_argument_errors_return_before_any_device_work():
     assert lib.smdm_forward_stepcausal_noalloc(ctypes.byref(bad), ctypes.byref(w), None, None,
                                                None, None, 4, None, 1, None, None) == \
         smdm.SMDM_ESHAPE
+
+
+def test_capacities_that_overflow_32_bit_indices_are_rejected():
+    lib = smdm.lib()
+    base = dict(dtype=smdm.SMDM_BF16, max_batch=1, max_step_rows=200, max_rows=300)
+    ok = smdm.make_config(2, 256, 2, 128, 704, 1000, max_len=300, **base)
+    assert lib.smdm_workspace_bytes(ctypes.byref(ok)) > 0
+    huge = smdm.make_config(2, 256, 2, 128, 704, 1000, max_len=(1 << 30), **base)
+    assert lib.smdm_workspace_bytes(ctypes.byref(huge)) == 0
+    regs = smdm.make_config(2, 256, 2, 128, 704, 1000, n_reg=(1 << 17), max_len=300, **base)
+    assert lib.smdm_workspace_bytes(ctypes.byref(regs)) == 0
