@@ -227,6 +227,18 @@ def forward_stepcausal(m: Model, ids, pos, types, labels, logit_rows) -> np.ndar
 # (papernotes "a complete example" / Figure 3; paperlayer Sec. 3.2)
 # ----------------------------------------------------------------------------------------------
 
+def tail_rows(shape: synth.ModelShape, L: int) -> Tuple[List[int], List[int]]:
+    """(ids, positions) of the rows that close a step's sequence and stand for its truncated
+    masks (papernotes "Key design 2"; paperlayer Sec. 3.1, Appendix 7.2): n_reg registers
+    REG_0.. at positions L+1..L+n_reg.  The register-count ablation (the paper notes' Table 7)
+    has a 0-register row: read as the single length token the notes describe before registers
+    were added, one [LEN] row at position L+1 (``shape.len_token``).  Either kind takes the
+    type REG and the step's label: it follows the masked block's attention rule."""
+    if shape.n_reg == 0 and shape.len_token:
+        return [shape.len_id], [L + 1]
+    return [shape.reg_id(j) for j in range(shape.n_reg)], [L + 1 + j for j in range(shape.n_reg)]
+
+
 @dataclass
 class Packed:
     """The sparse rows of one step: [new-cache | query | register]."""
@@ -245,19 +257,20 @@ def pack_step(shape: synth.ModelShape, prompt_len: int, gen_len: int, grid: np.n
     """Rows fed to the network at step k (paperlayer Appendix 7.2: |A| + |C| + m tokens).
 
     new_pos: positions decoded at step k-1 (enter the cache this step, label k-1, their ids
-    read from the grid); query_pos: the decode set C_k (id [MASK], label k); then n_reg
-    registers with ids REG_0.. and position ids L+1..L+n_reg (label k).
+    read from the grid); query_pos: the decode set C_k (id [MASK], label k); then the tail rows
+    (`tail_rows`: n_reg registers with ids REG_0.. and position ids L+1..L+n_reg, label k).
     """
     L = prompt_len + gen_len
     new_pos = np.asarray(new_pos, dtype=np.int64)
     query_pos = np.asarray(query_pos, dtype=np.int64)
-    n_new, n_q, m = len(new_pos), len(query_pos), shape.n_reg
+    t_ids, t_pos = tail_rows(shape, L)
+    n_new, n_q, m = len(new_pos), len(query_pos), len(t_ids)
     ids = np.concatenate([grid[new_pos - prompt_len - 1],
                           np.full(n_q, shape.mask_id),
-                          shape.vocab + 2 + np.arange(m)]).astype(np.int64)
+                          np.asarray(t_ids, dtype=np.int64)]).astype(np.int64)
     if n_new and (ids[:n_new] < 0).any():
         raise ValueError("new-cache position is still masked")
-    pos = np.concatenate([new_pos, query_pos, L + 1 + np.arange(m)]).astype(np.int64)
+    pos = np.concatenate([new_pos, query_pos, np.asarray(t_pos, dtype=np.int64)]).astype(np.int64)
     types = np.concatenate([np.full(n_new, CLEAN), np.full(n_q, MASK), np.full(m, REG)])
     labels = np.concatenate([np.full(n_new, k - 1), np.full(n_q, k), np.full(m, k)])
     return Packed(ids, pos, types.astype(np.int64), labels.astype(np.int64))
@@ -453,8 +466,9 @@ class Switched(Incremental):
             rest = [p for p in range(P + 1, L + 1) if self.grid[p - P - 1] < 0 and p not in inq]
             ids += [s.mask_id] * len(rest); pos += rest; types += [MASK] * len(rest)
             labels += [k] * len(rest); keep += [False] * len(rest)
-        ids += [s.vocab + 2 + j for j in range(s.n_reg)]; pos += [L + 1 + j for j in range(s.n_reg)]
-        types += [REG] * s.n_reg; labels += [k] * s.n_reg; keep += [False] * s.n_reg
+        t_ids, t_pos = tail_rows(s, L)
+        ids += t_ids; pos += t_pos
+        types += [REG] * len(t_ids); labels += [k] * len(t_ids); keep += [False] * len(t_ids)
         a = lambda v: np.asarray(v, dtype=np.int64)
         return Packed(a(ids), a(pos), a(types), a(labels)), c0, np.asarray(keep, dtype=bool)
 
@@ -503,7 +517,7 @@ def trajectory(prompt: np.ndarray, shape: synth.ModelShape, gen_len: int,
 
     Rows: the prompt and any given generation tokens (block 0); for every step j the tokens
     committed at j (clean block j); for every queried step k the decode set C_k as mask rows
-    plus n_reg registers, all labelled k.  Returns (ids, pos, types, labels,
+    plus its tail rows (`tail_rows`), all labelled k.  Returns (ids, pos, types, labels,
     {k: row indices of C_k}).
     """
     P = len(prompt)
@@ -528,10 +542,11 @@ def trajectory(prompt: np.ndarray, shape: synth.ModelShape, gen_len: int,
             continue
         start = len(ids)
         nq = len(r.query_pos)
-        ids += [shape.mask_id] * nq + [shape.vocab + 2 + j for j in range(shape.n_reg)]
-        pos += list(r.query_pos) + [L + 1 + j for j in range(shape.n_reg)]
-        types += [MASK] * nq + [REG] * shape.n_reg
-        labels += [r.k] * (nq + shape.n_reg)
+        t_ids, t_pos = tail_rows(shape, L)
+        ids += [shape.mask_id] * nq + t_ids
+        pos += list(r.query_pos) + t_pos
+        types += [MASK] * nq + [REG] * len(t_ids)
+        labels += [r.k] * (nq + len(t_ids))
         qrows[r.k] = np.arange(start, start + nq)
     return (np.array(ids), np.array(pos), np.array(types), np.array(labels), qrows)
 

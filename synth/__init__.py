@@ -52,6 +52,11 @@ class ModelShape:
     dtype: str = BF16
     rope_theta: float = 10000.0
     rms_eps: float = 1e-6
+    len_token: bool = False   # with n_reg == 0: the length-token variant (one [LEN] row per step)
+
+    def __post_init__(self):
+        if self.len_token and self.n_reg != 0:
+            raise ValueError("the length-token variant has no registers (n_reg == 0)")
 
     @property
     def emb_rows(self) -> int:

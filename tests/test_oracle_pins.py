@@ -622,3 +622,39 @@ def test_switches_visible_keys_are_one_range_per_row():
                 assert (lo, hi) == (exp_lo, exp_hi), (cp, cr, tr, i, lo, hi, exp_lo, exp_hi)
             sw.step_logits(r.query_pos)
             sw.commit(r.committed_pos, r.committed_tok)
+
+
+# ------------------------------------------------------------------------------------------
+# Length-token variant (the 0-register row of the register-count ablation): one [LEN] row at
+# L+1 instead of registers, under the masked block's attention rule.
+# ------------------------------------------------------------------------------------------
+
+def test_length_token_variant_rows():
+    """The worked example with the length token: 3 clean + 4 masks + one [LEN] row at L+1 = 8
+    (the sparse sequence carries the clean tokens, their positions and the length)."""
+    g = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    vocab = {w: i for i, w in enumerate(["I", "have", "dog"])}
+    shape = synth.ModelShape(1, 8, 1, 8, 8, 3, n_reg=0, dtype=synth.F32, len_token=True)
+    L = g["length"]
+    grid = np.full(L, -1)
+    for t, p in zip(g["clean"], g["positions"]):
+        grid[p - 1] = vocab[t]
+    masked = [p for p in range(1, L + 1) if p not in g["positions"]]
+    rows = oracle.pack_step(shape, 0, L, grid, g["positions"], masked, k=2)
+    assert rows.n == len(g["positions"]) + len(masked) + 1
+    assert rows.ids[-1] == shape.len_id == shape.vocab + 1
+    assert rows.pos[-1] == L + 1 and rows.types[-1] == oracle.REG and rows.labels[-1] == 2
+    with pytest.raises(ValueError):
+        synth.ModelShape(1, 8, 1, 8, 8, 3, n_reg=4, len_token=True)
+
+
+def test_length_token_training_form_equals_incremental():
+    """Invariant (b) with the length-token variant: the one-forward trajectory form reproduces
+    every cached step, and the [LEN] row does condition the decode set (dropping it changes
+    the logits)."""
+    m = tiny_model(n_reg=0, len_token=True)
+    assert check_training_equals_incremental(m) < 1e-10
+    prompt, plan, st, recs = _tiny_run(m)
+    bare = oracle.Model(synth.make_weights(tiny_shape(0), 7, gain_std=0.1, std=0.25))
+    st0, recs0 = oracle.generate(bare, prompt, st.Lg, plan, max_steps=1)
+    assert np.max(np.abs(recs0[0].logits - recs[0].logits)) > 1e-3
