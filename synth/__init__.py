@@ -281,8 +281,9 @@ class Plan:
 
     kind == "order": step k (1-based) queries order[offsets[k-1]:offsets[k]] and commits all of
     them.  kind == "semiar": blocks of `block` generation positions are processed left to
-    right; at each step the query set is every still-masked position of the current block and
-    the `commit` most confident are committed.
+    right, or in the order `block_order` gives (block indices from 0; a bidirectional task may
+    decode a middle block first); at each step the query set is every still-masked position of
+    the current block and the `commit` most confident are committed.
     Positions are 1-based absolute positions (P+1..P+Lg).
     """
     kind: str
@@ -292,6 +293,7 @@ class Plan:
     block: int = 0
     steps_per_block: int = 0
     commit: int = 0
+    block_order: Optional[np.ndarray] = None  # semiar: processing order of the blocks
 
     @property
     def offsets(self) -> np.ndarray:
@@ -368,6 +370,8 @@ def make_bidir_task(wl: Workload, kind: str, seq: int = 0, n_steps: Optional[int
 def semiar_block(plan: Plan, prompt_len: int, k: int):
     """1-based absolute position range [lo, hi) of the block processed at step k (semi-AR)."""
     b = (k - 1) // plan.steps_per_block
+    if plan.block_order is not None:
+        b = int(plan.block_order[b])
     lo = prompt_len + 1 + b * plan.block
     return lo, lo + plan.block
 
