@@ -90,7 +90,7 @@ def topn_commit_admissible(ref_logits: np.ndarray, rows, n_commit: int, tol: flo
 class StepCheck:
     k: int
     err: float
-    rows_exact: bool
+    rows_exact: bool     # packed rows and every sequence's KV-cache length, bit-exact
     tok_ok: bool
     commit_ok: bool
 
@@ -142,6 +142,10 @@ def run_teacher_forced(r: Runner, max_steps: Optional[int] = None, check_rows: b
         else:
             r.model.smdm_prefill(s, i32(r.prompts[s]), Lg, grids[s])
             states.append(oracle.Incremental(r.om, r.prompts[s], Lg))
+    # Expected KV-cache length per sequence: block 0 after prefill; a step appends the tokens
+    # committed at the step before it (its new-cache rows).
+    ctx_exp = [len(st.c_types) for st in states]
+    prev_commit = [0] * B
     n_steps = min(p.n_steps for p in r.plans)
     K = n_steps if max_steps is None else min(max_steps, n_steps)
     checks = []
@@ -223,6 +227,11 @@ def run_teacher_forced(r: Runner, max_steps: Optional[int] = None, check_rows: b
             untouched[newly] = False
             commit_ok &= bool(np.array_equal(grid_before[s][untouched], grid_after[s][untouched]))
             st.commit(cpos, ctok)   # teacher forcing: adopt the device's choice
+            ctx_exp[s] += prev_commit[s]
+            prev_commit[s] = len(cpos)
+            rows_exact &= r.model.smdm_context_length(s) == ctx_exp[s]
+            if with_logits:
+                rows_exact &= len(st.c_types) == ctx_exp[s]
             off += n_q
         checks.append(StepCheck(k, err, rows_exact, tok_ok, commit_ok))
     for s in range(B):
