@@ -228,6 +228,18 @@ class OracleSample:
         return dt, n_dec, desc, _blas_threads()
 
 
+def _cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def _blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -253,14 +265,14 @@ def run_reference(args, wl):
         if i >= args.warmup:
             times.append(dt)
     mean = sum(times) / len(times)
-    value = n_dec * wl.batch / mean
+    value = n_dec / mean          # the sample decodes one sequence
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": mean * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": describe(wl),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": desc},
+                             "sample": desc, "cpu": _cpu_model()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -597,8 +609,9 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu:
         try:
             dt, n_dec, desc, threads = OracleSample(wl).run()
-            line["cpu_baseline"] = {"value": n_dec * B / dt, "unit": UNIT, "cores": threads,
-                                    "kind": "oracle", "sample": desc, "seconds": dt}
+            line["cpu_baseline"] = {"value": n_dec / dt, "unit": UNIT, "cores": threads,
+                                    "kind": "oracle", "sample": desc, "seconds": dt,
+                                    "cpu": _cpu_model()}
         except MemoryError:
             line["cpu_baseline"] = None
     if rank == 0:
