@@ -122,3 +122,37 @@ def test_capacities_that_overflow_32_bit_indices_are_rejected():
     assert lib.smdm_workspace_bytes(ctypes.byref(huge)) == 0
     regs = smdm.make_config(2, 256, 2, 128, 704, 1000, n_reg=(1 << 17), max_len=300, **base)
     assert lib.smdm_workspace_bytes(ctypes.byref(regs)) == 0
+
+
+def test_binding_struct_layouts_match_the_header(tmp_path):
+    """Every ABI struct of the Python binding has the size and field offsets that a C compiler
+    gives the header's struct (a program compiled here against include/smdm.h prints them)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    structs = {"smdm_config": smdm.smdm_config, "smdm_weights": smdm.smdm_weights,
+               "smdm_step_desc": smdm.smdm_step_desc, "smdm_plan": smdm.smdm_plan,
+               "smdm_profile": smdm.smdm_profile}
+    lines = ['#include <stdio.h>', '#include "smdm.h"', "int main(void) {"]
+    for name, cls in structs.items():
+        lines.append(f'  printf("{name} size %zu\\n", sizeof({name}));')
+        for f in cls._fields_:
+            lines.append(f'  printf("{name} {f[0]} %zu\\n", offsetof({name}, {f[0]}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, str(src), "-o",
+                    str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True,
+                               text=True).stdout.splitlines():
+        name, field, value = line.split()
+        got[(name, field)] = int(value)
+    for name, cls in structs.items():
+        assert got[(name, "size")] == ctypes.sizeof(cls), name
+        for f in cls._fields_:
+            assert got[(name, f[0])] == getattr(cls, f[0]).offset, (name, f[0])
