@@ -180,6 +180,9 @@ typedef struct {
   int block;                  /* SEMIAR: block length (Lgen % block == 0) */
   int steps_per_block;        /* SEMIAR */
   int commit;                 /* SEMIAR: tokens committed per step (block == steps * commit) */
+  const int32_t* h_block_order; /* SEMIAR, optional: host [Lgen / block], the order in which the
+                                   blocks are decoded (a permutation of 0 .. Lgen/block - 1;
+                                   NULL = left to right) */
 } smdm_plan;
 
 /* Full generation of `batch` sequences (slots 0..batch-1) with the same P, Lgen and step

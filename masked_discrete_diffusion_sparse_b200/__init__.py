@@ -73,7 +73,7 @@ class smdm_plan(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("n_steps", ctypes.c_int),
                 ("h_n_per_step", ctypes.POINTER(ctypes.c_int32)), ("d_order", ctypes.c_void_p),
                 ("block", ctypes.c_int), ("steps_per_block", ctypes.c_int),
-                ("commit", ctypes.c_int)]
+                ("commit", ctypes.c_int), ("h_block_order", ctypes.POINTER(ctypes.c_int32))]
 
 
 class smdm_profile(ctypes.Structure):
@@ -252,7 +252,7 @@ class Model:
     def smdm_generate(self, prompts: torch.Tensor, gen_len: int, plans: Sequence[dict],
                       grids: torch.Tensor, mode: int = SMDM_MODE_SPARSE, stream=None):
         """plans: dicts with kind, n_steps, n_per_step (host int list), order (int32 CUDA
-        tensor), block, steps_per_block, commit."""
+        tensor), block, steps_per_block, commit, block_order (host int list, optional)."""
         B = len(plans)
         arr = (smdm_plan * B)()
         keep = []
@@ -262,11 +262,17 @@ class Model:
             if nps is not None:
                 h_n = (ctypes.c_int32 * len(nps))(*[int(v) for v in nps])
                 keep.append(h_n)
+            bo = p.get("block_order")
+            h_bo = None
+            if bo is not None:
+                h_bo = (ctypes.c_int32 * len(bo))(*[int(v) for v in bo])
+                keep.append(h_bo)
             order = p.get("order")
             arr[i] = smdm_plan(p["kind"], p["n_steps"],
                                ctypes.cast(h_n, ctypes.POINTER(ctypes.c_int32)) if h_n else None,
                                _ptr(_i32(order)) if order is not None else None,
-                               p.get("block", 0), p.get("steps_per_block", 0), p.get("commit", 0))
+                               p.get("block", 0), p.get("steps_per_block", 0), p.get("commit", 0),
+                               ctypes.cast(h_bo, ctypes.POINTER(ctypes.c_int32)) if h_bo else None)
         P = prompts.shape[-1] if prompts.numel() else 0
         self._check(lib().smdm_generate(self.h, B, _ptr(_i32(prompts)) if P else None, P, gen_len,
                                         arr, mode, _ptr(_i32(grids)), _stream(stream)))

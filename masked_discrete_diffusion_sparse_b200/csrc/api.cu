@@ -1014,6 +1014,16 @@ smdm_status smdm_generate(smdm_handle* h, int batch, const int32_t* d_prompts, i
       if (p.block < 1 || p.commit < 1 || p.steps_per_block < 1 || Lgen % p.block ||
           p.block != p.steps_per_block * p.commit || K != (Lgen / p.block) * p.steps_per_block)
         return fail(h, SMDM_EINVAL, "inconsistent SEMIAR plan");
+      if (p.h_block_order) {
+        const int nb = Lgen / p.block;
+        std::vector<char> seen(nb, 0);
+        for (int i = 0; i < nb; ++i) {
+          const int v = p.h_block_order[i];
+          if (v < 0 || v >= nb || seen[v])
+            return fail(h, SMDM_EINVAL, "block order of plan %d is not a permutation", b);
+          seen[v] = 1;
+        }
+      }
     } else {
       return fail(h, SMDM_EINVAL, "unknown plan kind");
     }
@@ -1057,7 +1067,8 @@ smdm_status smdm_generate(smdm_handle* h, int batch, const int32_t* d_prompts, i
         d.n_commit = d.n_query;
         off[b] += d.n_query;
       } else {
-        const int blk = (k - 1) / p.steps_per_block, j = (k - 1) % p.steps_per_block;
+        const int nth = (k - 1) / p.steps_per_block, j = (k - 1) % p.steps_per_block;
+        const int blk = p.h_block_order ? p.h_block_order[nth] : nth;
         d.d_query_pos = nullptr;
         d.block_lo = P + 1 + blk * p.block;
         d.block_hi = d.block_lo + p.block;
