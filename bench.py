@@ -56,8 +56,9 @@ def parse():
                     help="sampling: full sparse sampling runs (the headline); training: one "
                          "training-form forward over a whole step-labelled trajectory")
     ap.add_argument("--n-reg", type=int, default=None,
-                    help="register rows per step (the method's 64 by default); for the "
-                         "register-count sensitivity study")
+                    help="register rows per step (the method's 64 by default; 0 = the "
+                         "length-token variant, one [LEN] row); for the register-count "
+                         "sensitivity study")
     return ap.parse_args()
 
 
@@ -70,7 +71,8 @@ def describe(wl: synth.Workload) -> dict:
     return {"workload": {"A": "tiny-fp32", "B": "text-semiAR", "C": "T2I-1024", "D": "T2I-4096",
                          "D4": "T2I-4096-batch4", "E": "image-editing"}.get(wl.name, wl.name),
             "layers": m.n_layers, "d_model": m.d_model, "heads": f"{m.n_heads}x{m.d_head}",
-            "d_ffn": m.d_ffn, "vocab": m.vocab, "registers": m.n_reg, "prompt": wl.prompt_len,
+            "d_ffn": m.d_ffn, "vocab": m.vocab,
+            "registers": "[LEN]" if m.len_token else m.n_reg, "prompt": wl.prompt_len,
             "gen_len": wl.gen_len, "sampling_steps": wl.n_steps, "batch": wl.batch,
             "plan": wl.plan}
 
@@ -88,7 +90,7 @@ def step_shapes(wl: synth.Workload, plan: synth.Plan):
             j = (k - 1) % plan.steps_per_block
             q = plan.block - j * plan.commit
             c = plan.commit
-        R = n_new + q + m.n_reg
+        R = n_new + q + m.n_tail
         out.append((R, q, ctx, n_new))
         ctx += n_new
         n_new = c
@@ -334,10 +336,14 @@ def trajectory_rows(wl: synth.Workload, plan: synth.Plan, prompt: np.ndarray, se
         pos += list(q)
         types += [2] * n
         labels += [k] * n
-        ids += [m.vocab + 2 + j for j in range(m.n_reg)]
-        pos += [L + 1 + j for j in range(m.n_reg)]
-        types += [3] * m.n_reg
-        labels += [k] * m.n_reg
+        if m.len_token:                       # the one [LEN] row
+            ids += [m.vocab + 1]
+            pos += [L + 1]
+        else:                                 # the registers
+            ids += [m.vocab + 2 + j for j in range(m.n_reg)]
+            pos += [L + 1 + j for j in range(m.n_reg)]
+        types += [3] * m.n_tail
+        labels += [k] * m.n_tail
     as32 = lambda a: np.asarray(a, dtype=np.int32)
     return as32(ids), as32(pos), as32(types), as32(labels), as32(logit_rows)
 
@@ -356,7 +362,7 @@ def run_training_form(args, wl):
     ids, pos, types, labels, lrows = trajectory_rows(wl, plan, prompt, 0)
     n = len(ids)
     cfg = smdm.make_config(m.n_layers, m.d_model, m.n_heads, m.d_head, m.d_ffn, m.vocab,
-                           n_reg=m.n_reg,
+                           n_reg=smdm.SMDM_REG_LEN if m.len_token else m.n_reg,
                            dtype=smdm.SMDM_BF16 if m.dtype == synth.BF16 else smdm.SMDM_F32,
                            rope_theta=m.rope_theta, rms_eps=m.rms_eps, max_batch=1,
                            max_len=wl.prompt_len + wl.gen_len, max_step_rows=1, max_rows=n)
@@ -407,11 +413,14 @@ def main():
     args = parse()
     wl = synth.WORKLOADS[args.workload]
     if args.n_reg is not None and args.n_reg != wl.model.n_reg:
-        if args.n_reg < 1:
-            raise SystemExit("--n-reg must be >= 1")
+        if args.n_reg < 0:
+            raise SystemExit("--n-reg must be >= 0")
         import dataclasses
-        wl = dataclasses.replace(wl, name=f"{wl.name}-reg{args.n_reg}",
-                                 model=dataclasses.replace(wl.model, n_reg=args.n_reg))
+        # 0: the length-token variant (one [LEN] row instead of registers)
+        wl = dataclasses.replace(wl, name=f"{wl.name}-reg{args.n_reg}" if args.n_reg else
+                                 f"{wl.name}-len",
+                                 model=dataclasses.replace(wl.model, n_reg=args.n_reg,
+                                                           len_token=args.n_reg == 0))
     if args.impl == "reference":
         return run_reference(args, wl)
 
@@ -442,7 +451,7 @@ def main():
     prompts_np = np.stack([synth.make_prompt(wl, i) for i in seq_ids])
     msr, max_rows = capacities(wl, plans)
     cfg = smdm.make_config(m.n_layers, m.d_model, m.n_heads, m.d_head, m.d_ffn, m.vocab,
-                           n_reg=m.n_reg,
+                           n_reg=smdm.SMDM_REG_LEN if m.len_token else m.n_reg,
                            dtype=smdm.SMDM_BF16 if m.dtype == synth.BF16 else smdm.SMDM_F32,
                            rope_theta=m.rope_theta, rms_eps=m.rms_eps, max_batch=B,
                            max_len=wl.prompt_len + wl.gen_len, max_step_rows=msr,

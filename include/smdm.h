@@ -24,7 +24,7 @@
  *  - Positions are 1-based: prompt 1..P, generated tokens P+1..P+Lgen, registers
  *    L+1..L+n_reg with L = P + Lgen.
  *  - Token ids: content ids 0..vocab-1, [MASK] = vocab, [LEN] = vocab+1, register j =
- *    vocab+2+j.  The embedding table has vocab+2+n_reg rows; the LM head covers content ids
+ *    vocab+2+j.  The embedding table has vocab+2+max(n_reg, 0) rows; the LM head covers content ids
  *    only.  A grid (the generated part of a sequence) is int32 [Lgen], -1 = still masked.
  *  - Weight layout: every linear weight is [out_features][in_features], input features
  *    contiguous; dtype per smdm_config.dtype (float32 or bfloat16).
@@ -60,6 +60,11 @@ enum { SMDM_MODE_SPARSE = 0, SMDM_MODE_DENSE = 1 };
 enum { SMDM_TYPE_PROMPT = 0, SMDM_TYPE_CLEAN = 1, SMDM_TYPE_MASK = 2, SMDM_TYPE_REG = 3 };
 enum { SMDM_PLAN_ORDER = 0, SMDM_PLAN_SEMIAR = 1 };
 #define SMDM_MAX_BATCH 8
+/* smdm_config.n_reg value of the length-token variant: no registers, and a single [LEN] row
+ * (id vocab+1, position L+1, the registers' attention rule) closes every step's rows.  It is
+ * the 0-register setting of the register-count ablation (papernotes' Table 7), read with
+ * "Key design 2" (one length token standing for the truncated masks). */
+#define SMDM_REG_LEN (-1)
 
 /* Model and capacity.  The pages do not describe the base network; the library implements a
  * pre-RMSNorm transformer (multi-head attention with 1-D rotate-half RoPE on the original
@@ -70,13 +75,14 @@ enum { SMDM_PLAN_ORDER = 0, SMDM_PLAN_SEMIAR = 1 };
 typedef struct {
   int n_layers, d_model, n_heads, d_head, d_ffn;
   int vocab;         /* content vocabulary V */
-  int n_reg;         /* register tokens per step (64 in the method) */
+  int n_reg;         /* register tokens per step (64 in the method; >= 0), or SMDM_REG_LEN */
   int dtype;         /* SMDM_F32 or SMDM_BF16 (weights and activations) */
   float rope_theta;  /* e.g. 10000 */
   float rms_eps;     /* e.g. 1e-6 */
   int max_batch;     /* sequences held at once, <= SMDM_MAX_BATCH */
   int max_len;       /* max P + Lgen of one sequence */
-  int max_step_rows; /* max rows of one sequence in one sampling step: n_new + n_query + n_reg */
+  int max_step_rows; /* max rows of one sequence in one sampling step: n_new + n_query + n_reg
+                        (+ 1 for the [LEN] row of the length-token variant) */
   int max_rows;      /* max rows of any single forward: a batched step (sum over sequences),
                         a prefill (P), a dense step (P + Lgen, per sequence) or a
                         training-form forward (n) */
@@ -85,7 +91,7 @@ typedef struct {
 /* Device pointers to the weights (borrowed).  Per-layer fields are HOST arrays of n_layers
  * device pointers; the library copies the pointer arrays at create. */
 typedef struct {
-  const void* emb;        /* [vocab + 2 + n_reg][d] */
+  const void* emb;        /* [vocab + 2 + max(n_reg, 0)][d] */
   const void* final_norm; /* [d] */
   const void* lm_head;    /* [vocab][d] */
   const void* const* attn_norm; /* [d] */

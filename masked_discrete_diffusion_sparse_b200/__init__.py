@@ -25,6 +25,7 @@ SMDM_MODE_SPARSE, SMDM_MODE_DENSE = 0, 1
 SMDM_TYPE_PROMPT, SMDM_TYPE_CLEAN, SMDM_TYPE_MASK, SMDM_TYPE_REG = range(4)
 SMDM_PLAN_ORDER, SMDM_PLAN_SEMIAR = 0, 1
 SMDM_MAX_BATCH = 8
+SMDM_REG_LEN = -1      # n_reg of the length-token variant (one [LEN] row, no registers)
 
 STATUS_NAMES = {0: "SMDM_OK", 1: "SMDM_EINVAL", 2: "SMDM_ESHAPE", 3: "SMDM_ENOMEM",
                 4: "SMDM_ECUDA", 5: "SMDM_ESTATE", 6: "SMDM_ETIMEOUT", 7: "SMDM_EDEVICE"}

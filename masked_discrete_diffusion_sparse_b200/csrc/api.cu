@@ -151,6 +151,12 @@ struct Layout {
   size_t partial_bytes;
 };
 
+// Rows that close every sampling step: n_reg registers, or with n_reg == SMDM_REG_LEN a single
+// [LEN] row (the length-token variant, no registers).
+int tail_rows(const smdm_config* c) { return c->n_reg == SMDM_REG_LEN ? 1 : c->n_reg; }
+// Embedding rows: content ids, [MASK], [LEN] and the registers.
+int emb_rows(const smdm_config* c) { return c->vocab + 2 + std::max(c->n_reg, 0); }
+
 bool config_ok(const smdm_config* c, std::string* why) {
   auto fail = [&](const char* s) {
     if (why) *why = s;
@@ -158,7 +164,7 @@ bool config_ok(const smdm_config* c, std::string* why) {
   };
   if (!c) return fail("null config");
   if (c->n_layers < 1 || c->d_model < 1 || c->n_heads < 1 || c->d_head < 1 || c->d_ffn < 1 ||
-      c->vocab < 1 || c->n_reg < 0)
+      c->vocab < 1 || c->n_reg < SMDM_REG_LEN)
     return fail("non-positive model dimension");
   if (c->n_heads * c->d_head != c->d_model) return fail("n_heads * d_head != d_model");
   if (c->d_head % 2) return fail("d_head must be even (rotary pairs)");
@@ -166,7 +172,7 @@ bool config_ok(const smdm_config* c, std::string* why) {
   if (c->max_batch < 1 || c->max_batch > SMDM_MAX_BATCH) return fail("max_batch out of range");
   if (c->max_len < 1 || c->max_step_rows < 1 || c->max_rows < 1) return fail("bad capacity");
   // positions, cache slots and row indices are 32-bit on the device
-  if ((long long)c->max_len + c->max_step_rows + c->n_reg + 8 > (1LL << 30) ||
+  if ((long long)c->max_len + c->max_step_rows + tail_rows(c) + 8 > (1LL << 30) ||
       c->max_rows > (1 << 24) || c->n_reg > (1 << 16))
     return fail("capacity too large");
   if (c->dtype == SMDM_BF16) {
@@ -193,7 +199,7 @@ Layout make_layout(const smdm_config* c, int n_sms) {
   const size_t es = c->dtype == SMDM_BF16 ? 2 : 4;
   const size_t d = c->d_model, H = c->n_heads, dh = c->d_head;
   L.cap = (int)align_up((size_t)c->max_len + c->max_step_rows, 8);
-  L.max_pos = c->max_len + c->n_reg + 2;
+  L.max_pos = c->max_len + tail_rows(c) + 2;
   L.n_vt = (c->vocab + 127) / 128;
   L.n_sms = n_sms;
   const size_t MR = align_up((size_t)c->max_rows, 256);
@@ -614,7 +620,7 @@ smdm_status check_desc(smdm_handle* h, const smdm_step_desc& d, bool dense) {
   }
   if (d.n_query > q.Lg) return fail(h, SMDM_EINVAL, "n_query larger than Lgen");
   if (!dense) {
-    const int R = q.n_new + d.n_query + h->cfg.n_reg;
+    const int R = q.n_new + d.n_query + tail_rows(&h->cfg);
     if (R > h->cfg.max_step_rows)
       return fail(h, SMDM_ESHAPE, "step rows %d exceed max_step_rows %d", R, h->cfg.max_step_rows);
     if (q.ctx + R > h->L.cap) return fail(h, SMDM_ESHAPE, "KV cache capacity exceeded");
@@ -786,7 +792,7 @@ static smdm_status prefill_block0(smdm_handle* h, int seq, const int32_t* d_prom
     a.P = P;
     a.Lg = Lgen;
     a.vocab = h->cfg.vocab;
-    a.emb_rows = h->cfg.vocab + 2 + h->cfg.n_reg;
+    a.emb_rows = emb_rows(&h->cfg);
     a.max_pos = h->L.max_pos;
     a.prompt = h->prompt(seq);
     a.given_pos = d_given_pos;
@@ -829,13 +835,14 @@ smdm_status smdm_step(smdm_handle* h, int n_seq, const smdm_step_desc* hd, float
     if ((s = check_desc(h, hd[i], false))) return s;
     for (int j = 0; j < i; ++j)
       if (hd[j].seq == hd[i].seq) return fail(h, SMDM_EINVAL, "sequence %d twice in a batch", hd[i].seq);
-    R += h->seq[hd[i].seq].n_new + hd[i].n_query + h->cfg.n_reg;
+    R += h->seq[hd[i].seq].n_new + hd[i].n_query + tail_rows(&h->cfg);
     NQ += hd[i].n_query;
   }
   if (R > h->cfg.max_rows) return fail(h, SMDM_ESHAPE, "batched rows %d exceed max_rows", R);
   PackArgs pa{};
   pa.n_seq = n_seq;
   pa.vocab = h->cfg.vocab;
+  pa.len_token = h->cfg.n_reg == SMDM_REG_LEN;
   pa.rows = h->rows;
   pa.status = h->status();
   FwdSpec f{};
@@ -850,13 +857,13 @@ smdm_status smdm_step(smdm_handle* h, int n_seq, const smdm_step_desc* hd, float
   for (int i = 0; i < n_seq; ++i) {
     const smdm_step_desc& d = hd[i];
     SeqState& q = h->seq[d.seq];
-    const int Rs = q.n_new + d.n_query + h->cfg.n_reg;
+    const int Rs = q.n_new + d.n_query + tail_rows(&h->cfg);
     PackSeq& p = pa.s[i];
     p.seq = d.seq;
     p.row0 = row0;
     p.n_new = q.n_new;
     p.n_q = d.n_query;
-    p.n_reg = h->cfg.n_reg;
+    p.n_reg = tail_rows(&h->cfg);
     p.ctx = q.ctx;
     p.P = q.P;
     p.Lg = q.Lg;
@@ -942,7 +949,7 @@ smdm_status smdm_dense_step(smdm_handle* h, const smdm_step_desc* d, float* d_lo
   a.seq = d->seq;
   a.P = q.P;
   a.vocab = h->cfg.vocab;
-  a.emb_rows = h->cfg.vocab + 2 + h->cfg.n_reg;
+  a.emb_rows = emb_rows(&h->cfg);
   a.max_pos = h->L.max_pos;
   a.prompt = h->prompt(d->seq);
   a.grid = q.grid;
@@ -1036,7 +1043,7 @@ smdm_status smdm_generate(smdm_handle* h, int batch, const int32_t* d_prompts, i
         n_new = k ? p.commit : 0;
         n_q = p.block - (long long)(k % p.steps_per_block) * p.commit;
       }
-      const long long rows = n_new + n_q + h->cfg.n_reg;
+      const long long rows = n_new + n_q + tail_rows(&h->cfg);
       if (mode == SMDM_MODE_SPARSE && rows > h->cfg.max_step_rows)
         return fail(h, SMDM_ESHAPE, "plan %d step %d needs %lld rows, max_step_rows is %d", b,
                     k + 1, rows, h->cfg.max_step_rows);
@@ -1101,7 +1108,7 @@ smdm_status smdm_forward_stepcausal(smdm_handle* h, const int32_t* d_ids, const 
   a.n = n;
   a.seq = 0;
   a.vocab = h->cfg.vocab;
-  a.emb_rows = h->cfg.vocab + 2 + h->cfg.n_reg;
+  a.emb_rows = emb_rows(&h->cfg);
   a.max_pos = h->L.max_pos;
   a.ids = d_ids;
   a.pos = d_pos;

@@ -14,7 +14,8 @@ namespace smdm {
 // pack: one CTA per sequence of a sampling step.  Rows of sequence s, in order:
 //   new cache  (tokens decoded at step k-1; id from the grid; CLEAN, label k-1),
 //   queries    (the decode set C_k; id [MASK]; MASK, label k),
-//   registers  (ids V+2+j, positions L+1+j; REG, label k).
+//   registers  (ids V+2+j, positions L+1+j; REG, label k), or in the length-token variant one
+//              [LEN] row (id V+1, position L+1; REG, label k).
 // kvlen: new-cache rows see the cache plus the new-cache rows; query and register rows see
 // every row of the step.  slot: K/V of row i go to cache slot ctx + i.
 // ------------------------------------------------------------------------------------------
@@ -88,7 +89,7 @@ __global__ void pack_step_kernel(PackArgs a) {
     } else {
       const int j = i - s.n_new - s.n_q;
       pos = L + 1 + j;
-      id = a.vocab + 2 + j;
+      id = a.vocab + 2 + j - a.len_token;
       type = kTypeReg;
       label = s.label;
       kvlen = s.ctx + R;

@@ -22,6 +22,7 @@ struct PackArgs {
   int n_seq;
   PackSeq s[kMaxBatch];
   int vocab;
+  int len_token;    // 1: the one tail row is [LEN] (id vocab+1) instead of REG_0 (vocab+2)
   Rows rows;
   uint32_t* status;
 };

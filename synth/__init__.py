@@ -63,6 +63,11 @@ class ModelShape:
         return self.vocab + 2 + self.n_reg
 
     @property
+    def n_tail(self) -> int:
+        """Rows that close each sampling step: the registers, or the one [LEN] row."""
+        return 1 if self.len_token else self.n_reg
+
+    @property
     def mask_id(self) -> int:
         return self.vocab
 

@@ -33,8 +33,8 @@ def upload_weights(w: synth.Weights, device="cuda") -> dict:
 def step_rows_bound(wl: synth.Workload, plan: synth.Plan) -> int:
     if plan.kind == "order":
         n = list(plan.n_per_step)
-        return max((n[i - 1] if i else 0) + n[i] for i in range(len(n))) + wl.model.n_reg
-    return plan.commit + plan.block + wl.model.n_reg
+        return max((n[i - 1] if i else 0) + n[i] for i in range(len(n))) + wl.model.n_tail
+    return plan.commit + plan.block + wl.model.n_tail
 
 
 def config_for(wl: synth.Workload, batch: int = 1, train_rows: int = 0,
@@ -45,7 +45,7 @@ def config_for(wl: synth.Workload, batch: int = 1, train_rows: int = 0,
     L = wl.prompt_len + wl.gen_len
     max_rows = max(batch * msr, L, train_rows, 1)
     return smdm.make_config(m.n_layers, m.d_model, m.n_heads, m.d_head, m.d_ffn, m.vocab,
-                            n_reg=m.n_reg,
+                            n_reg=smdm.SMDM_REG_LEN if m.len_token else m.n_reg,
                             dtype=smdm.SMDM_BF16 if m.dtype == synth.BF16 else smdm.SMDM_F32,
                             rope_theta=m.rope_theta, rms_eps=m.rms_eps, max_batch=batch,
                             max_len=L, max_step_rows=msr, max_rows=max_rows)

@@ -56,6 +56,11 @@ def test_config_rules_for_bf16_models():
                   (2, 256, 2, 128, 704, 1002)]:  # vocab % 4
         bad = smdm.make_config(*shape, **ok)
         assert lib.smdm_workspace_bytes(ctypes.byref(bad)) == 0, shape
+    # the length-token variant (n_reg = SMDM_REG_LEN) is a valid config; below it is not
+    len_cfg = smdm.make_config(2, 256, 2, 128, 704, 1000, n_reg=smdm.SMDM_REG_LEN, **ok)
+    assert lib.smdm_workspace_bytes(ctypes.byref(len_cfg)) > 0
+    below = smdm.make_config(2, 256, 2, 128, 704, 1000, n_reg=-2, **ok)
+    assert lib.smdm_workspace_bytes(ctypes.byref(below)) == 0
     # the fp32 path has none of the tile rules
     f32 = smdm.make_config(2, 128, 2, 64, 320, 301, dtype=smdm.SMDM_F32, max_batch=1,
                            max_len=100, max_step_rows=100, max_rows=100)

@@ -51,7 +51,7 @@ def test_step_shapes_cover_every_generated_token():
         assert len(shapes) == wl.n_steps
         assert sum(q for (_, q, _, _) in shapes) == wl.gen_len
         for (R, q, ctx, n_new) in shapes:
-            assert R == n_new + q + wl.model.n_reg
+            assert R == n_new + q + wl.model.n_tail
 
 
 def test_streamed_parameters_per_step():
@@ -101,3 +101,27 @@ def test_step_shapes_and_attention_work_match_the_oracle_run():
                                     np.concatenate([cl, pk.labels]))
             kv_sum = n_new * (ctx + n_new) + (R - n_new) * (ctx + R)
             assert kv_sum == int(vis.sum()), (name, r.k)
+
+
+def test_length_token_variant_rows_in_the_bench():
+    """bench --n-reg 0 (the length-token variant): one [LEN] tail row per step, in the step
+    shapes and in the training-form rows, equal to the oracle's trajectory of the same plan."""
+    import dataclasses
+    b = _bench()
+    base = synth.WORKLOADS["tiny-f32-cos"]
+    wl = dataclasses.replace(base, model=dataclasses.replace(base.model, n_reg=0, len_token=True))
+    plan = synth.make_plan(wl, 0)
+    for (R, q, ctx, n_new) in b.step_shapes(wl, plan):
+        assert R == n_new + q + 1
+    prompt = synth.make_prompt(wl, 0)
+    ids, pos, types, labels, lrows = b.trajectory_rows(wl, plan, prompt, 0)
+    om = oracle.Model(synth.make_weights(wl.model, wl.seed))
+    st, recs = oracle.generate(om, prompt, wl.gen_len, plan)
+    o_ids, o_pos, o_types, o_labels, _ = oracle.trajectory(prompt, wl.model, wl.gen_len, recs)
+    tail = types == 3
+    assert (ids[tail] == wl.model.vocab + 1).all() and (pos[tail] == wl.prompt_len +
+                                                         wl.gen_len + 1).all()
+    mine = sorted(zip(pos.tolist(), types.tolist(), labels.tolist()))
+    ref = sorted(zip(o_pos.tolist(), o_types.tolist(), o_labels.tolist()))
+    assert mine == ref
+    assert sorted(ids[tail].tolist()) == sorted(o_ids[o_types == 3].tolist())
