@@ -168,6 +168,29 @@ typedef struct {
 smdm_status smdm_step(smdm_handle* h, int n_seq, const smdm_step_desc* h_desc, float* d_logits,
                       int32_t* d_tok, float* d_conf, cudaStream_t stream);
 
+/* Speed switches of the paper notes' Table 6 ablation (cache the prompt, cache decoded
+ * responses, truncate the masked responses); SMDM_SW_ALL is the method's own step. */
+enum { SMDM_SW_CACHE_PROMPT = 1, SMDM_SW_CACHE_RES = 2, SMDM_SW_TRUNCATE = 4, SMDM_SW_ALL = 7 };
+
+/* One sampling step of one sequence with some of the method's speed switches off.  Off states
+ * (the pages name the switches but do not define them; reading): without CACHE_PROMPT the
+ * prompt rows (label 0) are computed again every step; without CACHE_RES every decoded token
+ * is computed again every step (its label = the step it was decoded at) instead of staying in
+ * the cache; without TRUNCATE every other still-masked position joins the step as a [MASK] row
+ * of label k (the decode set sees it, so its logits change).  Logits, tokens and the commit are
+ * for the decode set only, as in smdm_step.
+ * Rows: [prompt?][decoded tokens][decode set][other masks?][registers], each row seeing a key
+ * prefix of the sequence's cache, which holds the prompt at slots [0, P) and decoded tokens in
+ * decode order after it.  The step needs max_step_rows and max_rows >= P (prompt not cached)
+ * + decoded tokens (responses not cached; else the previous step's commits) + n_query + the
+ * other masks (not truncated) + registers.
+ * The sequence must come from smdm_prefill (no given tokens), take explicit query positions,
+ * and keep one value of `switches` for its whole run; smdm_step and smdm_dense_step refuse a
+ * sequence that ran switched steps (SMDM_ESTATE). */
+smdm_status smdm_step_switched(smdm_handle* h, const smdm_step_desc* h_desc, int switches,
+                               float* d_logits, int32_t* d_tok, float* d_conf,
+                               cudaStream_t stream);
+
 /* The dense comparator (the standard MDM step the pages argue against, papernotes
  * "Key design 1"): all P+Lgen rows of sequence `seq`, [MASK] ids at undecoded positions, no
  * registers, no cache, full bidirectional attention, logits for every generated position

@@ -26,12 +26,14 @@ SMDM_TYPE_PROMPT, SMDM_TYPE_CLEAN, SMDM_TYPE_MASK, SMDM_TYPE_REG = range(4)
 SMDM_PLAN_ORDER, SMDM_PLAN_SEMIAR = 0, 1
 SMDM_MAX_BATCH = 8
 SMDM_REG_LEN = -1      # n_reg of the length-token variant (one [LEN] row, no registers)
+SMDM_SW_CACHE_PROMPT, SMDM_SW_CACHE_RES, SMDM_SW_TRUNCATE, SMDM_SW_ALL = 1, 2, 4, 7
 
 STATUS_NAMES = {0: "SMDM_OK", 1: "SMDM_EINVAL", 2: "SMDM_ESHAPE", 3: "SMDM_ENOMEM",
                 4: "SMDM_ECUDA", 5: "SMDM_ESTATE", 6: "SMDM_ETIMEOUT", 7: "SMDM_EDEVICE"}
 
 EXPORTED = ["smdm_workspace_bytes", "smdm_create", "smdm_destroy", "smdm_last_error",
-            "smdm_prefill", "smdm_prefill_given", "smdm_step", "smdm_dense_step", "smdm_generate",
+            "smdm_prefill", "smdm_prefill_given", "smdm_step", "smdm_step_switched",
+            "smdm_dense_step", "smdm_generate",
             "smdm_forward_stepcausal", "smdm_debug_mask", "smdm_debug_rows",
             "smdm_context_length", "smdm_device_status", "smdm_profile_begin",
             "smdm_profile_end", "smdm_forward_stepcausal_noalloc"]
@@ -110,6 +112,8 @@ def lib() -> ctypes.CDLL:
     L.smdm_prefill_given.restype = st
     L.smdm_step.argtypes = [vp, i32, ctypes.POINTER(smdm_step_desc), vp, vp, vp, vp]
     L.smdm_step.restype = st
+    L.smdm_step_switched.argtypes = [vp, ctypes.POINTER(smdm_step_desc), i32, vp, vp, vp, vp]
+    L.smdm_step_switched.restype = st
     L.smdm_dense_step.argtypes = [vp, ctypes.POINTER(smdm_step_desc), vp, vp, vp, vp]
     L.smdm_dense_step.restype = st
     L.smdm_generate.argtypes = [vp, i32, vp, i32, i32, ctypes.POINTER(smdm_plan), i32, vp, vp]
@@ -241,6 +245,16 @@ class Model:
                                     d.get("policy", SMDM_POLICY_ALL), d.get("n_commit", 0))
         self._check(lib().smdm_step(self.h, len(descs), arr, _ptr(logits), _ptr(tok), _ptr(conf),
                                     _stream(stream)))
+
+    def smdm_step_switched(self, desc: dict, switches: int, logits=None, tok=None, conf=None,
+                           stream=None):
+        """One step of one sequence with the Table-6 speed switches (SMDM_SW_* bits); desc as
+        in smdm_step, with query_pos required."""
+        qp = desc["query_pos"]
+        d = smdm_step_desc(desc["seq"], _ptr(_i32(qp)), desc["n_query"], 0, 0,
+                           desc.get("policy", SMDM_POLICY_ALL), desc.get("n_commit", 0))
+        self._check(lib().smdm_step_switched(self.h, ctypes.byref(d), switches, _ptr(logits),
+                                             _ptr(tok), _ptr(conf), _stream(stream)))
 
     def smdm_dense_step(self, desc: dict, logits=None, tok=None, conf=None, stream=None):
         qp = desc.get("query_pos")

@@ -145,7 +145,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
   size_t kc, vc, kscr, vscr, x, h, q, ao, act, hq, pmax, psum, parg, rows, rope, partial,
-      counters, status, newpos, prompts, aux, attn_part, total;
+      counters, status, newpos, prompts, aux, attn_part, sw, total;
   size_t attn_part_bytes;
   int cap, max_pos, n_vt, rt_max, max_tiles, n_sms;
   size_t partial_bytes;
@@ -242,6 +242,8 @@ Layout make_layout(const smdm_config* c, int n_sms) {
   const size_t step_rows = std::min((size_t)c->max_rows, (size_t)c->max_batch * c->max_step_rows);
   L.attn_part_bytes = 16 * step_rows * ((size_t)d * 4 + H * 8);
   L.attn_part = take(L.attn_part_bytes);
+  // switched steps: per sequence, decoded positions, their steps and the query marks
+  L.sw = take((size_t)c->max_batch * 3 * c->max_len * 4);
   L.total = off + 1024;
   return L;
 }
@@ -250,9 +252,12 @@ struct SeqState {
   bool active = false;
   bool dense = false;
   int P = 0, Lg = 0;
+  int n0 = 0;      // block-0 rows (prompt and given tokens)
   int ctx = 0;     // KV cache length (prompt + cached clean tokens)
   int n_new = 0;   // tokens committed at the previous step
   int k = 0;       // steps taken
+  int sw = -1;     // switches of smdm_step_switched (fixed at its first step), -1 = not used
+  int dec = 0;     // switched steps: tokens decoded before the previous step
   int32_t* grid = nullptr;
 };
 
@@ -289,6 +294,7 @@ struct smdm_handle {
   uint32_t* status() { return at<uint32_t>(L.status); }
   int* newpos(int s) { return at<int>(L.newpos) + (size_t)s * cfg.max_step_rows; }
   int* prompt(int s) { return at<int>(L.prompts) + (size_t)s * cfg.max_len; }
+  int* sw_arrays(int s) { return at<int>(L.sw) + (size_t)s * 3 * cfg.max_len; }
   size_t es() const { return bf16 ? 2 : 4; }
 };
 
@@ -605,6 +611,8 @@ smdm_status check_desc(smdm_handle* h, const smdm_step_desc& d, bool dense) {
   if (!q.active) return fail(h, SMDM_ESTATE, "sequence %d has not been prefilled", d.seq);
   if (q.dense != dense)
     return fail(h, SMDM_ESTATE, "sequence %d mixes sparse and dense steps", d.seq);
+  if (q.sw >= 0)
+    return fail(h, SMDM_ESTATE, "sequence %d runs switched steps (smdm_step_switched)", d.seq);
   if (d.n_query < 1) return fail(h, SMDM_EINVAL, "empty decode set");
   if (d.policy != SMDM_POLICY_ALL && d.policy != SMDM_POLICY_TOPN)
     return fail(h, SMDM_EINVAL, "unknown policy %d", d.policy);
@@ -809,6 +817,7 @@ static smdm_status prefill_block0(smdm_handle* h, int seq, const int32_t* d_prom
     if ((s = forward(h, f, st))) return s;
   }
   q.active = true;
+  q.n0 = n0;
   q.ctx = n0;
   return SMDM_OK;
 }
@@ -907,6 +916,110 @@ smdm_status smdm_step(smdm_handle* h, int n_seq, const smdm_step_desc* hd, float
     q.n_new = committed(hd[i]);
     q.k += 1;
   }
+  return SMDM_OK;
+}
+
+smdm_status smdm_step_switched(smdm_handle* h, const smdm_step_desc* hd, int switches,
+                               float* d_logits, int32_t* d_tok, float* d_conf, cudaStream_t st) {
+  if (!h) return SMDM_EINVAL;
+  if (!hd) return fail(h, SMDM_EINVAL, "null step descriptor");
+  if (switches < 0 || switches > SMDM_SW_ALL) return fail(h, SMDM_EINVAL, "bad switches %d", switches);
+  const smdm_step_desc& d = *hd;
+  smdm_status s;
+  if ((s = check_seq(h, d.seq))) return s;
+  SeqState& q = h->seq[d.seq];
+  if (!q.active) return fail(h, SMDM_ESTATE, "sequence %d has not been prefilled", d.seq);
+  if (q.dense) return fail(h, SMDM_ESTATE, "sequence %d runs dense steps", d.seq);
+  if (q.sw != switches && (q.k > 0 || q.sw >= 0))
+    return fail(h, SMDM_ESTATE, "sequence %d keeps one set of switches for its whole run", d.seq);
+  if (q.n0 != q.P)
+    return fail(h, SMDM_EINVAL, "switched steps need a prompt-only prefill (no given tokens)");
+  if (!d.d_query_pos) return fail(h, SMDM_EINVAL, "switched steps take explicit query positions");
+  if (d.policy != SMDM_POLICY_ALL && d.policy != SMDM_POLICY_TOPN)
+    return fail(h, SMDM_EINVAL, "unknown policy %d", d.policy);
+  if (d.policy == SMDM_POLICY_TOPN && d.n_commit < 1)
+    return fail(h, SMDM_EINVAL, "TOPN needs n_commit >= 1");
+  const int masked = q.Lg - q.dec - q.n_new;   // still masked before this step commits
+  if (d.n_query < 1 || d.n_query > masked)
+    return fail(h, SMDM_EINVAL, "n_query %d outside [1, %d masked positions]", d.n_query, masked);
+  const bool cp = switches & SMDM_SW_CACHE_PROMPT, cr = switches & SMDM_SW_CACHE_RES,
+             tr = switches & SMDM_SW_TRUNCATE;
+  const int n_tail = tail_rows(&h->cfg);
+  const int n_extra = tr ? 0 : masked - d.n_query;
+  const int n_dec = q.dec + q.n_new;
+  const int R = (cp ? 0 : q.P) + (cr ? q.n_new : n_dec) + d.n_query + n_extra + n_tail;
+  const int keys = q.P + n_dec + d.n_query + n_extra + n_tail;
+  if (R > h->cfg.max_step_rows || R > h->cfg.max_rows)
+    return fail(h, SMDM_ESHAPE, "switched step needs %d rows (max_step_rows %d, max_rows %d)", R,
+                h->cfg.max_step_rows, h->cfg.max_rows);
+  if (keys > h->L.cap) return fail(h, SMDM_ESHAPE, "KV cache capacity exceeded");
+  int* dec_pos = h->sw_arrays(d.seq);
+  int* dec_lab = dec_pos + h->cfg.max_len;
+  int* qmark = dec_lab + h->cfg.max_len;
+  if (q.sw < 0) {   // first switched step of the sequence: no position has been queried yet
+    Launch lg_(h, SMDM_K_OTHER, st);
+    CK(launch_fill_i32(qmark, q.Lg, 0, st));
+  }
+  PackSwArgs pa{};
+  pa.seq = d.seq;
+  pa.P = q.P;
+  pa.Lg = q.Lg;
+  pa.label = q.k + 1;
+  pa.vocab = h->cfg.vocab;
+  pa.n_tail = n_tail;
+  pa.len_token = h->cfg.n_reg == SMDM_REG_LEN;
+  pa.cache_prompt = cp;
+  pa.cache_res = cr;
+  pa.truncate = tr;
+  pa.n_new = q.n_new;
+  pa.dec_prev = q.dec;
+  pa.n_q = d.n_query;
+  pa.n_extra = n_extra;
+  pa.qpos = d.d_query_pos;
+  pa.newpos = h->newpos(d.seq);
+  pa.prompt = h->prompt(d.seq);
+  pa.grid = q.grid;
+  pa.dec_pos = dec_pos;
+  pa.dec_lab = dec_lab;
+  pa.qmark = qmark;
+  pa.rows = h->rows;
+  pa.status = h->status();
+  { Launch lg_(h, SMDM_K_PACK, st); CK(launch_pack_switched(pa, st)); }
+  FwdSpec f{};
+  f.R = R;
+  f.attn_mode = 0;
+  f.n_seg = 1;
+  f.seg[0] = AttnSeg{d.seq, 0, R, keys, 0};
+  f.n_logit = d.n_query;
+  f.logits = d_logits;
+  if ((s = forward(h, f, st))) return s;
+  UnmaskArgs ua{};
+  ua.n_seq = 1;
+  UnmaskSeq& u = ua.s[0];
+  u.qbase = 0;
+  u.n_q = d.n_query;
+  u.lbase = 0;
+  u.dense = 0;
+  u.policy = d.policy;
+  u.n_commit = d.policy == SMDM_POLICY_ALL ? d.n_query : d.n_commit;
+  u.P = q.P;
+  u.Lg = q.Lg;
+  u.grid = q.grid;
+  u.newpos = h->newpos(d.seq);
+  ua.n_vt = h->L.n_vt;
+  ua.pmax = h->at<float>(h->L.pmax);
+  ua.psum = h->at<float>(h->L.psum);
+  ua.parg = h->at<int>(h->L.parg);
+  ua.qpos_of = h->rows.qpos;
+  ua.tok_out = d_tok;
+  ua.conf_out = d_conf;
+  ua.status = h->status();
+  { Launch lg_(h, SMDM_K_UNMASK, st); CK(launch_unmask(ua, d.n_query, st)); }
+  q.sw = switches;
+  if (cr) q.ctx += q.n_new;    // decoded tokens stay in the cache only when it is on
+  q.dec += q.n_new;
+  q.n_new = committed(d);
+  q.k += 1;
   return SMDM_OK;
 }
 

@@ -111,6 +111,111 @@ __global__ void pack_step_kernel(PackArgs a) {
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// pack_switched: one CTA for one sequence (see PackSwArgs).  Slots and key prefixes:
+//   prompt rows          slot i (rewrites the prompt's K/V), keys [0, P)
+//   decoded rows, cached  the new-cache rows at slot P + dec_prev + i, keys [0, P + dec_prev + n_new)
+//   decoded rows, not cached  every decoded token j at slot P + j, keys [0, P + (first j' whose
+//                        step is later than j's))
+//   C, other masks, tail rows  slots from base = P + dec_prev + n_new on, keys: all of them.
+// ------------------------------------------------------------------------------------------
+__global__ void pack_switched_kernel(PackSwArgs a) {
+  griddep_launch();
+  griddep_wait();   // launched with programmatic dependent launch
+  __shared__ int warp_counts[32];
+  __shared__ int found;
+  const int tid = threadIdx.x, nth = blockDim.x;
+  const int P = a.P, L = a.P + a.Lg, k = a.label;
+  const int n_dec = a.dec_prev + a.n_new;
+  const int n_p = a.cache_prompt ? 0 : P;
+  const int n_d = a.cache_res ? a.n_new : n_dec;
+  const int r_c = n_p + n_d, r_e = r_c + a.n_q, r_t = r_e + a.n_extra;
+  const int base = P + n_dec;
+  const int all_keys = base + a.n_q + a.n_extra + a.n_tail;
+  Rows rw = a.rows;
+  auto put = [&](int r, int id, int pos, int type, int label, int slot, int kvlen) {
+    rw.ids[r] = id;
+    rw.pos[r] = pos;
+    rw.type[r] = type;
+    rw.label[r] = label;
+    rw.seq[r] = a.seq;
+    rw.slot[r] = slot;
+    rw.kvlen[r] = kvlen;
+  };
+  auto token_at = [&](int pos) {
+    const bool ok = pos > P && pos <= L;
+    const int id = ok ? a.grid[pos - P - 1] : -1;
+    if (id < 0) {
+      atomicOr(a.status, kStatusBounds);
+      return 0;
+    }
+    return id;
+  };
+  // the tokens committed at step k-1 join the decoded list; the decode set is marked
+  for (int i = tid; i < a.n_new; i += nth) {
+    a.dec_pos[a.dec_prev + i] = a.newpos[i];
+    a.dec_lab[a.dec_prev + i] = k - 1;
+  }
+  for (int j = tid; j < a.n_q; j += nth) {
+    const int p = a.qpos[j];
+    if (p <= P || p > L || a.grid[p - P - 1] >= 0) {
+      atomicOr(a.status, kStatusBounds);
+    } else {
+      a.qmark[p - P - 1] = k;
+    }
+  }
+  if (tid == 0) found = 0;
+  __syncthreads();
+  for (int i = tid; i < n_p; i += nth) put(i, a.prompt[i], i + 1, kTypePrompt, 0, i, P);
+  if (a.cache_res) {
+    for (int i = tid; i < a.n_new; i += nth) {
+      const int pos = a.dec_pos[a.dec_prev + i];
+      put(n_p + i, token_at(pos), pos, kTypeClean, k - 1, P + a.dec_prev + i, base);
+    }
+  } else {
+    for (int j = tid; j < n_dec; j += nth) {
+      const int lab = a.dec_lab[j];
+      int lo = j + 1, hi = n_dec;          // first entry decoded after step `lab`
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (a.dec_lab[mid] <= lab) lo = mid + 1; else hi = mid;
+      }
+      const int pos = a.dec_pos[j];
+      put(n_p + j, token_at(pos), pos, kTypeClean, lab, P + j, P + lo);
+    }
+  }
+  for (int j = tid; j < a.n_q; j += nth) {
+    const int pos = a.qpos[j];
+    put(r_c + j, a.vocab, pos, kTypeMask, k, base + j, all_keys);
+    rw.qrow[j] = r_c + j;
+    rw.qpos[j] = pos;
+  }
+  for (int t = tid; t < a.n_tail; t += nth)
+    put(r_t + t, a.vocab + 2 + t - a.len_token, L + 1 + t, kTypeReg, k,
+        base + a.n_q + a.n_extra + t, all_keys);
+  if (!a.truncate) {
+    // every other still-masked position, in position order (block-wide stream compaction)
+    const int lane = tid & 31, w = tid >> 5, nw = nth >> 5;
+    for (int b0 = 0; b0 < a.Lg; b0 += nth) {
+      const int i = b0 + tid;
+      const bool extra = i < a.Lg && a.grid[i] < 0 && a.qmark[i] != k;
+      const unsigned ballot = __ballot_sync(0xffffffffu, extra);
+      if (lane == 0) warp_counts[w] = __popc(ballot);
+      __syncthreads();
+      int before = found;
+      for (int x = 0; x < w; ++x) before += warp_counts[x];
+      const int idx = before + __popc(ballot & ((1u << lane) - 1u));
+      if (extra && idx < a.n_extra)
+        put(r_e + idx, a.vocab, P + 1 + i, kTypeMask, k, base + a.n_q + idx, all_keys);
+      __syncthreads();
+      if (tid == 0)
+        for (int x = 0; x < nw; ++x) found += warp_counts[x];
+      __syncthreads();
+    }
+    if (tid == 0 && found != a.n_extra) atomicOr(a.status, kStatusBounds);
+  }
+}
+
 // Prefill / dense / training-form rows: one thread per row.
 __global__ void pack_linear_kernel(LinearPackArgs a) {
   griddep_launch();
@@ -362,6 +467,9 @@ cudaError_t launch_pack_step(const PackArgs& a, cudaStream_t st) {
 cudaError_t launch_pack_linear(const LinearPackArgs& a, cudaStream_t st) {
   if (a.n <= 0) return cudaSuccess;
   return launch_pdl(pack_linear_kernel, dim3((a.n + 255) / 256), dim3(256), 0, st, 1, a);
+}
+cudaError_t launch_pack_switched(const PackSwArgs& a, cudaStream_t st) {
+  return launch_pdl(pack_switched_kernel, dim3(1), dim3(512), 0, st, 1, a);
 }
 cudaError_t launch_gather_rows(const int* src, int n, int* qrow, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;

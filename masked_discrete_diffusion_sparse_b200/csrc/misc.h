@@ -29,6 +29,31 @@ struct PackArgs {
 
 enum { kPackPrefill = 0, kPackDense = 1, kPackTrain = 2, kPackPrefillGiven = 3 };
 
+// One sampling step of one sequence under the speed switches of the Table-6 ablation (cache the
+// prompt, cache decoded tokens, truncate the other masks).  Cache slots: the prompt at
+// [0, P), decoded tokens in decode order from P on, then this step's masks and tail rows.
+// Rows, in label order: recomputed prompt (!cache_prompt), decoded tokens (the new-cache rows,
+// or with !cache_res every decoded token), the decode set C, the other masks (!truncate), the
+// tail rows.  Every row sees a key prefix of that layout.
+struct PackSwArgs {
+  int seq, P, Lg;
+  int label;         // step number k
+  int vocab, n_tail, len_token;
+  int cache_prompt, cache_res, truncate;
+  int n_new;         // tokens committed at step k-1 (this step's new-cache rows)
+  int dec_prev;      // tokens decoded before step k-1
+  int n_q, n_extra;  // decode set; other still-masked positions (!truncate)
+  const int* qpos;   // [n_q] decode set positions
+  const int* newpos; // [n_new]
+  const int* prompt; // [P]
+  const int* grid;   // [Lg]
+  int* dec_pos;      // [Lg] decoded positions in decode order (appended here)
+  int* dec_lab;      // [Lg] the step each was decoded at
+  int* qmark;        // [Lg] the last step that queried the position (0 = never)
+  Rows rows;
+  uint32_t* status;
+};
+
 struct LinearPackArgs {
   int mode;
   int n;            // rows
@@ -85,6 +110,7 @@ struct UnmaskArgs {
 
 cudaError_t launch_pack_step(const PackArgs& a, cudaStream_t st);
 cudaError_t launch_pack_linear(const LinearPackArgs& a, cudaStream_t st);
+cudaError_t launch_pack_switched(const PackSwArgs& a, cudaStream_t st);
 cudaError_t launch_gather_rows(const int* src, int n, int* qrow, cudaStream_t st);
 template <typename T>
 cudaError_t launch_rmsnorm(const NormArgs& a, int rows, cudaStream_t st);

@@ -86,6 +86,7 @@ def test_argument_errors_return_before_any_device_work():
     assert lib.smdm_prefill(None, 0, None, 4, 8, None, None) == E
     assert lib.smdm_prefill_given(None, 0, None, 4, 8, None, None, 0, None, None) == E
     assert lib.smdm_step(None, 1, None, None, None, None, None) == E
+    assert lib.smdm_step_switched(None, None, 7, None, None, None, None) == E
     assert lib.smdm_dense_step(None, None, None, None, None, None) == E
     assert lib.smdm_generate(None, 1, None, 4, 8, None, 0, None, None) == E
     assert lib.smdm_forward_stepcausal(None, None, None, None, None, 1, None, 1, None, None) == E

@@ -1,5 +1,6 @@
 """GPU parity cases for device modes that have not yet run on a B200: the length-token variant
-(n_reg = SMDM_REG_LEN) and semi-AR plans with the blocks in a permuted order.  They carry the
+(n_reg = SMDM_REG_LEN), semi-AR plans with the blocks in a permuted order, and the Table-6
+speed switches (smdm_step_switched).  They carry the
 `gpu_pending` marker instead of `gpu`, so the regular GPU suite does not select them; run them
 with `pytest -m gpu_pending` on a B200, and move them to the `gpu` marker once green.  On a
 machine without CUDA they skip."""
@@ -85,3 +86,60 @@ def test_generate_with_block_order_equals_the_stepwise_run():
         assert np.array_equal(grids.cpu().numpy()[0], stepwise.cpu().numpy()[0])
     finally:
         r.close()
+
+
+@pytest.mark.parametrize("switches", [smdm.SMDM_SW_ALL,
+                                      smdm.SMDM_SW_ALL & ~smdm.SMDM_SW_CACHE_PROMPT,
+                                      smdm.SMDM_SW_ALL & ~smdm.SMDM_SW_CACHE_RES,
+                                      smdm.SMDM_SW_ALL & ~smdm.SMDM_SW_TRUNCATE, 0])
+def test_switched_steps_match_the_oracle(switches):
+    """smdm_step_switched against oracle.Switched, step by step (teacher-forced): the rows as a
+    set, the decode set's logits within tolerance, admissible tokens, the grid."""
+    from smdm_testlib import config_for, logit_err, token_admissible, upload_weights, TOL
+    import oracle
+    wl = synth.WORKLOADS["tiny-bf16-cos"]
+    P, Lg, V = wl.prompt_len, wl.gen_len, wl.model.vocab
+    cp = bool(switches & smdm.SMDM_SW_CACHE_PROMPT)
+    cr = bool(switches & smdm.SMDM_SW_CACHE_RES)
+    tr = bool(switches & smdm.SMDM_SW_TRUNCATE)
+    w = synth.make_weights(wl.model, wl.seed, gain_std=0.02)
+    om = oracle.Model(w)
+    plan = synth.make_plan(wl)
+    prompt = synth.make_prompt(wl)
+    cfg = config_for(wl)
+    cfg.max_step_rows = cfg.max_rows = P + Lg + wl.model.n_tail
+    model = smdm.Model(cfg, upload_weights(w))
+    tol = TOL[wl.model.dtype]
+    try:
+        grid = torch.empty(Lg, dtype=torch.int32, device="cuda")
+        model.smdm_prefill(0, i32(prompt), Lg, grid)
+        st = oracle.Switched(om, prompt, Lg, cache_prompt=cp, cache_res=cr, truncate=tr)
+        for k in range(1, plan.n_steps + 1):
+            qp = np.asarray(plan.query_positions(k), dtype=np.int64)
+            logits = torch.empty((len(qp), V), dtype=torch.float32, device="cuda")
+            tok = torch.empty(len(qp), dtype=torch.int32, device="cuda")
+            model.smdm_step_switched(dict(seq=0, query_pos=i32(qp), n_query=len(qp),
+                                          policy=smdm.SMDM_POLICY_ALL), switches,
+                                     logits=logits, tok=tok)
+            R = model.smdm_debug_rows()
+            ids = torch.empty(R, dtype=torch.int32, device="cuda")
+            pos, typ, lab = torch.empty_like(ids), torch.empty_like(ids), torch.empty_like(ids)
+            model.smdm_debug_rows(ids, pos, typ, lab)
+            torch.cuda.synchronize()
+            assert model.smdm_device_status() == 0
+            rows, _, _ = st.rows(qp)
+            got = sorted(zip(ids.cpu().tolist(), pos.cpu().tolist(), typ.cpu().tolist(),
+                             lab.cpu().tolist()))
+            ref_rows = sorted(zip(rows.ids.tolist(), rows.pos.tolist(), rows.types.tolist(),
+                                  rows.labels.tolist()))
+            assert got == ref_rows, f"step {k}: rows differ"
+            ref = st.step_logits(qp)
+            assert logit_err(logits.cpu().numpy().astype(np.float64), ref) <= tol, f"step {k}"
+            tk = tok.cpu().numpy()
+            assert token_admissible(tk, ref, tol).all(), f"step {k}"
+            g = grid.cpu().numpy()
+            assert (g[qp - P - 1] == tk).all()
+            st.commit(qp, tk)          # teacher forcing
+        assert np.array_equal(grid.cpu().numpy(), st.grid)
+    finally:
+        model.close()
