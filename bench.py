@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--form", default="sampling", choices=["sampling", "training"],
                     help="sampling: full sparse sampling runs (the headline); training: one "
                          "training-form forward over a whole step-labelled trajectory")
+    ap.add_argument("--switches", type=int, default=7, choices=range(8),
+                    help="Table-6 speed switches as bits (1 cache prompt, 2 cache decoded "
+                         "tokens, 4 truncate); 7 = the method (the default run)")
     ap.add_argument("--n-reg", type=int, default=None,
                     help="register rows per step (the method's 64 by default; 0 = the "
                          "length-token variant, one [LEN] row); for the register-count "
@@ -399,6 +402,74 @@ def run_training_form(args, wl):
     return 0
 
 
+def run_switched(args, wl):
+    """--switches S (bits 1 cache prompt, 2 cache decoded tokens, 4 truncate; 7 = the method):
+    one sequence's sampling run through smdm_step_switched, replayed as a CUDA graph (prefill
+    + every step).  One line per setting gives the speed side of the Table-6 ablation."""
+    import torch
+    import masked_discrete_diffusion_sparse_b200 as smdm
+    if wl.plan == "semiar" or wl.batch != 1:
+        raise SystemExit("--switches supports single-sequence order plans")
+    m = wl.model
+    P, Lg = wl.prompt_len, wl.gen_len
+    dev = torch.device("cuda", 0)
+    plan = synth.make_plan(wl, 0)
+    prompt = synth.make_prompt(wl, 0)
+    rows = P + Lg + m.n_tail           # the largest step: nothing cached, nothing truncated
+    cfg = smdm.make_config(m.n_layers, m.d_model, m.n_heads, m.d_head, m.d_ffn, m.vocab,
+                           n_reg=smdm.SMDM_REG_LEN if m.len_token else m.n_reg,
+                           dtype=smdm.SMDM_BF16 if m.dtype == synth.BF16 else smdm.SMDM_F32,
+                           rope_theta=m.rope_theta, rms_eps=m.rms_eps, max_batch=1,
+                           max_len=P + Lg, max_step_rows=rows, max_rows=rows)
+    model = smdm.Model(cfg, device_weights(wl, wl.seed + 7919, dev))
+    stream = torch.cuda.Stream(device=dev)
+    d_prompt = torch.as_tensor(prompt.astype(np.int32), device=dev)
+    d_order = torch.as_tensor(plan.order.astype(np.int32), device=dev)
+    offs = [int(o) for o in plan.offsets]
+    grid = torch.empty(Lg, dtype=torch.int32, device=dev)
+
+    def run():
+        model.smdm_prefill(0, d_prompt, Lg, grid, stream=stream)
+        for k in range(1, plan.n_steps + 1):
+            qp = d_order[offs[k - 1]:offs[k]]
+            model.smdm_step_switched(dict(seq=0, query_pos=qp, n_query=int(qp.numel())),
+                                     args.switches, stream=stream)
+
+    with torch.cuda.stream(stream):
+        run()
+    torch.cuda.synchronize()
+    assert model.smdm_device_status(stream) == 0
+    assert bool((grid >= 0).all())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        run()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            graph.replay()
+        torch.cuda.synchronize()
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    assert model.smdm_device_status(stream) == 0
+    names = {1: "cache_prompt", 2: "cache_res", 4: "truncate"}
+    cfg_line = describe(wl)
+    cfg_line["switches"] = {v: bool(args.switches & b) for b, v in names.items()}
+    cfg_line["timed"] = "CUDA-graph replay of prefill + all sampling steps (smdm_step_switched)"
+    print(json.dumps({"metric": METRIC, "value": Lg / (ms / 1e3), "unit": UNIT, "n_gpus": 1,
+                      "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+                      "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                      "dtype": "bf16" if m.dtype == synth.BF16 else "f32",
+                      "data": "synthetic", "config": cfg_line}), flush=True)
+    del graph
+    model.close()
+    return 0
+
+
 def capacities(wl, plans):
     m = wl.model
     msr = 1
@@ -426,6 +497,8 @@ def main():
 
     if args.form == "training":
         return run_training_form(args, wl)
+    if args.switches != 7:
+        return run_switched(args, wl)
 
     import torch
     import torch.distributed as dist
