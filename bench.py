@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--switches", type=int, default=7, choices=range(8),
                     help="Table-6 speed switches as bits (1 cache prompt, 2 cache decoded "
                          "tokens, 4 truncate); 7 = the method (the default run)")
+    ap.add_argument("--task", default=None, choices=["inpaint", "outpaint", "infill"],
+                    help="bidirectional task: given generation tokens prefilled with the "
+                         "prompt, the plan decodes the rest")
     ap.add_argument("--n-reg", type=int, default=None,
                     help="register rows per step (the method's 64 by default; 0 = the "
                          "length-token variant, one [LEN] row); for the register-count "
@@ -470,6 +473,81 @@ def run_switched(args, wl):
     return 0
 
 
+def run_task(args, wl):
+    """--task inpaint|outpaint|infill: a bidirectional generation task (given generation tokens
+    prefilled with the prompt as block-0 clean rows, smdm_prefill_given) whose plan decodes
+    only the other positions, step by step through smdm_step, replayed as a CUDA graph."""
+    import torch
+    import masked_discrete_diffusion_sparse_b200 as smdm
+    if wl.plan == "semiar" or wl.batch != 1:
+        raise SystemExit("--task supports single-sequence order plans")
+    m = wl.model
+    P, Lg = wl.prompt_len, wl.gen_len
+    dev = torch.device("cuda", 0)
+    task = synth.make_bidir_task(wl, args.task)
+    plan = task.plan
+    prompt = synth.make_prompt(wl, 0)
+    n = [int(v) for v in plan.n_per_step]
+    msr = max((n[i - 1] if i else 0) + n[i] for i in range(len(n))) + m.n_tail
+    n0 = P + len(task.preset_pos)
+    cfg = smdm.make_config(m.n_layers, m.d_model, m.n_heads, m.d_head, m.d_ffn, m.vocab,
+                           n_reg=smdm.SMDM_REG_LEN if m.len_token else m.n_reg,
+                           dtype=smdm.SMDM_BF16 if m.dtype == synth.BF16 else smdm.SMDM_F32,
+                           rope_theta=m.rope_theta, rms_eps=m.rms_eps, max_batch=1,
+                           max_len=P + Lg, max_step_rows=msr, max_rows=max(msr, n0))
+    model = smdm.Model(cfg, device_weights(wl, wl.seed + 7919, dev))
+    stream = torch.cuda.Stream(device=dev)
+    t32 = lambda a: torch.as_tensor(np.asarray(a, dtype=np.int32), device=dev)
+    d_prompt, d_gpos, d_gtok = t32(prompt), t32(task.preset_pos), t32(task.preset_tok)
+    d_order = t32(plan.order)
+    offs = [int(o) for o in plan.offsets]
+    grid = torch.empty(Lg, dtype=torch.int32, device=dev)
+
+    def run():
+        model.smdm_prefill_given(0, d_prompt, Lg, d_gpos, d_gtok, grid, stream=stream)
+        for k in range(1, plan.n_steps + 1):
+            qp = d_order[offs[k - 1]:offs[k]]
+            model.smdm_step([dict(seq=0, query_pos=qp, n_query=int(qp.numel()),
+                                  policy=smdm.SMDM_POLICY_ALL, n_commit=int(qp.numel()))],
+                            stream=stream)
+
+    with torch.cuda.stream(stream):
+        run()
+    torch.cuda.synchronize()
+    assert model.smdm_device_status(stream) == 0
+    assert bool((grid >= 0).all())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        run()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            graph.replay()
+        torch.cuda.synchronize()
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    assert model.smdm_device_status(stream) == 0
+    decoded = len(plan.order)
+    cfg_line = describe(wl)
+    cfg_line.update({"task": args.task, "given_tokens": int(len(task.preset_pos)),
+                     "decoded_tokens": decoded, "sampling_steps": plan.n_steps,
+                     "timed": "CUDA-graph replay of the block-0 prefill (prompt + given "
+                              "tokens) + all sampling steps"})
+    print(json.dumps({"metric": METRIC, "value": decoded / (ms / 1e3), "unit": UNIT,
+                      "n_gpus": 1, "steps": args.steps, "warmup": max(3, args.warmup),
+                      "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                      "vs_baseline": None, "dtype": "bf16" if m.dtype == synth.BF16 else "f32",
+                      "data": "synthetic", "config": cfg_line}), flush=True)
+    del graph
+    model.close()
+    return 0
+
+
 def capacities(wl, plans):
     m = wl.model
     msr = 1
@@ -499,6 +577,8 @@ def main():
         return run_training_form(args, wl)
     if args.switches != 7:
         return run_switched(args, wl)
+    if args.task is not None:
+        return run_task(args, wl)
 
     import torch
     import torch.distributed as dist
