@@ -375,6 +375,7 @@ def test_semiar_run_structure():
         assert ((r.committed_pos >= lo) & (r.committed_pos < hi)).all()
         j = (r.k - 1) % plan.steps_per_block
         assert len(r.query_pos) == wl.block - j * wl.commit
+        assert (np.diff(r.query_pos) > 0).all()          # the block's masks in position order
 
 
 # ------------------------------------------------------------------------------------------
