@@ -10,10 +10,11 @@ CVPR-2026 notes, the paperlayer.ai section summary and the gist.science technica
 that it follows.  Where the pages are silent the reading taken is stated next to the code.
 
 Pinned by ``tests/test_oracle_*.py`` against the worked example, the Figure-3 example, the
-two-path training example, brute-force attention, torch CPU fp64 primitives and the method's
+two-path training example, brute-force attention, torch CPU fp64 primitives, special cases of the
+transformer layer that reduce to closed forms (``test_oracle_layer_pins.py``) and the method's
 exactness invariants (training form == incremental form; truncation/dropping of masks outside C).
-Logit values of random-init models have no printed counterpart on the pages: beyond those
-invariants they are "parity unpinned".
+Logit values of random-init models have no printed counterpart on the pages: beyond those pins
+they are "parity unpinned".
 """
 from __future__ import annotations
 
