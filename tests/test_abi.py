@@ -162,3 +162,47 @@ def test_binding_struct_layouts_match_the_header(tmp_path):
         assert got[(name, "size")] == ctypes.sizeof(cls), name
         for f in cls._fields_:
             assert got[(name, f[0])] == getattr(cls, f[0]).offset, (name, f[0])
+
+
+def test_plain_c_program_links_and_calls_the_library(tmp_path):
+    """The boundary is usable from C: a C program compiled against include/smdm.h and linked
+    with libsmdm.so sizes a workspace and gets the host-side errors (no GPU needed)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    if not os.path.exists(smdm.LIB_PATH):
+        from masked_discrete_diffusion_sparse_b200 import build
+        build.build()
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    src = tmp_path / "use.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "smdm.h"
+int main(void) {
+  smdm_config c = {0};
+  c.n_layers = 2; c.d_model = 256; c.n_heads = 2; c.d_head = 128; c.d_ffn = 704;
+  c.vocab = 1000; c.n_reg = 64; c.dtype = SMDM_BF16; c.rope_theta = 10000.f; c.rms_eps = 1e-6f;
+  c.max_batch = 1; c.max_len = 300; c.max_step_rows = 200; c.max_rows = 300;
+  size_t ws = smdm_workspace_bytes(&c);
+  smdm_handle* h = (smdm_handle*)1;
+  int s1 = smdm_create(&c, NULL, NULL, ws, &h);
+  int s2 = smdm_step(NULL, 1, NULL, NULL, NULL, NULL, 0);
+  c.d_model = 192;
+  size_t bad = smdm_workspace_bytes(&c);
+  printf("%zu %d %d %d %zu %s\n", ws, s1, h == NULL, s2, bad, smdm_last_error(NULL));
+  return 0;
+}
+''')
+    exe = tmp_path / "use"
+    libdir = os.path.dirname(smdm.LIB_PATH)
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), "-I", os.path.join(cuda, "include"),
+                    str(src), "-o", str(exe), "-L", libdir, "-lsmdm",
+                    "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert int(out[0]) > 0
+    assert int(out[1]) == smdm.SMDM_EINVAL and out[2] == "1"
+    assert int(out[3]) == smdm.SMDM_EINVAL
+    assert int(out[4]) == 0
+    assert " ".join(out[5:]) == "null handle"
