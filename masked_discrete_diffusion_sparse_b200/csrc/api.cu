@@ -93,6 +93,22 @@ bool encode_head_tiles(CUtensorMap* m, const void* base, uint64_t row_elems, uin
   return r == CUDA_SUCCESS;
 }
 
+// The same 3-D head-tile view with another box: {64, box_rows, box_sub} (the CTA-pair attention
+// loads half key tiles: 64 rows of all chunks, or 128 rows of one 64-wide chunk).
+bool encode_head_tiles_box(CUtensorMap* m, const void* base, uint64_t row_elems, uint64_t rows,
+                           uint32_t box_rows, uint32_t box_sub) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn || row_elems % 64) return false;
+  cuuint64_t dims[3] = {64, rows, row_elems / 64};
+  cuuint64_t strides[2] = {row_elems * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, box_sub};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // 2-D output map for the GEMM epilogue's TMA stores: `cols` x `rows` elements (bf16 or fp32),
 // row pitch `ld` elements, box {box_cols, 32}, no swizzle.
 bool encode_out(CUtensorMap* m, const void* base, bool f32, uint64_t cols, uint64_t rows,
@@ -286,6 +302,10 @@ struct smdm_handle {
   std::vector<CUtensorMap> tm_qkv, tm_o, tm_gate, tm_up, tm_down, tm_gu;
   std::vector<int> gu_il;   // per layer: 0 two-box gate/up tiles, 1/2 interleaved (tm_gu)
   CUtensorMap tm_lm, tm_kc, tm_vc, tm_kscr, tm_vscr, tm_q;
+  // half-tile K / V views for the CTA-pair attention kernel (d_head 128); pair_maps false when
+  // they could not be encoded (the single-CTA kernel is used)
+  CUtensorMap tm_kc_h, tm_vc_h, tm_kscr_h, tm_vscr_h;
+  bool pair_maps = false;
   std::string err;
   SeqState seq[SMDM_MAX_BATCH];
   int last_rows = 0;
@@ -518,6 +538,8 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
       a.tmQ = &h->tm_q;
       a.tmK = f.scratch_kv ? &h->tm_kscr : &h->tm_kc;
       a.tmV = f.scratch_kv ? &h->tm_vscr : &h->tm_vc;
+      a.tmKh = h->pair_maps ? (f.scratch_kv ? &h->tm_kscr_h : &h->tm_kc_h) : nullptr;
+      a.tmVh = h->pair_maps ? (f.scratch_kv ? &h->tm_vscr_h : &h->tm_vc_h) : nullptr;
       a.cache_rows_per_seq = f.scratch_kv ? 0 : (long long)c.n_layers * c.n_heads * h->L.cap;
       a.cap = kv.cap;
       a.out = ao;
@@ -738,6 +760,15 @@ smdm_status smdm_create(const smdm_config* cfg, const smdm_weights* w, void* d_w
     ok &= encode_head_tiles(&h->tm_kscr, h->at<uint8_t>(h->L.kscr), dh, (uint64_t)H * MR, dh / 64);
     ok &= encode_head_tiles(&h->tm_vscr, h->at<uint8_t>(h->L.vscr), dh, (uint64_t)H * MR, dh / 64);
     ok &= encode_head_tiles(&h->tm_q, h->at<uint8_t>(h->L.q), d, MR, dh / 64);
+    if (dh == 128) {
+      bool pm = encode_head_tiles_box(&h->tm_kc_h, h->at<uint8_t>(h->L.kc), dh, cache_rows, 64, 2);
+      pm &= encode_head_tiles_box(&h->tm_vc_h, h->at<uint8_t>(h->L.vc), dh, cache_rows, 128, 1);
+      pm &= encode_head_tiles_box(&h->tm_kscr_h, h->at<uint8_t>(h->L.kscr), dh, (uint64_t)H * MR,
+                                  64, 2);
+      pm &= encode_head_tiles_box(&h->tm_vscr_h, h->at<uint8_t>(h->L.vscr), dh, (uint64_t)H * MR,
+                                  128, 1);
+      h->pair_maps = pm;
+    }
     if (!ok) {
       delete h;
       return SMDM_ECUDA;

@@ -143,3 +143,21 @@ def test_switched_steps_match_the_oracle(switches):
         assert np.array_equal(grid.cpu().numpy(), st.grid)
     finally:
         model.close()
+
+
+def test_pair_attention_kernel_parity():
+    """The CTA-pair attention kernel (SMDM_ATTN_PAIR=1, d_head 128): the d_head-128 parity cases
+    — sparse runs, the training form, the dense step, bidirectional tasks, the T2I runs — in a
+    child process with the switch on (it is read once per process)."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SMDM_ATTN_PAIR="1")
+    sel = ("tiny-bf16-cos or batched or bidirectional or register_count or config_t2i or "
+           "config_D_batch4 or dense_step_config_C")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-m", "gpu", "-k", sel,
+                        os.path.join(root, "tests", "test_gpu_parity.py"),
+                        os.path.join(root, "tests", "test_gpu_full_configs.py")],
+                       env=env, cwd=root, capture_output=True, text=True, timeout=1800)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
