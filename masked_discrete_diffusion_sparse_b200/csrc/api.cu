@@ -161,7 +161,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
   size_t kc, vc, kscr, vscr, x, h, q, ao, act, hq, pmax, psum, parg, rows, rope, partial,
-      counters, status, newpos, prompts, aux, attn_part, sw, total;
+      counters, status, newpos, prompts, aux, attn_part, lbound, sw, total;
   size_t attn_part_bytes;
   int cap, max_pos, n_vt, rt_max, max_tiles, n_sms;
   size_t partial_bytes;
@@ -172,6 +172,16 @@ struct Layout {
 int tail_rows(const smdm_config* c) { return c->n_reg == SMDM_REG_LEN ? 1 : c->n_reg; }
 // Embedding rows: content ids, [MASK], [LEN] and the registers.
 int emb_rows(const smdm_config* c) { return c->vocab + 2 + std::max(c->n_reg, 0); }
+
+// Process-wide switch: SMDM_TRAIN_BOUND=1 gives the training-form attention per-row key
+// bounds (tiles past a query tile's last visible key are skipped; off by default).
+int train_bound_enabled() {
+  static int v = [] {
+    const char* e = getenv("SMDM_TRAIN_BOUND");
+    return (e && e[0] == '1') ? 1 : 0;
+  }();
+  return v;
+}
 
 bool config_ok(const smdm_config* c, std::string* why) {
   auto fail = [&](const char* s) {
@@ -258,6 +268,8 @@ Layout make_layout(const smdm_config* c, int n_sms) {
   const size_t step_rows = std::min((size_t)c->max_rows, (size_t)c->max_batch * c->max_step_rows);
   L.attn_part_bytes = 16 * step_rows * ((size_t)d * 4 + H * 8);
   L.attn_part = take(L.attn_part_bytes);
+  // training form with key bounds: per-label last indices, their prefix maximum, a flag
+  L.lbound = take((3 * (MR + 1) + 1) * 4);
   // switched steps: per sequence, decoded positions, their steps and the query marks
   L.sw = take((size_t)c->max_batch * 3 * c->max_len * 4);
   L.total = off + 1024;
@@ -417,6 +429,7 @@ struct FwdSpec {
   AttnSeg seg[SMDM_MAX_BATCH];
   int n_logit;                // decode-set rows (0 = no LM head)
   float* logits;              // optional [n_logit][V]
+  bool attn_bound;            // label mode: rows.kvlen holds per-row key bounds
 };
 
 smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensorMap* tmA2,
@@ -526,6 +539,7 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
     if (h->bf16) {
       AttnCall a{};
       a.mode = f.attn_mode;
+      a.bound = f.attn_bound ? 1 : 0;
       a.H = c.n_heads;
       a.dh = c.d_head;
       a.d_model = d;
@@ -1262,9 +1276,16 @@ smdm_status smdm_forward_stepcausal(smdm_handle* h, const int32_t* d_ids, const 
   a.status = h->status();
   { Launch lg_(h, SMDM_K_PACK, st); CK(launch_pack_linear(a, st)); }
   { Launch lg_(h, SMDM_K_OTHER, st); CK(launch_gather_rows(d_logit_rows, n_rows, h->rows.qrow, st)); }
+  const bool bound = h->bf16 && train_bound_enabled();
+  if (bound) {
+    Launch lg_(h, SMDM_K_OTHER, st);
+    CK(launch_label_bounds(h->rows.type, h->rows.label, n, h->at<int>(h->L.lbound),
+                           h->rows.kvlen, st));
+  }
   FwdSpec f{};
   f.R = n;
   f.attn_mode = 1;
+  f.attn_bound = bound;
   f.scratch_kv = true;
   f.n_seg = 1;
   f.seg[0] = AttnSeg{0, 0, n, n, 0};

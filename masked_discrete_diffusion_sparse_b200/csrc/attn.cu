@@ -66,7 +66,9 @@ SMDM_DEV uint32_t pack_bf16x2(float a, float b) {
 
 // DH: head dim (64 or 128) as a compile-time constant so that every MMA issue sequence is
 // straight-line code (control flow between tcgen05.mma instructions stalls the issue).
-template <int DH>
+// kBound (label mode): kvlen[row] bounds the keys a row may see, and a query tile scans key
+// tiles only up to the largest bound of its rows.
+template <int DH, bool kBound = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnDev a) {
@@ -96,7 +98,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int tile = blk - sg.tile0;
   const int qrow0 = sg.row0 + tile * 128;            // first forward row of this tile
   const int nq = min(128, sg.rows - tile * 128);     // valid query rows
-  const int nkeys = sg.nkeys;
+  int nkeys = sg.nkeys;
+  if constexpr (kBound) {
+    __shared__ int tile_hi;
+    griddep_wait();   // the bounds come from an earlier kernel
+    if (threadIdx.x == 0) tile_hi = 0;
+    __syncthreads();
+    for (int r = threadIdx.x; r < nq; r += blockDim.x) atomicMax(&tile_hi, a.kvlen[qrow0 + r]);
+    __syncthreads();
+    nkeys = min(nkeys, tile_hi);
+  }
   const int nkv_all = (nkeys + 127) / 128;
   const int j0 = split * nkv_all / a.nsplit, j1 = (split + 1) * nkv_all / a.nsplit;
   const int nkv = j1 - j0;                           // key tiles of this split
@@ -223,7 +234,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int kv_lim = 0, tq = 0, lq = 0;
     if (valid) {
       if (a.mode == 0) kv_lim = a.kvlen[row];
-      else { tq = a.type[row]; lq = a.label[row]; kv_lim = nkeys; }
+      else { tq = a.type[row]; lq = a.label[row]; kv_lim = kBound ? a.kvlen[row] : nkeys; }
     }
     float m_ref = -INFINITY, l = 0.f;
     const bool warp_any = __any_sync(0xffffffffu, valid);
@@ -923,6 +934,31 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t stream) {
     const int smem = attn_pair_layout(d);
     e = launch_pdl(attn_pair_kernel, dim3((unsigned)(npb * d.nsplit * 2), c.H),
                    dim3(kAttnThreads), smem, stream, 2, *c.tmQ, *c.tmKh, *c.tmVh, d);
+  } else if (c.bound && c.mode == 1) {
+    // label mode with per-row key bounds (training form over step-grouped rows)
+    static bool attr_set[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+      // these instantiations hold a few bytes of static shared memory: leave room for them
+      e = cudaFuncSetAttribute(attn_tc_kernel<128, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(attn_tc_kernel<64, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+    const int smem = attn_layout(c.dh, d);
+    dim3 grid(nb * d.nsplit, c.H);
+    if (c.dh == 128)
+      e = launch_pdl(attn_tc_kernel<128, true>, grid, dim3(kAttnThreads), smem, stream, 1,
+                     *c.tmQ, *c.tmK, *c.tmV, d);
+    else if (c.dh == 64)
+      e = launch_pdl(attn_tc_kernel<64, true>, grid, dim3(kAttnThreads), smem, stream, 1,
+                     *c.tmQ, *c.tmK, *c.tmV, d);
+    else
+      return cudaErrorInvalidValue;
   } else {
     const int smem = attn_layout(c.dh, d);
     dim3 grid(nb * d.nsplit, c.H);

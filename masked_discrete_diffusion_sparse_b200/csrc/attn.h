@@ -15,6 +15,8 @@ struct AttnSeg {
 
 struct AttnCall {
   int mode;                 // 0 = prefix (kvlen per row), 1 = label (step-causal predicate)
+  int bound;                // label mode: kvlen[row] bounds the row's keys (tiles past a query
+                            // tile's largest bound are skipped)
   int H, dh, d_model, layer;
   int n_seg;
   AttnSeg seg[kMaxBatch];

@@ -216,6 +216,79 @@ __global__ void pack_switched_kernel(PackSwArgs a) {
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// Training form, key bounds: kvlen[r] = 1 + the last key index row r may see under the
+// step-causal rule, exact for any row order (rows grouped by step make the bounds triangular,
+// so the attention kernel skips the key tiles after a query tile's last visible key).
+//   lastc[l] / lastm[l]: last index of a clean / mask-or-register row with label l;
+//   a clean query sees clean keys with label <= own: max over l' <= lq of lastc[l'];
+//   a mask or register query: max(max over l' < lq of lastc[l'], lastm[lq]).
+// Scratch: lastc, lastm, prefix (n + 1 each) and a flag, all -1 on entry; a label outside
+// [0, n] sets the flag and every bound stays n.
+// ------------------------------------------------------------------------------------------
+__global__ void label_last_kernel(const int* type, const int* label, int n, int* lastc,
+                                  int* lastm, int* flag) {
+  griddep_launch();
+  griddep_wait();   // launched with programmatic dependent launch
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= n) return;
+  const int l = label[j], t = type[j];
+  if (l < 0 || l > n) {
+    atomicMax(flag, 1);
+    return;
+  }
+  atomicMax((t == kTypePrompt || t == kTypeClean) ? &lastc[l] : &lastm[l], j);
+}
+
+// prefix[l] = max(lastc[0..l]); one CTA, block-wide scan in chunks with a running carry.
+__global__ void label_prefix_kernel(const int* lastc, int n_labels, int* prefix) {
+  griddep_launch();
+  griddep_wait();   // launched with programmatic dependent launch
+  __shared__ int wmax[32];
+  __shared__ int carry;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
+  if (tid == 0) carry = -1;
+  __syncthreads();
+  for (int b0 = 0; b0 < n_labels; b0 += blockDim.x) {
+    const int i = b0 + tid;
+    int v = i < n_labels ? lastc[i] : -1;
+    for (int o = 1; o < 32; o <<= 1) {              // inclusive warp scan (max)
+      const int u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v = max(v, u);
+    }
+    if (lane == 31) wmax[w] = v;
+    __syncthreads();
+    int before = carry;
+    for (int x = 0; x < w; ++x) before = max(before, wmax[x]);
+    v = max(v, before);
+    if (i < n_labels) prefix[i] = v;
+    __syncthreads();
+    if (tid == 0) {
+      int c = carry;
+      for (int x = 0; x < nw; ++x) c = max(c, wmax[x]);
+      carry = c;
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void label_bound_kernel(const int* type, const int* label, int n, const int* lastm,
+                                   const int* prefix, const int* flag, int* kvlen) {
+  griddep_launch();
+  griddep_wait();   // launched with programmatic dependent launch
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= n) return;
+  if (*flag > 0) {
+    kvlen[r] = n;
+    return;
+  }
+  const int l = label[r], t = type[r];
+  const int hi = (t == kTypePrompt || t == kTypeClean)
+                     ? prefix[l]
+                     : max(l > 0 ? prefix[l - 1] : -1, lastm[l]);
+  kvlen[r] = min(n, max(hi + 1, r + 1));   // every row sees itself
+}
+
 // Prefill / dense / training-form rows: one thread per row.
 __global__ void pack_linear_kernel(LinearPackArgs a) {
   griddep_launch();
@@ -470,6 +543,24 @@ cudaError_t launch_pack_linear(const LinearPackArgs& a, cudaStream_t st) {
 }
 cudaError_t launch_pack_switched(const PackSwArgs& a, cudaStream_t st) {
   return launch_pdl(pack_switched_kernel, dim3(1), dim3(512), 0, st, 1, a);
+}
+cudaError_t launch_label_bounds(const int* type, const int* label, int n, int* scratch,
+                                int* kvlen, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  int* lastc = scratch;
+  int* lastm = lastc + (n + 1);
+  int* prefix = lastm + (n + 1);
+  int* flag = prefix + (n + 1);
+  cudaError_t e = launch_fill_i32(scratch, 3 * (n + 1) + 1, -1, st);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(label_last_kernel, dim3((n + 255) / 256), dim3(256), 0, st, 1, type, label, n,
+                 lastc, lastm, flag);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(label_prefix_kernel, dim3(1), dim3(1024), 0, st, 1, (const int*)lastc, n + 1,
+                 prefix);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(label_bound_kernel, dim3((n + 255) / 256), dim3(256), 0, st, 1, type, label,
+                    n, (const int*)lastm, (const int*)prefix, (const int*)flag, kvlen);
 }
 cudaError_t launch_gather_rows(const int* src, int n, int* qrow, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;

@@ -161,3 +161,21 @@ def test_pair_attention_kernel_parity():
                         os.path.join(root, "tests", "test_gpu_full_configs.py")],
                        env=env, cwd=root, capture_output=True, text=True, timeout=1800)
     assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
+
+
+def test_training_form_key_bounds_parity():
+    """The training form with per-row key bounds (SMDM_TRAIN_BOUND=1): its GPU parity cases —
+    the tiny shapes, the text model's first block and the allocation-free entry point — in a
+    child process with the switch on (it is read once per process)."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SMDM_TRAIN_BOUND="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-m", "gpu", "-k",
+                        "forward_stepcausal or noalloc",
+                        os.path.join(root, "tests", "test_gpu_parity.py"),
+                        os.path.join(root, "tests", "test_gpu_full_configs.py"),
+                        os.path.join(root, "tests", "test_zz_no_alloc.py")],
+                       env=env, cwd=root, capture_output=True, text=True, timeout=1800)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
