@@ -3,7 +3,6 @@ the first step) and one-token steps (a single query row, a single new-cache row)
 C ABI against the fp64 oracle with the same bar as the other parity tests."""
 import dataclasses
 
-import numpy as np
 import pytest
 import torch
 

@@ -16,7 +16,7 @@ import torch
 import masked_discrete_diffusion_sparse_b200 as smdm
 import oracle
 import synth
-from smdm_testlib import Runner, i32, logit_err, run_teacher_forced, upload_weights, config_for
+from smdm_testlib import Runner, i32, logit_err, run_teacher_forced
 
 pytestmark = pytest.mark.gpu
 

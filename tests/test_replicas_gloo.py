@@ -5,9 +5,7 @@ multi-rank."""
 import os
 import socket
 
-import numpy as np
 import pytest
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
