@@ -153,6 +153,34 @@ def gemm_bytes_per_run(wl: synth.Workload, plan: synth.Plan, es=2):
     return tot
 
 
+def class_roofline_ms(wl: synth.Workload, plan: synth.Plan, hbm_gbs: float, tflops: float,
+                      es=2) -> dict:
+    """Roofline time per run of each kernel class, max(bytes / HBM, flops / tensor peak) summed
+    over the run's forwards: the weight GEMMs (weights, activation reads, outputs; residual
+    read-modify-write in fp32), attention (K/V read once per layer and written for the step's
+    rows; 4 d flops per visible key) and RMSNorm (fp32 read, activation write)."""
+    m = wl.model
+    d, f, V, L = m.d_model, m.d_ffn, m.vocab, m.n_layers
+    t = lambda byt, fl: max(byt / (hbm_gbs * 1e9), fl / (tflops * 1e12)) * 1e3
+    out = dict.fromkeys(["gemm_qkv", "gemm_o", "gemm_gateup", "gemm_down", "gemm_lmhead",
+                         "attn", "norm"], 0.0)
+    P = wl.prompt_len
+    fwd = ([(P, 0, P * P, 0, P)] if P else []) + \
+          [(R, q, n_new * (ctx + n_new) + (R - n_new) * (ctx + R), ctx, R)
+           for (R, q, ctx, n_new) in step_shapes(wl, plan)]
+    for R, q, kv_sum, ctx, _ in fwd:
+        out["gemm_qkv"] += L * t(es * (3 * d * d + R * d + R * 3 * d), 2 * R * d * 3 * d)
+        out["gemm_o"] += L * t(es * (d * d + R * d) + 4 * 2 * R * d, 2 * R * d * d)
+        out["gemm_gateup"] += L * t(es * (2 * f * d + R * d + R * f), 2 * R * d * 2 * f)
+        out["gemm_down"] += L * t(es * (d * f + R * f) + 4 * 2 * R * d, 2 * R * f * d)
+        if q:
+            out["gemm_lmhead"] += t(es * (V * d + q * d) + 4 * 3 * q * ((V + 127) // 128),
+                                    2 * q * V * d)
+        out["attn"] += L * t((ctx + R) * 2 * d * es + R * 2 * d * es, 4 * d * kv_sum)
+        out["norm"] += t((2 * L * R + q) * (4 * d + es * d), 0)
+    return {k: round(v, 4) for k, v in out.items()}
+
+
 # ----------------------------------------------------------------------------------------------
 # clocks
 # ----------------------------------------------------------------------------------------------
@@ -764,6 +792,7 @@ def main():
                           "frac": roof_s * 1e3 / ms,
                           "peaks": {"hbm_gbs": hbm, "bf16_tflops_sustained": tfl_s}},
         "per_class_ms_per_run": {k: round(v, 4) for k, v in prof["class_ms"].items()},
+        "per_class_roofline_ms_per_run": class_roofline_ms(wl, plans[0], hbm, tfl_s),
         "per_step_ms": ms / wl.n_steps,
         "dense": dense,
     }

@@ -125,3 +125,18 @@ def test_length_token_variant_rows_in_the_bench():
     ref = sorted(zip(o_pos.tolist(), o_types.tolist(), o_labels.tolist()))
     assert mine == ref
     assert sorted(ids[tail].tolist()) == sorted(o_ids[o_types == 3].tolist())
+
+
+def test_class_roofline_agrees_with_the_gemm_byte_count():
+    """With an unbounded tensor peak every class is HBM-bound, so the GEMM classes' roofline
+    times times the bandwidth give back gemm_bytes_per_run, the bytes the bench's roofline
+    line divides by the measured GEMM time."""
+    b = _bench()
+    for name in ("B", "D"):
+        wl = synth.WORKLOADS[name]
+        plan = synth.make_plan(wl, 0)
+        hbm = 1000.0    # GB/s
+        cls = b.class_roofline_ms(wl, plan, hbm, 1e12)
+        gemm_ms = sum(cls[c] for c in ("gemm_qkv", "gemm_o", "gemm_gateup", "gemm_down",
+                                       "gemm_lmhead"))
+        assert abs(gemm_ms * 1e-3 * hbm * 1e9 / b.gemm_bytes_per_run(wl, plan) - 1) < 1e-5
