@@ -118,14 +118,32 @@ def forward_cost(m: synth.ModelShape, R: int, q: int, kv_sum: int, kv_keys: int,
     return wbytes + act + kv, flops
 
 
-def run_cost(wl: synth.Workload, plan: synth.Plan):
-    """List of (bytes, flops) per forward of one full run (prefill first)."""
-    m, P = wl.model, wl.prompt_len
-    costs = [forward_cost(m, P, 0, P * P, P)] if P else []
-    for (R, q, ctx, n_new) in step_shapes(wl, plan):
-        kv_sum = n_new * (ctx + n_new) + (R - n_new) * (ctx + R)
-        costs.append(forward_cost(m, R, q, kv_sum, ctx + R))
-    return costs
+def run_forwards(wl: synth.Workload, plans):
+    """Shapes of the forwards of one full run of the plans' sequences (one plan, or one per
+    sequence of a batch): each sequence's prefill, then one batched forward per step.  Yields
+    (rows R, decode rows q, visible keys summed over rows, keys read per layer)."""
+    if isinstance(plans, synth.Plan):
+        plans = [plans]
+    P = wl.prompt_len
+    if P:
+        for _ in plans:
+            yield P, 0, P * P, P
+    shapes = [step_shapes(wl, p) for p in plans]
+    for k in range(min(len(sh) for sh in shapes)):
+        R = q = kv_sum = keys = 0
+        for sh in shapes:
+            Rb, qb, ctx, n_new = sh[k]
+            R += Rb
+            q += qb
+            kv_sum += n_new * (ctx + n_new) + (Rb - n_new) * (ctx + Rb)
+            keys += ctx + Rb
+        yield R, q, kv_sum, keys
+
+
+def run_cost(wl: synth.Workload, plans):
+    """List of (bytes, flops) per forward of one full run (prefills first)."""
+    return [forward_cost(wl.model, R, q, kv_sum, keys)
+            for (R, q, kv_sum, keys) in run_forwards(wl, plans)]
 
 
 # DRAM bytes (read + write) over algorithmic bytes of gemm_tc_kernel, from one ncu capture of
@@ -134,15 +152,13 @@ def run_cost(wl: synth.Workload, plan: synth.Plan):
 GEMM_TRAFFIC_RATIO = 327.8 / 321.4
 
 
-def gemm_bytes_per_run(wl: synth.Workload, plan: synth.Plan, es=2):
+def gemm_bytes_per_run(wl: synth.Workload, plans, es=2):
     """Algorithmic bytes of the GEMM launches of one full run: weights once per launch plus
     activation operand reads and output writes."""
     m = wl.model
     d, f, V, L = m.d_model, m.d_ffn, m.vocab, m.n_layers
     tot = 0
-    fwd = ([(wl.prompt_len, 0)] if wl.prompt_len else []) + \
-          [(R, q) for (R, q, _, _) in step_shapes(wl, plan)]
-    for R, q in fwd:
+    for R, q, _, _ in run_forwards(wl, plans):
         per_layer = (es * (3 * d * d + R * d + R * 3 * d)            # qkv: W, X, q/k/v out
                      + es * (d * d + R * d) + 4 * 2 * R * d          # o-proj: W, X, x rmw
                      + es * (2 * f * d + R * d + R * f)              # gate/up: W, X, act out
@@ -153,7 +169,7 @@ def gemm_bytes_per_run(wl: synth.Workload, plan: synth.Plan, es=2):
     return tot
 
 
-def class_roofline_ms(wl: synth.Workload, plan: synth.Plan, hbm_gbs: float, tflops: float,
+def class_roofline_ms(wl: synth.Workload, plans, hbm_gbs: float, tflops: float,
                       es=2) -> dict:
     """Roofline time per run of each kernel class, max(bytes / HBM, flops / tensor peak) summed
     over the run's forwards: the weight GEMMs (weights, activation reads, outputs; residual
@@ -164,11 +180,7 @@ def class_roofline_ms(wl: synth.Workload, plan: synth.Plan, hbm_gbs: float, tflo
     t = lambda byt, fl: max(byt / (hbm_gbs * 1e9), fl / (tflops * 1e12)) * 1e3
     out = dict.fromkeys(["gemm_qkv", "gemm_o", "gemm_gateup", "gemm_down", "gemm_lmhead",
                          "attn", "norm"], 0.0)
-    P = wl.prompt_len
-    fwd = ([(P, 0, P * P, 0, P)] if P else []) + \
-          [(R, q, n_new * (ctx + n_new) + (R - n_new) * (ctx + R), ctx, R)
-           for (R, q, ctx, n_new) in step_shapes(wl, plan)]
-    for R, q, kv_sum, ctx, _ in fwd:
+    for R, q, kv_sum, keys in run_forwards(wl, plans):
         out["gemm_qkv"] += L * t(es * (3 * d * d + R * d + R * 3 * d), 2 * R * d * 3 * d)
         out["gemm_o"] += L * t(es * (d * d + R * d) + 4 * 2 * R * d, 2 * R * d * d)
         out["gemm_gateup"] += L * t(es * (2 * f * d + R * d + R * f), 2 * R * d * 2 * f)
@@ -176,7 +188,7 @@ def class_roofline_ms(wl: synth.Workload, plan: synth.Plan, hbm_gbs: float, tflo
         if q:
             out["gemm_lmhead"] += t(es * (V * d + q * d) + 4 * 3 * q * ((V + 127) // 128),
                                     2 * q * V * d)
-        out["attn"] += L * t((ctx + R) * 2 * d * es + R * 2 * d * es, 4 * d * kv_sum)
+        out["attn"] += L * t(keys * 2 * d * es + R * 2 * d * es, 4 * d * kv_sum)
         out["norm"] += t((2 * L * R + q) * (4 * d + es * d), 0)
     return {k: round(v, 4) for k, v in out.items()}
 
@@ -763,10 +775,9 @@ def main():
     gemm_cls = ["gemm_qkv", "gemm_o", "gemm_gateup", "gemm_down", "gemm_lmhead"]
     gemm_ms = sum(prof["class_ms"][c] for c in gemm_cls)
     gemm_n = sum(prof["class_launches"][c] for c in gemm_cls)
-    gb = sum(gemm_bytes_per_run(wl, p) for p in plans) / B if B == 1 else \
-        gemm_bytes_per_run(wl, plans[0])
+    gb = gemm_bytes_per_run(wl, plans)
     achieved = gb / (gemm_ms / 1e3) / 1e9 if gemm_ms > 0 else None
-    costs = run_cost(wl, plans[0])
+    costs = run_cost(wl, plans)
     roof_s = sum(max(b / (hbm * 1e9), f / (tfl_s * 1e12)) for b, f in costs)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -792,7 +803,7 @@ def main():
                           "frac": roof_s * 1e3 / ms,
                           "peaks": {"hbm_gbs": hbm, "bf16_tflops_sustained": tfl_s}},
         "per_class_ms_per_run": {k: round(v, 4) for k, v in prof["class_ms"].items()},
-        "per_class_roofline_ms_per_run": class_roofline_ms(wl, plans[0], hbm, tfl_s),
+        "per_class_roofline_ms_per_run": class_roofline_ms(wl, plans, hbm, tfl_s),
         "per_step_ms": ms / wl.n_steps,
         "dense": dense,
     }

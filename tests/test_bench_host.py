@@ -140,3 +140,19 @@ def test_class_roofline_agrees_with_the_gemm_byte_count():
         gemm_ms = sum(cls[c] for c in ("gemm_qkv", "gemm_o", "gemm_gateup", "gemm_down",
                                        "gemm_lmhead"))
         assert abs(gemm_ms * 1e-3 * hbm * 1e9 / b.gemm_bytes_per_run(wl, plan) - 1) < 1e-5
+
+
+def test_batched_cost_counts_every_sequence():
+    """A batch of sequences: one prefill per sequence, then one forward per step whose rows are
+    the sum of the sequences' rows; for one sequence the cost model is unchanged."""
+    b = _bench()
+    wl = synth.WORKLOADS["D4"]
+    plans = [synth.make_plan(wl, i) for i in range(4)]
+    fwd = list(b.run_forwards(wl, plans))
+    assert len(fwd) == 4 + wl.n_steps
+    singles = [list(b.run_forwards(wl, p)) for p in plans]
+    for k in range(wl.n_steps):
+        R, q, kv_sum, keys = fwd[4 + k]
+        parts = [s[1 + k] for s in singles]
+        assert R == sum(p[0] for p in parts) and q == sum(p[1] for p in parts)
+        assert kv_sum == sum(p[2] for p in parts) and keys == sum(p[3] for p in parts)
