@@ -359,9 +359,10 @@ def device_weights(wl: synth.Workload, seed: int, device):
 
 
 def trajectory_rows(wl: synth.Workload, plan: synth.Plan, prompt: np.ndarray, seed: int):
-    """Rows of a whole sampling trajectory in the step-labelled training form (order plans):
-    the prompt (label 0), then for every step k the clean copies of the tokens decoded at step
-    k, the mask copies of the same positions (the decode set C_k) and the registers, all
+    """Rows of a whole sampling trajectory in the step-labelled training form (order plans),
+    laid out as the oracle's trajectory: the prompt (label 0); the clean copies of the tokens
+    decoded at every step k (label k), step by step; then, step by step, the mask copies of the
+    same positions (the decode set C_k) and the step's tail rows (registers or [LEN]), all
     labelled k.  Token values are random (structure and sizes are what the forward's cost
     depends on).  Returns ids, pos, types, labels and the logit rows (the mask copies)."""
     m = wl.model
@@ -369,15 +370,17 @@ def trajectory_rows(wl: synth.Workload, plan: synth.Plan, prompt: np.ndarray, se
     L = P + Lg
     g = np.random.Generator(np.random.PCG64([wl.seed, 7000 + seed]))
     ids, pos, types, labels, logit_rows = list(prompt), list(range(1, P + 1)), [0] * P, [0] * P, []
-    for k in range(1, plan.n_steps + 1):
-        q = plan.query_positions(k)
+    steps = [plan.query_positions(k) for k in range(1, plan.n_steps + 1)]
+    for k, q in enumerate(steps, start=1):      # clean copies
         n = len(q)
         ids += list(g.integers(0, m.vocab, n))
         pos += list(q)
-        types += [1] * n                      # clean copies
+        types += [1] * n
         labels += [k] * n
+    for k, q in enumerate(steps, start=1):      # mask copies and tail rows
+        n = len(q)
         logit_rows += list(range(len(ids), len(ids) + n))
-        ids += [m.vocab] * n                  # [MASK] copies
+        ids += [m.vocab] * n
         pos += list(q)
         types += [2] * n
         labels += [k] * n

@@ -161,7 +161,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
   size_t kc, vc, kscr, vscr, x, h, q, ao, act, hq, pmax, psum, parg, rows, rope, partial,
-      counters, status, newpos, prompts, aux, attn_part, lbound, sw, total;
+      counters, status, newpos, prompts, aux, attn_part, lbound, tlist, sw, total;
   size_t attn_part_bytes;
   int cap, max_pos, n_vt, rt_max, max_tiles, n_sms;
   size_t partial_bytes;
@@ -270,6 +270,10 @@ Layout make_layout(const smdm_config* c, int n_sms) {
   L.attn_part = take(L.attn_part_bytes);
   // training form with key bounds: per-label last indices, their prefix maximum, a flag
   L.lbound = take((3 * (MR + 1) + 1) * 4);
+  {
+    const size_t T = MR / 128;   // query / key tiles of a training-form forward
+    L.tlist = take((5 * T + T * T) * 4);
+  }
   // switched steps: per sequence, decoded positions, their steps and the query marks
   L.sw = take((size_t)c->max_batch * 3 * c->max_len * 4);
   L.total = off + 1024;
@@ -429,7 +433,9 @@ struct FwdSpec {
   AttnSeg seg[SMDM_MAX_BATCH];
   int n_logit;                // decode-set rows (0 = no LM head)
   float* logits;              // optional [n_logit][V]
-  bool attn_bound;            // label mode: rows.kvlen holds per-row key bounds
+  bool attn_bound;            // label mode: rows.kvlen holds per-row key bounds and
+  const int* tile_list;       // tile_list / tile_count the key tiles of each query tile
+  const int* tile_count;
 };
 
 smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensorMap* tmA2,
@@ -540,6 +546,9 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
       AttnCall a{};
       a.mode = f.attn_mode;
       a.bound = f.attn_bound ? 1 : 0;
+      a.tile_list = f.tile_list;
+      a.tile_count = f.tile_count;
+      a.n_ktiles = (R + 127) / 128;
       a.H = c.n_heads;
       a.dh = c.d_head;
       a.d_model = d;
@@ -1277,15 +1286,21 @@ smdm_status smdm_forward_stepcausal(smdm_handle* h, const int32_t* d_ids, const 
   { Launch lg_(h, SMDM_K_PACK, st); CK(launch_pack_linear(a, st)); }
   { Launch lg_(h, SMDM_K_OTHER, st); CK(launch_gather_rows(d_logit_rows, n_rows, h->rows.qrow, st)); }
   const bool bound = h->bf16 && train_bound_enabled();
+  int* tile_list = nullptr;
+  int* tile_count = nullptr;
   if (bound) {
     Launch lg_(h, SMDM_K_OTHER, st);
     CK(launch_label_bounds(h->rows.type, h->rows.label, n, h->at<int>(h->L.lbound),
                            h->rows.kvlen, st));
+    CK(launch_tile_lists(h->rows.type, h->rows.label, n, h->at<int>(h->L.tlist), &tile_list,
+                         &tile_count, st));
   }
   FwdSpec f{};
   f.R = n;
   f.attn_mode = 1;
   f.attn_bound = bound;
+  f.tile_list = tile_list;
+  f.tile_count = tile_count;
   f.scratch_kv = true;
   f.n_seg = 1;
   f.seg[0] = AttnSeg{0, 0, n, n, 0};

@@ -43,6 +43,9 @@ struct AttnDev {
   int rows_total;
   float* part_o;                  // [nsplit][rows_total][d_model]
   float* part_ml;                 // [nsplit][rows_total][H][2]
+  const int* tile_list;           // bounded label mode: [query tile][n_ktiles] key tiles
+  const int* tile_count;          // [query tile] listed key tiles
+  int n_ktiles;
 };
 
 SMDM_DEV void p_store_swizzled(uint8_t* P, int row, int key8, uint4 val) {
@@ -98,17 +101,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int tile = blk - sg.tile0;
   const int qrow0 = sg.row0 + tile * 128;            // first forward row of this tile
   const int nq = min(128, sg.rows - tile * 128);     // valid query rows
-  int nkeys = sg.nkeys;
+  const int nkeys = sg.nkeys;
+  // key tiles to scan: all of [0, nkeys), or with kBound the listed ones of this query tile
+  const int* tlist = nullptr;
+  int nkv_all = (nkeys + 127) / 128;
   if constexpr (kBound) {
-    __shared__ int tile_hi;
-    griddep_wait();   // the bounds come from an earlier kernel
-    if (threadIdx.x == 0) tile_hi = 0;
-    __syncthreads();
-    for (int r = threadIdx.x; r < nq; r += blockDim.x) atomicMax(&tile_hi, a.kvlen[qrow0 + r]);
-    __syncthreads();
-    nkeys = min(nkeys, tile_hi);
+    griddep_wait();   // the lists come from earlier kernels
+    const int tq = qrow0 >> 7;   // training form: one segment starting at row 0
+    tlist = a.tile_list + (size_t)tq * a.n_ktiles;
+    nkv_all = a.tile_count[tq];
   }
-  const int nkv_all = (nkeys + 127) / 128;
   const int j0 = split * nkv_all / a.nsplit, j1 = (split + 1) * nkv_all / a.nsplit;
   const int nkv = j1 - j0;                           // key tiles of this split
   constexpr int dh = DH;
@@ -169,7 +171,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!mbar_wait(&kv_empty[stage], phase ^ 1, abort_flag, a.status)) break;
         uint8_t* Ks = smem + a.k_off + stage * a.stage_bytes;
         uint8_t* Vs = smem + a.v_off + stage * a.stage_bytes;
-        const int y = (int)(cache_base + (long long)(j0 + j) * 128);
+        const int kt = kBound ? tlist[j0 + j] : (j0 + j);
+        const int y = (int)(cache_base + (long long)kt * 128);
         mbar_arrive_expect_tx(&k_full[stage], 128 * dh * 2);
         tma_load_3d(Ks, &tmK, &k_full[stage], 0, y, 0, pol_kv);
         mbar_arrive_expect_tx(&v_full[stage], 128 * dh * 2);
@@ -254,7 +257,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (lane == 0) mbar_arrive(&p_full[j & 1]);
         continue;
       }
-      const int key0 = (j0 + j) * 128;
+      const int key0 = (kBound ? tlist[j0 + j] : (j0 + j)) * 128;
       // visibility of the 128 keys as four 32-bit masks (registers only, no local arrays)
       uint32_t mw[4];
 #pragma unroll
@@ -901,6 +904,9 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t stream) {
   d.scale_log2 = 1.4426950408889634f / sqrtf((float)c.dh);
   d.out = c.out;
   d.status = c.status;
+  d.tile_list = c.tile_list;
+  d.tile_count = c.tile_count;
+  d.n_ktiles = c.n_ktiles;
   if (c.n_seg < 1 || c.n_seg > kMaxBatch) return cudaErrorInvalidValue;
   int nb = 0;
   d.n_seg = c.n_seg;
@@ -934,7 +940,8 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t stream) {
     const int smem = attn_pair_layout(d);
     e = launch_pdl(attn_pair_kernel, dim3((unsigned)(npb * d.nsplit * 2), c.H),
                    dim3(kAttnThreads), smem, stream, 2, *c.tmQ, *c.tmKh, *c.tmVh, d);
-  } else if (c.bound && c.mode == 1) {
+  } else if (c.bound && c.mode == 1 && c.tile_list && c.tile_count && c.n_seg == 1 &&
+             c.seg[0].row0 == 0) {
     // label mode with per-row key bounds (training form over step-grouped rows)
     static bool attr_set[64];
     int dev = 0;

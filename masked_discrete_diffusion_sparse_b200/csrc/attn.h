@@ -15,8 +15,11 @@ struct AttnSeg {
 
 struct AttnCall {
   int mode;                 // 0 = prefix (kvlen per row), 1 = label (step-causal predicate)
-  int bound;                // label mode: kvlen[row] bounds the row's keys (tiles past a query
-                            // tile's largest bound are skipped)
+  int bound;                // label mode: kvlen[row] bounds the row's keys, and each 128-row
+                            // query tile scans only the key tiles listed for it
+  const int* tile_list;     // [query tile][n_ktiles] key tiles (ascending), bounded mode
+  const int* tile_count;    // [query tile] number of listed key tiles
+  int n_ktiles;
   int H, dh, d_model, layer;
   int n_seg;
   AttnSeg seg[kMaxBatch];

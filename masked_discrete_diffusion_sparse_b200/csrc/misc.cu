@@ -6,6 +6,8 @@
 //   unmask      — confidence/argmax from the LM-head partials, top-n selection and the
 //                 scatter of committed tokens into the grid (Figure-3 example, Sec. 3.2);
 //   debug_mask  — the device step-causal predicate as a bitmap (test hook).
+#include <climits>
+
 #include "misc.h"
 
 namespace smdm {
@@ -289,6 +291,74 @@ __global__ void label_bound_kernel(const int* type, const int* label, int n, con
   kvlen[r] = min(n, max(hi + 1, r + 1));   // every row sees itself
 }
 
+// ------------------------------------------------------------------------------------------
+// Training form, key-tile lists: for every 128-row query tile, the 128-row key tiles that may
+// hold a key visible to one of its rows (the keys are the forward's own rows).  A tile is
+// summarised by the label ranges of its clean rows [cmin, cmax] and of its mask/register rows
+// [mmin, mmax] (empty: INT_MAX / INT_MIN).  Key tile T may matter to query tile Q when
+//   Q has clean rows and T a clean key with label <= Q's largest clean label, or
+//   Q has mask/register rows and T a clean key with label < Q's largest such label, or T's
+//   mask/register labels overlap Q's —
+// a superset of the tiles the step-causal rule needs (each visible pair satisfies one of them).
+// ------------------------------------------------------------------------------------------
+__global__ void tile_summary_kernel(const int* type, const int* label, int n, int4* summary) {
+  griddep_launch();
+  griddep_wait();   // launched with programmatic dependent launch
+  __shared__ int s[4];
+  if (threadIdx.x == 0) {
+    s[0] = INT_MAX;
+    s[1] = INT_MIN;
+    s[2] = INT_MAX;
+    s[3] = INT_MIN;
+  }
+  __syncthreads();
+  const int r = blockIdx.x * 128 + threadIdx.x;
+  if (r < n) {
+    const int l = label[r], t = type[r];
+    if (t == kTypePrompt || t == kTypeClean) {
+      atomicMin(&s[0], l);
+      atomicMax(&s[1], l);
+    } else {
+      atomicMin(&s[2], l);
+      atomicMax(&s[3], l);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) summary[blockIdx.x] = make_int4(s[0], s[1], s[2], s[3]);
+}
+
+__global__ void tile_list_kernel(const int4* summary, int n_tiles, int* lists, int* counts) {
+  griddep_launch();
+  griddep_wait();   // launched with programmatic dependent launch
+  __shared__ int warp_counts[4];
+  __shared__ int found;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int4 q = summary[blockIdx.x];
+  int* list = lists + (size_t)blockIdx.x * n_tiles;
+  if (tid == 0) found = 0;
+  __syncthreads();
+  for (int b0 = 0; b0 < n_tiles; b0 += 128) {
+    const int t = b0 + tid;
+    bool vis = false;
+    if (t < n_tiles) {
+      const int4 k = summary[t];
+      vis = (k.x <= q.y) ||                                   // clean query, clean key
+            (k.x < q.w) ||                                    // mask/register query, clean key
+            (max(k.z, q.z) <= min(k.w, q.w));                 // same mask/register label
+    }
+    const unsigned ballot = __ballot_sync(0xffffffffu, vis);
+    if (lane == 0) warp_counts[w] = __popc(ballot);
+    __syncthreads();
+    int before = found;
+    for (int x = 0; x < w; ++x) before += warp_counts[x];
+    if (vis) list[before + __popc(ballot & ((1u << lane) - 1u))] = t;
+    __syncthreads();
+    if (tid == 0) found += warp_counts[0] + warp_counts[1] + warp_counts[2] + warp_counts[3];
+    __syncthreads();
+  }
+  if (tid == 0) counts[blockIdx.x] = found;
+}
+
 // Prefill / dense / training-form rows: one thread per row.
 __global__ void pack_linear_kernel(LinearPackArgs a) {
   griddep_launch();
@@ -561,6 +631,19 @@ cudaError_t launch_label_bounds(const int* type, const int* label, int n, int* s
   if (e != cudaSuccess) return e;
   return launch_pdl(label_bound_kernel, dim3((n + 255) / 256), dim3(256), 0, st, 1, type, label,
                     n, (const int*)lastm, (const int*)prefix, (const int*)flag, kvlen);
+}
+cudaError_t launch_tile_lists(const int* type, const int* label, int n, int* scratch,
+                              int** lists, int** counts, cudaStream_t st) {
+  const int T = (n + 127) / 128;
+  int4* summary = reinterpret_cast<int4*>(scratch);
+  *counts = scratch + 4 * T;
+  *lists = *counts + T;
+  if (n <= 0) return cudaSuccess;
+  cudaError_t e = launch_pdl(tile_summary_kernel, dim3(T), dim3(128), 0, st, 1, type, label, n,
+                             summary);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(tile_list_kernel, dim3(T), dim3(128), 0, st, 1, (const int4*)summary, T,
+                    *lists, *counts);
 }
 cudaError_t launch_gather_rows(const int* src, int n, int* qrow, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;

@@ -116,6 +116,10 @@ cudaError_t launch_gather_rows(const int* src, int n, int* qrow, cudaStream_t st
 // scratch: 3 * (n + 1) + 1 ints.
 cudaError_t launch_label_bounds(const int* type, const int* label, int n, int* scratch,
                                 int* kvlen, cudaStream_t st);
+// Training form: per 128-row query tile, the key tiles that may hold a visible key (see
+// misc.cu).  scratch: 5 * T + T * T ints, T = ceil(n / 128); returns the list and count arrays.
+cudaError_t launch_tile_lists(const int* type, const int* label, int n, int* scratch,
+                              int** lists, int** counts, cudaStream_t st);
 template <typename T>
 cudaError_t launch_rmsnorm(const NormArgs& a, int rows, cudaStream_t st);
 cudaError_t launch_unmask(const UnmaskArgs& a, int max_nq, cudaStream_t st);

@@ -72,3 +72,76 @@ def test_trajectory_rows_get_triangular_bounds():
     assert np.array_equal(kv, [np.flatnonzero(vis[r]).max() + 1 for r in range(n)])
     assert np.all(np.diff(kv) >= 0)
     assert kv.sum() < 0.6 * n * n          # about half of the full n x n scan
+
+
+# ------------------------------------------------------------------------------------------
+# Key-tile lists: per 128-row query tile, the key tiles that may hold a visible key.
+# ------------------------------------------------------------------------------------------
+
+BIG, SMALL = 2 ** 31 - 1, -2 ** 31
+
+
+def tile_summary(types, labels, tile):
+    """Per tile: label ranges of its clean rows and of its mask/register rows (empty: BIG/SMALL)."""
+    out = []
+    for t0 in range(0, len(types), tile):
+        ty, lb = types[t0:t0 + tile], labels[t0:t0 + tile]
+        c = [l for t, l in zip(ty, lb) if t in CLEAN_TYPES]
+        m = [l for t, l in zip(ty, lb) if t not in CLEAN_TYPES]
+        out.append((min(c, default=BIG), max(c, default=SMALL),
+                    min(m, default=BIG), max(m, default=SMALL)))
+    return out
+
+
+def library_tile_lists(types, labels, tile=128):
+    s = tile_summary(types, labels, tile)
+    lists = []
+    for q in s:
+        lists.append([t for t, k in enumerate(s)
+                      if k[0] <= q[1] or k[0] < q[3] or max(k[2], q[2]) <= min(k[3], q[3])])
+    return lists
+
+
+def test_tile_lists_cover_every_visible_key():
+    g = np.random.Generator(np.random.PCG64(23))
+    tile = 8   # small tiles, the same rule as the library's 128
+    for trial in range(30):
+        n = int(g.integers(1, 90))
+        types = g.integers(0, 4, n)
+        labels = g.integers(0, 7, n)
+        labels[types == oracle.PROMPT] = 0
+        vis = oracle.cross_mask(types, labels, types, labels)
+        lists = library_tile_lists(types, labels, tile)
+        for qt, lst in enumerate(lists):
+            need = {j // tile for r in range(qt * tile, min(n, qt * tile + tile))
+                    for j in np.flatnonzero(vis[r])}
+            assert need <= set(lst), (trial, qt)
+            assert lst == sorted(lst)
+
+
+def test_tile_lists_skip_most_of_a_trajectory():
+    """Rows laid out as the oracle's trajectory and bench.py --form training lay them out
+    (the prompt, every step's clean tokens by step, then every step's masks and registers by
+    step): a query tile's list holds the clean prefix it may see and its own mask block, so the
+    lists cover a small part of the full scan and of the triangular bound, and still every
+    tile a visible key needs."""
+    P, Lg, K, nreg, tile = 16, 256, 16, 8, 16
+    n = synth.cosine_schedule(Lg, K)
+    types, labels = [oracle.PROMPT] * P, [0] * P
+    for k in range(1, K + 1):
+        types += [oracle.CLEAN] * n[k - 1]
+        labels += [k] * n[k - 1]
+    for k in range(1, K + 1):
+        types += [oracle.MASK] * n[k - 1] + [oracle.REG] * nreg
+        labels += [k] * (n[k - 1] + nreg)
+    types, labels = np.array(types), np.array(labels)
+    vis = oracle.cross_mask(types, labels, types, labels)
+    lists = library_tile_lists(types, labels, tile)
+    kv = library_bounds(types, labels)
+    T = len(lists)
+    rows_of = lambda q: range(q * tile, min(len(kv), q * tile + tile))
+    listed = sum(len(x) for x in lists)
+    bounded = sum((max(kv[r] for r in rows_of(q)) + tile - 1) // tile for q in range(T))
+    for q in range(T):
+        assert {j // tile for r in rows_of(q) for j in np.flatnonzero(vis[r])} <= set(lists[q])
+    assert listed < 0.6 * bounded and listed < 0.3 * T * T
