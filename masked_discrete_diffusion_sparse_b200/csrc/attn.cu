@@ -69,8 +69,8 @@ SMDM_DEV uint32_t pack_bf16x2(float a, float b) {
 
 // DH: head dim (64 or 128) as a compile-time constant so that every MMA issue sequence is
 // straight-line code (control flow between tcgen05.mma instructions stalls the issue).
-// kBound (label mode): kvlen[row] bounds the keys a row may see, and a query tile scans key
-// tiles only up to the largest bound of its rows.
+// kBound (label mode, training form from row 0): kvlen[row] bounds the keys a row may see, and
+// a query tile scans only the key tiles listed for it (tile_list / tile_count).
 template <int DH, bool kBound = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
