@@ -15,6 +15,9 @@
 // shared-memory buffers, final 1/l scaling (or the unnormalised partial for the combine).  The running maximum is
 // only moved (and O rescaled) when it grows by more than 2^8, so most tiles skip the rescale;
 // the result is exact because numerator and denominator share the reference maximum.
+// Opt-in variants: attn_pair_kernel (d_head 128, SMDM_ATTN_PAIR=1) streams each key tile once
+// for two query tiles as M=256 MMAs of a CTA pair; the bounded label-mode instantiation
+// (SMDM_TRAIN_BOUND=1) scans only the key tiles listed for each query tile.
 // fp32 path: one warp per (row, head), SIMT.
 #include <algorithm>
 
