@@ -143,9 +143,11 @@ smdm_status smdm_prefill_given(smdm_handle* h, int seq, const int32_t* d_prompt,
 
 /* One sampling step for one sequence (Figure-3 example; Sec. 3.2; Appendix 7.2).
  * Rows, in this order: the tokens decoded at the previous step of this sequence (new cache:
- * their ids from the grid, label k-1), the decode set C (id [MASK], label k), n_reg registers.
- *  - d_query_pos != NULL: C is this explicit list of n_query 1-based positions (each still
- *    masked, no duplicates — validated on the device only in checked builds).
+ * their ids from the grid, label k-1), the decode set C (id [MASK], label k), n_reg registers
+ * (or the one [LEN] row when n_reg = SMDM_REG_LEN).
+ *  - d_query_pos != NULL: C is this explicit list of n_query 1-based positions, each in the
+ *    generated region and still masked (checked on the device: a violation sets the status
+ *    word, SMDM_EDEVICE at the next synchronising call); duplicates are not detected.
  *  - d_query_pos == NULL: C is every still-masked position in [block_lo, block_hi) in
  *    position order (semi-autoregressive block decoding); n_query must equal their number.
  * After the forward: tok = argmax of the row's logits (ties -> lowest id), conf = max softmax
