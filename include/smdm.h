@@ -233,7 +233,10 @@ smdm_status smdm_generate(smdm_handle* h, int batch, const int32_t* d_prompts, i
  * CLEAN label = the step they were decoded at) see clean rows with label <= theirs; MASK and
  * REG rows of label s see clean rows with label < s and the MASK/REG rows of label s.
  * Writes fp32 logits [n_rows][vocab] for the rows listed in d_logit_rows.  Does not touch any
- * sequence's generation state. */
+ * sequence's generation state.  Any row order is allowed.  With the environment variable
+ * SMDM_TRAIN_BOUND=1 (bf16 models) the attention skips the 128-key tiles that hold no key
+ * visible to a 128-row query tile (same result); rows laid out as prompt, clean tokens by
+ * step, then each step's masks and registers skip most of them. */
 smdm_status smdm_forward_stepcausal(smdm_handle* h, const int32_t* d_ids, const int32_t* d_pos,
                                     const int32_t* d_type, const int32_t* d_label, int n,
                                     const int32_t* d_logit_rows, int n_rows, float* d_logits,
