@@ -163,6 +163,8 @@ struct Layout {
   size_t kc, vc, kscr, vscr, x, h, q, ao, act, hq, pmax, psum, parg, rows, rope, partial,
       counters, status, newpos, prompts, aux, attn_part, lbound, tlist, sw, total;
   size_t attn_part_bytes;
+  size_t qkv32 = 0;          // split QKV: fp32 q|k|v rows [max rows][3 d] (when has_qkv32)
+  bool has_qkv32 = false;
   int cap, max_pos, n_vt, rt_max, max_tiles, n_sms;
   size_t partial_bytes;
 };
@@ -175,6 +177,17 @@ int emb_rows(const smdm_config* c) { return c->vocab + 2 + std::max(c->n_reg, 0)
 
 // Process-wide switch: SMDM_TRAIN_BOUND=1 gives the training-form attention per-row key
 // bounds (tiles past a query tile's last visible key are skipped; off by default).
+// Process-wide switch: SMDM_QKV_SPLIT=1 runs the QKV GEMM (bf16 models) with an additive fp32
+// epilogue spread over all SMs, and a finalize kernel for RoPE and the K/V append (off by
+// default).
+int qkv_split_enabled() {
+  static int v = [] {
+    const char* e = getenv("SMDM_QKV_SPLIT");
+    return (e && e[0] == '1') ? 1 : 0;
+  }();
+  return v;
+}
+
 int train_bound_enabled() {
   static int v = [] {
     const char* e = getenv("SMDM_TRAIN_BOUND");
@@ -220,7 +233,8 @@ int query_sms() {
   return n;
 }
 
-Layout make_layout(const smdm_config* c, int n_sms) {
+// extras: also the opt-in split-QKV buffer (not for the allocation-free path)
+Layout make_layout(const smdm_config* c, int n_sms, bool extras = true) {
   Layout L{};
   const size_t es = c->dtype == SMDM_BF16 ? 2 : 4;
   const size_t d = c->d_model, H = c->n_heads, dh = c->d_head;
@@ -274,6 +288,10 @@ Layout make_layout(const smdm_config* c, int n_sms) {
     const size_t T = MR / 128;   // query / key tiles of a training-form forward
     L.tlist = take((5 * T + T * T) * 4);
   }
+  if (extras && qkv_split_enabled() && c->dtype == SMDM_BF16) {
+    L.qkv32 = take(MR * 3 * d * 4);
+    L.has_qkv32 = true;
+  }
   // switched steps: per sequence, decoded positions, their steps and the query marks
   L.sw = take((size_t)c->max_batch * 3 * c->max_len * 4);
   L.total = off + 1024;
@@ -322,6 +340,9 @@ struct smdm_handle {
   // they could not be encoded (the single-CTA kernel is used)
   CUtensorMap tm_kc_h, tm_vc_h, tm_kscr_h, tm_vscr_h;
   bool pair_maps = false;
+  // split QKV (SMDM_QKV_SPLIT=1): plain 2-D maps of W_qkv; qkv_split false when not in use
+  std::vector<CUtensorMap> tm_qkv_plain;
+  bool qkv_split = false;
   std::string err;
   SeqState seq[SMDM_MAX_BATCH];
   int last_rows = 0;
@@ -440,7 +461,7 @@ struct FwdSpec {
 
 smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensorMap* tmA2,
                  const void* W, const void* W2, void* X, int K, int n_out, int rows, int swiglu,
-                 const EpiParams& ep, cudaStream_t st, int a_interleave = 0) {
+                 const EpiParams& ep, cudaStream_t st, int a_interleave = 0, int sched = 0) {
   if (rows <= 0) return SMDM_OK;
   Launch lg(h, cls, st);
   if (h->bf16) {
@@ -476,6 +497,7 @@ smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensor
     c.swiglu = swiglu;
     c.swiglu_il = swiglu && ep.swiglu_il;
     c.a_interleave = a_interleave;
+    c.sched = sched;
     c.num_ctas = h->L.n_sms;
     c.partial = h->at<float>(h->L.partial);
     c.partial_bytes = h->L.partial_bytes;
@@ -538,9 +560,35 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
     ep.row_slot = rw.slot;
     ep.row_pos = rw.pos;
     ep.rope = h->at<float2>(h->L.rope);
-    if ((s = gemm(h, SMDM_K_GEMM_QKV, h->bf16 ? &h->tm_qkv[l] : nullptr, nullptr, h->w_qkv[l], nullptr, hb, d,
-                  3 * d, R, 0, ep, st, c.d_head)))
+    if (h->qkv_split) {
+      // additive fp32 q|k|v over all SMs (stream-K, no fix-up), then RoPE + K/V append
+      EpiParams eq{};
+      eq.kind = kEpiResid;
+      eq.rows = R;
+      eq.n_valid = 3 * d;
+      eq.x = h->at<float>(h->L.qkv32);
+      eq.ld_x = 3 * d;
+      if ((s = gemm(h, SMDM_K_GEMM_QKV, &h->tm_qkv_plain[l], nullptr, h->w_qkv[l], nullptr, hb,
+                    d, 3 * d, R, 0, eq, st, 0, 2)))
+        return s;
+      QkvFinalArgs qa{};
+      qa.qkv32 = eq.x;
+      qa.rows = R;
+      qa.d = d;
+      qa.dh = c.d_head;
+      qa.layer = ep.layer;
+      qa.pos = rw.pos;
+      qa.seq = rw.seq;
+      qa.slot = rw.slot;
+      qa.rope = ep.rope;
+      qa.q_out = static_cast<__nv_bfloat16*>(q);
+      qa.kv = kv;
+      Launch lgq(h, SMDM_K_GEMM_QKV, st);
+      CK(launch_qkv_finalize(qa, st));
+    } else if ((s = gemm(h, SMDM_K_GEMM_QKV, h->bf16 ? &h->tm_qkv[l] : nullptr, nullptr,
+                         h->w_qkv[l], nullptr, hb, d, 3 * d, R, 0, ep, st, c.d_head))) {
       return s;
+    }
     // step-causal attention
     if (h->bf16) {
       AttnCall a{};
@@ -783,6 +831,14 @@ smdm_status smdm_create(const smdm_config* cfg, const smdm_weights* w, void* d_w
     ok &= encode_head_tiles(&h->tm_kscr, h->at<uint8_t>(h->L.kscr), dh, (uint64_t)H * MR, dh / 64);
     ok &= encode_head_tiles(&h->tm_vscr, h->at<uint8_t>(h->L.vscr), dh, (uint64_t)H * MR, dh / 64);
     ok &= encode_head_tiles(&h->tm_q, h->at<uint8_t>(h->L.q), d, MR, dh / 64);
+    if (h->L.has_qkv32) {
+      bool qs = true;
+      h->tm_qkv_plain.resize(nl);
+      for (int l = 0; l < nl; ++l)
+        qs &= encode_2d(&h->tm_qkv_plain[l], w->w_qkv[l], d, 3 * (uint64_t)d, (uint64_t)d * 2, 64,
+                        128);
+      h->qkv_split = qs;
+    }
     if (dh == 128) {
       bool pm = encode_head_tiles_box(&h->tm_kc_h, h->at<uint8_t>(h->L.kc), dh, cache_rows, 64, 2);
       pm &= encode_head_tiles_box(&h->tm_vc_h, h->at<uint8_t>(h->L.vc), dh, cache_rows, 128, 1);
@@ -1448,7 +1504,7 @@ extern "C" smdm_status smdm_forward_stepcausal_noalloc(
   vc.max_batch = 1;
   vc.max_step_rows = 1;
   vc.max_rows = std::max(n, n_rows);
-  const Layout L = make_layout(&vc, SMDM_NOALLOC_GEMM_CTAS);
+  const Layout L = make_layout(&vc, SMDM_NOALLOC_GEMM_CTAS, false);
   if (L.total > SMDM_NOALLOC_SCRATCH_BYTES) return SMDM_ESHAPE;
   smdm_handle* h = D.handle;
   h->cfg = vc;

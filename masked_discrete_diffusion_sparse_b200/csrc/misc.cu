@@ -359,6 +359,49 @@ __global__ void tile_list_kernel(const int4* summary, int n_tiles, int* lists, i
   if (tid == 0) counts[blockIdx.x] = found;
 }
 
+// ------------------------------------------------------------------------------------------
+// Split-QKV finalize (SMDM_QKV_SPLIT=1).  The QKV GEMM ran with an additive fp32 epilogue into
+// qkv32 [rows][3d] (split segments of a tile add independently, so every tile's K range can be
+// spread over all SMs with no fix-up).  Here: the rotary embedding of q and k (rotate-half
+// pairs (i, i + dh/2) of each head, angles of the row's position), q to q_out, k and v to the
+// cache rows at (seq, layer, head, slot), all bf16; the fp32 rows are zeroed for the next
+// launch.  One CTA per row.
+// ------------------------------------------------------------------------------------------
+__global__ void qkv_finalize_kernel(QkvFinalArgs a) {
+  griddep_launch();
+  griddep_wait();   // launched with programmatic dependent launch
+  const int r = blockIdx.x;
+  const int d = a.d, dh = a.dh, half = dh >> 1;
+  float* row = a.qkv32 + (size_t)r * 3 * d;
+  const float2* cs = a.rope + (size_t)a.pos[r] * half;
+  const long long kvoff = (long long)a.seq[r] * a.kv.seq_stride +
+                          (long long)a.layer * a.kv.layer_stride + (long long)a.slot[r] * dh;
+  __nv_bfloat16* q = a.q_out + (size_t)r * d;
+  __nv_bfloat16* K = reinterpret_cast<__nv_bfloat16*>(a.kv.k) + kvoff;
+  __nv_bfloat16* V = reinterpret_cast<__nv_bfloat16*>(a.kv.v) + kvoff;
+  for (int t = threadIdx.x; t < d / 2; t += blockDim.x) {   // rotary pairs of q and k
+    const int h = t / half, i = t - h * half;
+    const int f1 = h * dh + i, f2 = f1 + half;
+    const float2 c = cs[i];
+    const float q1 = row[f1], q2 = row[f2];
+    q[f1] = __float2bfloat16_rn(q1 * c.x - q2 * c.y);
+    q[f2] = __float2bfloat16_rn(q2 * c.x + q1 * c.y);
+    const float k1 = row[d + f1], k2 = row[d + f2];
+    __nv_bfloat16* Kh = K + (long long)h * a.kv.head_stride;
+    Kh[i] = __float2bfloat16_rn(k1 * c.x - k2 * c.y);
+    Kh[i + half] = __float2bfloat16_rn(k2 * c.x + k1 * c.y);
+    row[f1] = 0.f;
+    row[f2] = 0.f;
+    row[d + f1] = 0.f;
+    row[d + f2] = 0.f;
+  }
+  for (int f = threadIdx.x; f < d; f += blockDim.x) {      // v
+    const int h = f / dh;
+    V[(long long)h * a.kv.head_stride + (f - h * dh)] = __float2bfloat16_rn(row[2 * d + f]);
+    row[2 * d + f] = 0.f;
+  }
+}
+
 // Prefill / dense / training-form rows: one thread per row.
 __global__ void pack_linear_kernel(LinearPackArgs a) {
   griddep_launch();
@@ -606,6 +649,10 @@ __global__ void fill_i32_kernel(int* p, int n, int v) {
 // ------------------------------------------------------------------------------------------
 cudaError_t launch_pack_step(const PackArgs& a, cudaStream_t st) {
   return launch_pdl(pack_step_kernel, dim3(a.n_seq), dim3(256), 0, st, 1, a);
+}
+cudaError_t launch_qkv_finalize(const QkvFinalArgs& a, cudaStream_t st) {
+  if (a.rows <= 0) return cudaSuccess;
+  return launch_pdl(qkv_finalize_kernel, dim3(a.rows), dim3(256), 0, st, 1, a);
 }
 cudaError_t launch_pack_linear(const LinearPackArgs& a, cudaStream_t st) {
   if (a.n <= 0) return cudaSuccess;

@@ -179,3 +179,23 @@ def test_training_form_key_bounds_parity():
                         os.path.join(root, "tests", "test_zz_no_alloc.py")],
                        env=env, cwd=root, capture_output=True, text=True, timeout=1800)
     assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
+
+
+def test_split_qkv_parity():
+    """The split QKV path (SMDM_QKV_SPLIT=1: an additive fp32 QKV GEMM over all SMs and a
+    finalize kernel for RoPE and the K/V append): the bf16 GPU parity cases — sparse runs of
+    both head sizes, the batched step, the dense step and the training form — in a child
+    process with the switch on (it is read once per process)."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SMDM_QKV_SPLIT="1")
+    sel = ("bf16 or batched or bidirectional or register_count or config_t2i or "
+           "config_B_text or dense_step_config_C or forward_stepcausal_config_B or edge")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-m", "gpu", "-k", sel,
+                        os.path.join(root, "tests", "test_gpu_edge_cases.py"),
+                        os.path.join(root, "tests", "test_gpu_parity.py"),
+                        os.path.join(root, "tests", "test_gpu_full_configs.py")],
+                       env=env, cwd=root, capture_output=True, text=True, timeout=2400)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
