@@ -1,7 +1,8 @@
 // C ABI of the sparse sampling library: handle, workspace carving, TMA descriptors and the
 // forward driver that chains the kernels of one step (pack -> [QKV+RoPE+KV append ->
 // step-causal attention -> O-proj+residual -> RMSNorm -> gate/up+SwiGLU -> down+residual ->
-// RMSNorm] x layers -> LM head over the decode set -> unmask).
+// RMSNorm] x layers -> LM head over the decode set -> unmask), plus the switched step, the
+// training form and the allocation-free entry point.
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>

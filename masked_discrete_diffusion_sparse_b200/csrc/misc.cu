@@ -5,7 +5,10 @@
 //   rmsnorm     — RMSNorm (optionally gathering the decode-set rows for the LM head);
 //   unmask      — confidence/argmax from the LM-head partials, top-n selection and the
 //                 scatter of committed tokens into the grid (Figure-3 example, Sec. 3.2);
-//   debug_mask  — the device step-causal predicate as a bitmap (test hook).
+//   debug_mask  — the device step-causal predicate as a bitmap (test hook);
+//   pack_switched — the row set of a step under the Table-6 speed switches;
+//   label bounds, tile lists — the training form's key skipping (SMDM_TRAIN_BOUND=1);
+//   qkv_finalize — RoPE and the K/V append after an additive QKV GEMM (SMDM_QKV_SPLIT=1).
 #include <climits>
 
 #include "misc.h"
