@@ -16,8 +16,9 @@ far larger than the 126 MB L2, so every run streams them from HBM; no L2 flush i
 N > 1 GPUs (torchrun): independent replicas, one sequence set per rank, no collective on the
 data path; value = all ranks' decoded tokens / the slowest rank's time.
 
-`--impl reference` times the fp64 CPU oracle on the host cores on a bounded sample of the same
-workload (prefill + the first sampling step) and prints the same JSON line.
+`--impl reference` times the fp64 CPU oracle, single-threaded, on a bounded sample of the same
+workload (the prefill and sampling steps 1, K/2 and K; the full run extrapolated by each step's
+algorithmic FLOPs) and prints the same JSON line.
 """
 from __future__ import annotations
 
@@ -248,31 +249,116 @@ class ClockSampler:
 # ----------------------------------------------------------------------------------------------
 
 class OracleSample:
-    """The fp64 oracle on the host cores, timed on a bounded sample of the workload: prefill of
-    sequence 0 plus its first sampling step.  Weights are generated once, outside the timing."""
+    """The fp64 oracle on the host cores, timed on a bounded sample of the workload.
+
+    A full fp64 run of the 4096-token workload is about 20 TFLOP, hours on one core, so the
+    sample is: the prefill, and the sampling steps 1, K/2 and K (K = 64: steps 1, 32 and 64).
+    A step k after the first runs on a state with that step's shape: a KV cache of the step's
+    length (the prefill's entries repeated, all visible, as every cached entry is to every row of
+    a real step), the tokens decoded at step k-1 as its new-cache rows and its own decode set.
+    The full run is extrapolated, not measured: prefill + sum over all K steps of each step's
+    algorithmic FLOPs (`forward_cost`) times the sampled steps' seconds per FLOP.  Weights and
+    states are built outside the timing.  `threads` pins the BLAS thread pool (1 = the
+    single-threaded oracle; numpy's elementwise work is single-threaded either way)."""
 
     def __init__(self, wl: synth.Workload):
         import oracle
-        self.oracle = oracle
+        self.o = oracle
         self.wl = wl
         self.om = oracle.Model(synth.make_weights(wl.model, wl.seed))
         self.prompt = synth.make_prompt(wl)
         self.plan = synth.make_plan(wl)
+        K = self.plan.n_steps
+        self.steps = sorted({1, max(1, K // 2), K})
+        self.components = ["prefill"] + [f"step {k}" for k in self.steps]
+        fw = list(run_forwards(wl, self.plan))
+        costs = [forward_cost(wl.model, *f)[1] for f in fw]
+        self.prefill_flops = costs[0] if wl.prompt_len else 0.0
+        self.step_flops = costs[1:] if wl.prompt_len else costs
+        self._base = None
+        self._states = {}
 
-    def run(self):
-        """Returns (seconds, decoded tokens, description, threads)."""
-        o, wl = self.oracle, self.wl
-        t0 = time.perf_counter()
-        st = o.Incremental(self.om, self.prompt, wl.gen_len)
-        qp = o.query_set(self.plan, st, 1)
-        lg = st.step_logits(qp)
-        tok, conf, rows = o.unmask(lg, o.POLICY_ALL if self.plan.kind == "order"
-                                   else o.POLICY_TOPN, self.plan.commit)
-        dt = time.perf_counter() - t0
-        n_dec = len(rows)
-        desc = (f"oracle prefill ({wl.prompt_len} rows) + sampling step 1 ({len(qp)} decode rows, "
-                f"{n_dec} tokens committed) of the same workload, fp64 numpy")
-        return dt, n_dec, desc, _blas_threads()
+    def _decode_sets(self, kmax):
+        """Positions decoded at steps 1..kmax (semi-AR: the first `commit` still-masked
+        positions of the step's block stand in for the most confident ones; only the counts
+        matter for the cost)."""
+        o, plan, wl = self.o, self.plan, self.wl
+        sim = type("S", (), {})()
+        sim.P, sim.grid = wl.prompt_len, np.full(wl.gen_len, -1, dtype=np.int64)
+        out = []
+        for j in range(1, kmax + 1):
+            qp = o.query_set(plan, sim, j)
+            c = qp if plan.kind == "order" else qp[:plan.commit]
+            sim.grid[c - wl.prompt_len - 1] = 0
+            out.append((qp, c))
+        return out
+
+    def _state_before(self, k):
+        import copy
+        o, wl = self.o, self.wl
+        if self._base is None:
+            self._base = o.Incremental(self.om, self.prompt, wl.gen_len)
+        base = self._base
+        sets = self._decode_sets(k)
+        P = wl.prompt_len
+        ctx = len(base.c_types) + sum(len(c) for _, c in sets[:max(0, k - 2)])
+        st = copy.copy(base)
+        reps = np.arange(ctx) % max(1, len(base.c_types))
+        st.k_cache = [kc[reps] for kc in base.k_cache]
+        st.v_cache = [vc[reps] for vc in base.v_cache]
+        st.c_types = np.zeros(ctx, dtype=np.int64)
+        st.c_labels = np.zeros(ctx, dtype=np.int64)
+        g = np.random.Generator(np.random.PCG64([wl.seed, 9100 + k]))
+        st.grid = np.full(wl.gen_len, -1, dtype=np.int64)
+        for _, c in sets[:k - 1]:
+            st.grid[c - P - 1] = g.integers(0, wl.model.vocab, len(c))
+        st.new_pos = sets[k - 2][1] if k >= 2 else np.zeros(0, dtype=np.int64)
+        st.step_k = k - 1
+        return st, sets[k - 1][0]
+
+    def time_component(self, c: str, threads: int) -> float:
+        """Seconds of one sample component ("prefill" or "step k") on `threads` BLAS threads."""
+        from threadpoolctl import threadpool_limits
+        o, wl = self.o, self.wl
+        if c != "prefill":
+            k = int(c.split()[1])
+            if k not in self._states:
+                self._states[k] = self._state_before(k)
+        with threadpool_limits(limits=threads, user_api="blas"):
+            t0 = time.perf_counter()
+            if c == "prefill":
+                o.Incremental(self.om, self.prompt, wl.gen_len)
+            else:
+                import copy
+                st, qp = self._states[k]
+                st = copy.copy(st)
+                lg = st.step_logits(qp)
+                o.unmask(lg, o.POLICY_ALL if self.plan.kind == "order" else o.POLICY_TOPN,
+                         self.plan.commit)
+            return time.perf_counter() - t0
+
+    def extrapolate(self, secs: dict) -> float:
+        """Full-run seconds from the component times: prefill + sum_k FLOPs_k x (sampled
+        seconds / sampled FLOPs)."""
+        t_steps = sum(secs[f"step {k}"] for k in self.steps)
+        f_steps = sum(self.step_flops[k - 1] for k in self.steps)
+        return secs["prefill"] + t_steps / f_steps * sum(self.step_flops)
+
+    def describe(self) -> str:
+        wl = self.wl
+        return (f"fp64 numpy oracle: prefill ({wl.prompt_len} rows) and sampling steps "
+                f"{', '.join(map(str, self.steps))} of {self.plan.n_steps} timed (steps after the "
+                f"first on a state with that step's cache length, new-cache rows and decode set); "
+                f"the full run of {wl.gen_len} decoded tokens is extrapolated by the algorithmic "
+                f"FLOPs of every step")
+
+    def run(self, threads: int) -> dict:
+        """Time every component once on `threads` BLAS threads; returns the full-run figures."""
+        secs = {c: self.time_component(c, threads) for c in self.components}
+        full = self.extrapolate(secs)
+        return {"value": self.wl.gen_len * self.wl.batch / full, "full_run_s": full,
+                "sampled_s": {c: round(v, 3) for c, v in secs.items()},
+                "sample_s": sum(secs.values())}
 
 
 def _cpu_model() -> str:
@@ -287,39 +373,40 @@ def _cpu_model() -> str:
     return "unknown"
 
 
-def _blas_threads() -> int:
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        if n:
-            return int(max(n))
-    except Exception:
-        pass
-    return os.cpu_count() or 1
-
-
 def run_reference(args, wl):
+    """The reference arm: the fp64 oracle, single-threaded, as it stands.  Each bench step times
+    one component of the oracle sample (prefill, step 1, step K/2, step K, in rotation); the
+    value is the extrapolated full-run rate from the mean time of each component over the timed
+    steps (a component the timed steps did not reach is timed once more after them)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    times = []
-    n_dec = 1
-    desc = ""
-    threads = 1
     sample = OracleSample(wl)
+    comps = sample.components
+    times = {c: [] for c in comps}
     for i in range(args.warmup + args.steps):
-        dt, n_dec, desc, threads = sample.run()
+        c = comps[i % len(comps)]
+        dt = sample.time_component(c, 1)
         if i >= args.warmup:
-            times.append(dt)
-    mean = sum(times) / len(times)
-    value = n_dec / mean          # the sample decodes one sequence
+            times[c].append(dt)
+    extra = [c for c in comps if not times[c]]
+    for c in extra:
+        times[c].append(sample.time_component(c, 1))
+    secs = {c: sum(v) / len(v) for c, v in times.items()}
+    full = sample.extrapolate(secs)
+    value = wl.gen_len * wl.batch / full
+    desc = sample.describe() + (f"; one component per bench step, {', '.join(extra)} timed once "
+                                f"after the timed steps" if extra else
+                                "; one component per bench step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": mean * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": full * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": describe(wl),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": desc, "cpu": _cpu_model()},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": desc, "extrapolated": True,
+                             "sampled_s": {c: round(v, 3) for c, v in secs.items()},
+                             "cpu": _cpu_model()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -812,9 +899,17 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         try:
-            dt, n_dec, desc, threads = OracleSample(wl).run()
-            line["cpu_baseline"] = {"value": n_dec / dt, "unit": UNIT, "cores": threads,
-                                    "kind": "oracle", "sample": desc, "seconds": dt,
+            sample = OracleSample(wl)
+            one = sample.run(1)
+            cores = os.cpu_count() or 1
+            allc = sample.run(cores)
+            line["cpu_baseline"] = {"value": one["value"], "unit": UNIT, "cores": 1,
+                                    "kind": "oracle", "sample": sample.describe(),
+                                    "extrapolated": True, "full_run_s": one["full_run_s"],
+                                    "sampled_s": one["sampled_s"],
+                                    "all_cores": {"value": allc["value"], "cores": cores,
+                                                  "full_run_s": allc["full_run_s"],
+                                                  "sampled_s": allc["sampled_s"]},
                                     "cpu": _cpu_model()}
         except MemoryError:
             line["cpu_baseline"] = None

@@ -571,30 +571,3 @@ def dense_step_logits(m: Model, prompt: np.ndarray, grid: np.ndarray) -> np.ndar
         x = m.attn_out(l, x, attention(q, k, v, vis))
         x = m.mlp(l, x)
     return m.logits(x[P:])
-
-
-def dense_generate(m: Model, prompt: np.ndarray, gen_len: int, plan: synth.Plan,
-                   max_steps: Optional[int] = None, teacher=None):
-    """Full dense-MDM sampling run with the same decode sets / commit policy as `generate`."""
-    P = len(prompt)
-    grid = np.full(gen_len, -1, dtype=np.int64)
-    recs = []
-    K = plan.n_steps if max_steps is None else min(max_steps, plan.n_steps)
-    for k in range(1, K + 1):
-        if plan.kind == "order":
-            qp = np.asarray(plan.query_positions(k), dtype=np.int64)
-        else:
-            lo, hi = synth.semiar_block(plan, P, k)
-            qp = semiar_queries(grid, P, lo, hi)
-        full = dense_step_logits(m, prompt, grid)
-        lg = full[qp - P - 1]
-        policy = POLICY_ALL if plan.kind == "order" else POLICY_TOPN
-        tok, conf, rows = unmask(lg, policy, plan.commit)
-        cpos, ctok = qp[rows], tok[rows]
-        if teacher is not None:
-            got = teacher(k, qp, lg, tok, conf, rows)
-            if got is not None:
-                cpos, ctok = got
-        grid[np.asarray(cpos) - P - 1] = ctok
-        recs.append(StepRecord(k, None, qp, lg, np.asarray(cpos), np.asarray(ctok)))
-    return grid, recs

@@ -4,7 +4,7 @@ from __future__ import annotations
 
 import math
 from dataclasses import dataclass
-from typing import List, Optional
+from typing import List, Optional, Sequence
 
 import numpy as np
 import torch
@@ -121,13 +121,22 @@ class Runner:
 
 
 def run_teacher_forced(r: Runner, max_steps: Optional[int] = None, check_rows: bool = True,
-                       logit_steps: Optional[int] = None):
+                       logit_steps: Optional[int] = None, late_steps: Sequence[int] = (),
+                       late_seqs: Optional[Sequence[int]] = None):
     """Sparse sampling, batch of r.batch sequences in one forward per step, checked against the
     oracle's incremental run per sequence after every step.  Returns a list of StepCheck.
 
     logit_steps: compare logits only for the first `logit_steps` steps (the oracle's fp64
     forward is the expensive part at full model size); later steps still check packing, the
-    commit rule and the scatter bit-exactly, with the oracle adopting the device's tokens."""
+    commit rule and the scatter bit-exactly, with the oracle adopting the device's tokens.
+
+    late_steps: steps after `logit_steps` whose logits are still compared, without running the
+    oracle's incremental form up to them: the device's logits of those steps are kept, and after
+    the run ONE training-form forward of the oracle per sequence (`oracle.trajectory` of the
+    teacher-forced run + `oracle.forward_stepcausal`) gives every late step's reference logits.
+    The two forms agree exactly (the method's invariant (b), pinned on the CPU), so this is the
+    same comparison at a fraction of the oracle's cost.  late_seqs: the sequences checked this
+    way (default: all)."""
     wl, P, Lg = r.wl, r.wl.prompt_len, r.wl.gen_len
     B = r.batch
     V = wl.model.vocab
@@ -149,6 +158,10 @@ def run_teacher_forced(r: Runner, max_steps: Optional[int] = None, check_rows: b
     n_steps = min(p.n_steps for p in r.plans)
     K = n_steps if max_steps is None else min(max_steps, n_steps)
     checks = []
+    late = set(int(k) for k in late_steps)
+    late_seqs = list(range(B)) if late_seqs is None else list(late_seqs)
+    history = [[] for _ in range(B)]      # per sequence: StepRecord of every step (no logits)
+    kept = {}                             # (seq, k) -> (device logits, device tokens)
     for k in range(1, K + 1):
         descs, qsets, packs = [], [], []
         for s in range(B):
@@ -205,6 +218,8 @@ def run_teacher_forced(r: Runner, max_steps: Optional[int] = None, check_rows: b
             else:
                 st.step_k += 1          # packing-only step: no fp64 forward
                 ref = None
+                if k in late and s in late_seqs:
+                    kept[(s, k)] = (lg[off:off + n_q].copy(), tks.copy())
             qidx = {int(p): j for j, p in enumerate(qp)}
             newly = np.nonzero((grid_before[s] < 0) & (grid_after[s] >= 0))[0]
             # committed positions in query-row order (the order of next step's new-cache rows)
@@ -227,6 +242,8 @@ def run_teacher_forced(r: Runner, max_steps: Optional[int] = None, check_rows: b
             untouched[newly] = False
             commit_ok &= bool(np.array_equal(grid_before[s][untouched], grid_after[s][untouched]))
             st.commit(cpos, ctok)   # teacher forcing: adopt the device's choice
+            history[s].append(oracle.StepRecord(k, None, np.asarray(qp, dtype=np.int64), None,
+                                                cpos.astype(np.int64), ctok.astype(np.int64)))
             ctx_exp[s] += prev_commit[s]
             prev_commit[s] = len(cpos)
             rows_exact &= r.model.smdm_context_length(s) == ctx_exp[s]
@@ -236,4 +253,43 @@ def run_teacher_forced(r: Runner, max_steps: Optional[int] = None, check_rows: b
         checks.append(StepCheck(k, err, rows_exact, tok_ok, commit_ok))
     for s in range(B):
         assert np.array_equal(grids[s].cpu().numpy(), states[s].grid)
+    for s in late_seqs:
+        steps = sorted(k for (q, k) in kept if q == s)
+        if not steps:
+            continue
+        ref = late_reference(r, s, history[s], steps)
+        for k in steps:
+            g, tks = kept[(s, k)]
+            c = checks[k - 1]
+            c.err = max(c.err, logit_err(g, ref[k]))
+            c.tok_ok = c.tok_ok and bool(token_admissible(tks, ref[k], r.tol).all())
+            if r.plans[s].kind != "order":
+                c.commit_ok = c.commit_ok and topn_commit_admissible(
+                    ref[k], [int(np.nonzero(history[s][k - 1].query_pos == p)[0][0])
+                             for p in history[s][k - 1].committed_pos],
+                    r.plans[s].commit, r.tol)
     return checks, grids, states
+
+
+def late_reference(r: Runner, s: int, history, steps) -> dict:
+    """Oracle logits of the given steps of sequence s, from one training-form forward over the
+    teacher-forced trajectory: block 0, the tokens committed at every step before the last one
+    asked for (clean, labelled by their step) and each asked step's decode set and tail rows
+    (labelled by the step).  Returns {k: logits [n_q][V]}."""
+    kmax = max(steps)
+    t = r.tasks[s] if r.tasks else None
+    ids, pos, types, labels, qrows = oracle.trajectory(
+        r.prompts[s], r.wl.model, r.wl.gen_len, history[:kmax], steps=steps,
+        preset_pos=None if t is None else t.preset_pos,
+        preset_tok=None if t is None else t.preset_tok)
+    # the tokens committed AT step kmax are not visible to any asked step: leave them out
+    keep = ~((types == oracle.CLEAN) & (labels == kmax))
+    idx = np.cumsum(keep) - 1
+    rows = np.concatenate([idx[qrows[k]] for k in steps])
+    lg = oracle.forward_stepcausal(r.om, ids[keep], pos[keep], types[keep], labels[keep], rows)
+    out, off = {}, 0
+    for k in steps:
+        n = len(qrows[k])
+        out[k] = lg[off:off + n]
+        off += n
+    return out

@@ -156,3 +156,26 @@ def test_batched_cost_counts_every_sequence():
         parts = [s[1 + k] for s in singles]
         assert R == sum(p[0] for p in parts) and q == sum(p[1] for p in parts)
         assert kv_sum == sum(p[2] for p in parts) and keys == sum(p[3] for p in parts)
+
+
+def test_oracle_sample_states_have_the_run_shapes():
+    """The CPU baseline times sampling steps on states built from the prefill (not on a full
+    run): each such state packs the real step's row count and has the real cache length, for an
+    order plan and a semi-AR plan; the sampled prefill and step times extrapolate to a full
+    run through the per-step FLOPs."""
+    b = _bench()
+    for name in ("tiny-f32-cos", "tiny-bf16-semiar"):
+        wl = synth.WORKLOADS[name]
+        s = b.OracleSample(wl)
+        plan = synth.make_plan(wl, 0)
+        shapes = b.step_shapes(wl, plan)
+        for k in s.steps:
+            st, qp = s._state_before(k)
+            R, q, ctx, n_new = shapes[k - 1]
+            assert st.ctx == ctx and len(qp) == q and st.pack(qp).n == R, (name, k)
+        out = s.run(1)
+        assert out["value"] > 0 and set(out["sampled_s"]) == set(s.components)
+        secs = out["sampled_s"]
+        # doubling every sampled time halves the extrapolated rate
+        assert abs(s.extrapolate({c: 2 * v for c, v in secs.items()})
+                   - 2 * s.extrapolate(secs)) < 1e-9 * s.extrapolate(secs) + 1e-12

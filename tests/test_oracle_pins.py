@@ -363,6 +363,37 @@ def test_reduces_to_standard_mdm_when_C_is_all_masks():
     np.testing.assert_allclose(sparse, dense, rtol=0, atol=1e-11)
 
 
+def test_dense_step_with_prompt_and_decoded_tokens():
+    """The dense comparator at P > 0 with part of the grid decoded: every one of the P + Lg rows
+    sees every other ("Key design 1": masks included, full attention), which is the training
+    form with every row a clean row of block 0.  Both must give the same generated-row logits;
+    dropping the prompt offset of the logit rows or the [MASK] ids of undecoded positions is
+    caught."""
+    m = tiny_model(n_reg=0)
+    g = np.random.Generator(np.random.PCG64(17))
+    P, Lg = 9, 14
+    prompt = g.integers(0, m.shape.vocab, P)
+    grid = np.full(Lg, -1, dtype=np.int64)
+    done = g.permutation(Lg)[:6]
+    grid[done] = g.integers(0, m.shape.vocab, len(done))
+    dense = oracle.dense_step_logits(m, prompt, grid)
+    assert dense.shape == (Lg, m.shape.vocab)
+    ids = np.concatenate([prompt, np.where(grid < 0, m.shape.mask_id, grid)])
+    n = P + Lg
+    ref = oracle.forward_stepcausal(m, ids, np.arange(1, n + 1), np.full(n, oracle.CLEAN),
+                                    np.zeros(n, dtype=np.int64), np.arange(P, n))
+    np.testing.assert_allclose(dense, ref, rtol=0, atol=1e-11)
+    # planted: logits of the first Lg rows instead of the generated rows
+    wrong = oracle.forward_stepcausal(m, ids, np.arange(1, n + 1), np.full(n, oracle.CLEAN),
+                                      np.zeros(n, dtype=np.int64), np.arange(Lg))
+    assert np.abs(wrong - dense).max() > 1e-3
+    # planted: undecoded positions carrying token 0 instead of [MASK]
+    ids0 = np.concatenate([prompt, np.where(grid < 0, 0, grid)])
+    wrong = oracle.forward_stepcausal(m, ids0, np.arange(1, n + 1), np.full(n, oracle.CLEAN),
+                                      np.zeros(n, dtype=np.int64), np.arange(P, n))
+    assert np.abs(wrong - dense).max() > 1e-3
+
+
 def test_semiar_run_structure():
     wl = synth.WORKLOADS["tiny-bf16-semiar"]
     m = oracle.Model(synth.make_weights(wl.model, wl.seed))

@@ -147,3 +147,32 @@ def test_planted_device_fault_is_caught(fault, field):
         assert bad.err > smdm_testlib.TOL[synth.F32]
     else:
         assert not getattr(bad, field)
+
+
+@pytest.mark.parametrize("name", ["tiny-f32-cos", "tiny-bf16-semiar"])
+def test_late_steps_reference_matches_the_incremental_logits(name):
+    """Late-step logits judged through one training-form forward of the oracle (no incremental
+    oracle run up to them): the faithful stand-in's incremental logits agree to fp64 rounding."""
+    r = _runner(name)
+    checks, _, _ = smdm_testlib.run_teacher_forced(r, logit_steps=1, late_steps=[3, 6])
+    assert len(checks) == r.plans[0].n_steps
+    for k in (3, 6):
+        c = checks[k - 1]
+        assert c.rows_exact and c.tok_ok and c.commit_ok and c.err < 1e-6, c
+
+
+def test_planted_late_step_logit_fault_is_caught():
+    r = _runner("tiny-f32-cos", "logits")
+    r.model.fault_step = 5
+    checks, _, _ = smdm_testlib.run_teacher_forced(r, logit_steps=1, late_steps=[4, 5])
+    assert checks[3].err < 1e-6
+    assert checks[4].err > smdm_testlib.TOL[synth.F32]
+
+
+def test_late_steps_with_a_bidirectional_task():
+    wl = synth.WORKLOADS["tiny-f32-cos"]
+    task = synth.make_bidir_task(wl, "inpaint")
+    r = _runner("tiny-f32-cos", tasks=[task])
+    checks, _, _ = smdm_testlib.run_teacher_forced(r, logit_steps=0, late_steps=[2, 4])
+    for k in (2, 4):
+        assert checks[k - 1].err < 1e-6 and checks[k - 1].tok_ok
