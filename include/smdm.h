@@ -233,7 +233,10 @@ smdm_status smdm_generate(smdm_handle* h, int batch, const int32_t* d_prompts, i
  * CLEAN label = the step they were decoded at) see clean rows with label <= theirs; MASK and
  * REG rows of label s see clean rows with label < s and the MASK/REG rows of label s.
  * Writes fp32 logits [n_rows][vocab] for the rows listed in d_logit_rows.  Does not touch any
- * sequence's generation state.  Any row order is allowed.  With the environment variable
+ * sequence's generation state.  Any row order is allowed.  Ids must lie in the embedding
+ * table, positions in [0, max_len + tail rows + 2), types in 0..3, labels in [0, n] and logit
+ * rows in [0, n): an id, position or logit row outside its range sets the device status word
+ * (SMDM_EDEVICE at the next smdm_device_status) and is replaced by 0.  With the environment variable
  * SMDM_TRAIN_BOUND=1 (bf16 models) the attention skips the 128-key tiles that hold no key
  * visible to a 128-row query tile (same result); rows laid out as prompt, clean tokens by
  * step, then each step's masks and registers skip most of them. */
@@ -291,7 +294,13 @@ smdm_status smdm_profile_end(smdm_handle* h, smdm_profile* out, cudaStream_t str
  *    attributes; make that first call before any stream capture.
  *  - Every call shares the array and overwrites it (the call clears it first); calls that
  *    overlap on the GPU — on different streams, or from different host threads — race.
- *    Serialise them.  Device-side status bits of this path are not reported. */
+ *    Serialise them.
+ *  - There is no status word to read back: SMDM_OK means the arguments passed the host checks
+ *    and the launches were accepted, NOT that the logits are valid.  A device-side wait that
+ *    timed out, or an id outside the embedding table or a position outside
+ *    [0, max_len + tail rows + 2) (replaced by 0 on the device), leaves wrong logits and no
+ *    error.  Check the inputs on the host before the call: ids and positions in those ranges,
+ *    types in 0..3, labels in [0, n], logit rows in [0, n). */
 smdm_status smdm_forward_stepcausal_noalloc(const smdm_config* cfg, const smdm_weights* w,
                                             const int32_t* d_ids, const int32_t* d_pos,
                                             const int32_t* d_type, const int32_t* d_label, int n,

@@ -234,7 +234,9 @@ int query_sms() {
   return n;
 }
 
-// extras: also the opt-in split-QKV buffer (not for the allocation-free path)
+// extras: the buffers of sampling sequences (KV caches, new-cache lists, prompt copies,
+// switched-step lists) and the opt-in split-QKV buffer; the allocation-free training form needs
+// none of them and lays its scratch out with extras = false.
 Layout make_layout(const smdm_config* c, int n_sms, bool extras = true) {
   Layout L{};
   const size_t es = c->dtype == SMDM_BF16 ? 2 : 4;
@@ -250,7 +252,7 @@ Layout make_layout(const smdm_config* c, int n_sms, bool extras = true) {
     off = align_up(off + bytes, 1024);
     return o;
   };
-  const size_t cache_elems = (size_t)c->max_batch * c->n_layers * H * L.cap * dh;
+  const size_t cache_elems = extras ? (size_t)c->max_batch * c->n_layers * H * L.cap * dh : 0;
   L.kc = take(cache_elems * es);
   L.vc = take(cache_elems * es);
   L.kscr = take(H * MR * dh * es);
@@ -277,8 +279,8 @@ Layout make_layout(const smdm_config* c, int n_sms, bool extras = true) {
   L.max_tiles = max_nt * rb;
   L.counters = take((size_t)L.max_tiles * 4);
   L.status = take(256);
-  L.newpos = take((size_t)c->max_batch * c->max_step_rows * 4);
-  L.prompts = take((size_t)c->max_batch * c->max_len * 4);
+  L.newpos = take(extras ? (size_t)c->max_batch * c->max_step_rows * 4 : 0);
+  L.prompts = take(extras ? (size_t)c->max_batch * c->max_len * 4 : 0);
   // split-KV partials for up to 16 key splits of a sampling step's rows
   const size_t step_rows = std::min((size_t)c->max_rows, (size_t)c->max_batch * c->max_step_rows);
   L.attn_part_bytes = 16 * step_rows * ((size_t)d * 4 + H * 8);
@@ -294,7 +296,7 @@ Layout make_layout(const smdm_config* c, int n_sms, bool extras = true) {
     L.has_qkv32 = true;
   }
   // switched steps: per sequence, decoded positions, their steps and the query marks
-  L.sw = take((size_t)c->max_batch * 3 * c->max_len * 4);
+  L.sw = take(extras ? (size_t)c->max_batch * 3 * c->max_len * 4 : 0);
   L.total = off + 1024;
   return L;
 }
@@ -1341,7 +1343,7 @@ smdm_status smdm_forward_stepcausal(smdm_handle* h, const int32_t* d_ids, const 
   a.rows = h->rows;
   a.status = h->status();
   { Launch lg_(h, SMDM_K_PACK, st); CK(launch_pack_linear(a, st)); }
-  { Launch lg_(h, SMDM_K_OTHER, st); CK(launch_gather_rows(d_logit_rows, n_rows, h->rows.qrow, st)); }
+  { Launch lg_(h, SMDM_K_OTHER, st); CK(launch_gather_rows(d_logit_rows, n_rows, n, h->rows.qrow, h->status(), st)); }
   const bool bound = h->bf16 && train_bound_enabled();
   int* tile_list = nullptr;
   int* tile_count = nullptr;
@@ -1485,6 +1487,12 @@ extern "C" smdm_status smdm_forward_stepcausal_noalloc(
   if (!d_ids || !d_pos || !d_type || !d_label || !d_logit_rows || !d_logits || n < 1 ||
       n_rows < 1)
     return SMDM_EINVAL;
+  // every layer's weights, as smdm_create checks them (a null norm gain would otherwise reach
+  // a kernel as a device address)
+  for (int l = 0; l < cfg->n_layers; ++l)
+    if (!w->attn_norm[l] || !w->w_qkv[l] || !w->w_o[l] || !w->mlp_norm[l] || !w->w_gate[l] ||
+        !w->w_up[l] || !w->w_down[l])
+      return SMDM_EINVAL;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= SMDM_NOALLOC_MAX_DEVICES)
     return SMDM_ECUDA;

@@ -461,11 +461,20 @@ __global__ void pack_linear_kernel(LinearPackArgs a) {
   a.rows.kvlen[i] = a.n;
 }
 
-__global__ void gather_rows_kernel(const int* __restrict__ src_rows, int n, int* __restrict__ qrow) {
+// Logit row j -> forward row src_rows[j]; a row index outside [0, n_fwd) is flagged in the
+// status word and replaced by row 0, so that no later kernel reads outside the activations.
+__global__ void gather_rows_kernel(const int* __restrict__ src_rows, int n, int n_fwd,
+                                   int* __restrict__ qrow, uint32_t* status) {
   griddep_launch();
   griddep_wait();   // launched with programmatic dependent launch
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) qrow[i] = src_rows[i];
+  if (i >= n) return;
+  int r = src_rows[i];
+  if (r < 0 || r >= n_fwd) {
+    atomicOr(status, kStatusBounds);
+    r = 0;
+  }
+  qrow[i] = r;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -695,9 +704,11 @@ cudaError_t launch_tile_lists(const int* type, const int* label, int n, int* scr
   return launch_pdl(tile_list_kernel, dim3(T), dim3(128), 0, st, 1, (const int4*)summary, T,
                     *lists, *counts);
 }
-cudaError_t launch_gather_rows(const int* src, int n, int* qrow, cudaStream_t st) {
+cudaError_t launch_gather_rows(const int* src, int n, int n_fwd, int* qrow, uint32_t* status,
+                               cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  return launch_pdl(gather_rows_kernel, dim3((n + 255) / 256), dim3(256), 0, st, 1, src, n, qrow);
+  return launch_pdl(gather_rows_kernel, dim3((n + 255) / 256), dim3(256), 0, st, 1, src, n, n_fwd, qrow,
+                    status);
 }
 template <typename T>
 cudaError_t launch_rmsnorm(const NormArgs& a, int rows, cudaStream_t st) {

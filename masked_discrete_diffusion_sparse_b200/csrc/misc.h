@@ -125,7 +125,8 @@ cudaError_t launch_pack_step(const PackArgs& a, cudaStream_t st);
 cudaError_t launch_qkv_finalize(const QkvFinalArgs& a, cudaStream_t st);
 cudaError_t launch_pack_linear(const LinearPackArgs& a, cudaStream_t st);
 cudaError_t launch_pack_switched(const PackSwArgs& a, cudaStream_t st);
-cudaError_t launch_gather_rows(const int* src, int n, int* qrow, cudaStream_t st);
+cudaError_t launch_gather_rows(const int* src, int n, int n_fwd, int* qrow, uint32_t* status,
+                               cudaStream_t st);
 // Training form: per-row key bounds of the step-causal rule into kvlen (see misc.cu);
 // scratch: 3 * (n + 1) + 1 ints.
 cudaError_t launch_label_bounds(const int* type, const int* label, int n, int* scratch,

@@ -117,6 +117,18 @@ def test_argument_errors_return_before_any_device_work():
     assert lib.smdm_forward_stepcausal_noalloc(ctypes.byref(bad), ctypes.byref(w), None, None,
                                                None, None, 4, None, 1, None, None) == \
         smdm.SMDM_ESHAPE
+    # one layer's norm gain missing: refused on the host, before any CUDA call (the pointers
+    # below are never dereferenced)
+    fake = ctypes.c_void_p(0x1000)
+    nl = good.n_layers
+    per_layer = {k: (ctypes.c_void_p * nl)(*([fake.value] * nl))
+                 for k in ("attn_norm", "w_qkv", "w_o", "mlp_norm", "w_gate", "w_up", "w_down")}
+    per_layer["mlp_norm"][nl - 1] = None
+    w2 = smdm.smdm_weights(fake, fake, fake, *[ctypes.cast(per_layer[k], smdm._PP) for k in
+                                              ("attn_norm", "w_qkv", "w_o", "mlp_norm",
+                                               "w_gate", "w_up", "w_down")])
+    assert lib.smdm_forward_stepcausal_noalloc(ctypes.byref(good), ctypes.byref(w2), fake, fake,
+                                               fake, fake, 4, fake, 1, fake, None) == E
 
 
 def test_capacities_that_overflow_32_bit_indices_are_rejected():

@@ -1,4 +1,5 @@
-"""The allocation-free training-form forward, checked against the handle-based one.
+"""The allocation-free training-form forward, checked against the handle-based one and the
+oracle.
 
 smdm_forward_stepcausal_noalloc is for callers that cannot allocate device memory when they
 need a forward (a frozen allocator, a plug-in that is only handed pointers): it keeps all its
@@ -12,7 +13,7 @@ import torch
 import masked_discrete_diffusion_sparse_b200 as smdm
 import oracle
 import synth
-from smdm_testlib import config_for, i32, logit_err, upload_weights, TOL
+from smdm_testlib import config_for, i32, logit_err, token_admissible, upload_weights, TOL
 
 pytestmark = pytest.mark.gpu
 
@@ -50,3 +51,9 @@ def test_noalloc_forward_matches_handle_forward_twice():
         assert np.isfinite(got).all(), f"call {call}: non-finite logits"
         err = logit_err(got, ref_np)
         assert err <= tol, f"call {call}: {err:.3g} > {tol}"
+        # and against the oracle's incremental logits of the same two steps (invariant (b)),
+        # with every row's argmax admissible under the lowest-id tie rule
+        inc = np.concatenate([rec.logits for rec in recs])
+        err_o = logit_err(got, inc)
+        assert err_o <= tol, f"call {call}: {err_o:.3g} > {tol} against the oracle"
+        assert token_admissible(np.argmax(got, axis=1), inc, tol).all()
