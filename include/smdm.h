@@ -202,7 +202,11 @@ smdm_status smdm_step_switched(smdm_handle* h, const smdm_step_desc* h_desc, int
 smdm_status smdm_dense_step(smdm_handle* h, const smdm_step_desc* h_desc, float* d_logits,
                             int32_t* d_tok, float* d_conf, cudaStream_t stream);
 
-/* A whole sampling plan. */
+/* A whole sampling plan: the decode set of every step (paperlayer.ai Sec. 3.2).  ORDER plans
+ * give the positions in decode order and the count per step: image generation and editing
+ * follow a pre-generated 2-D unmasking order with no confidence scores.  SEMIAR plans decode
+ * blocks one after another (left to right, or in any order for infilling), querying every
+ * masked position of the current block and committing the most confident. */
 typedef struct {
   int kind;                   /* SMDM_PLAN_ORDER or SMDM_PLAN_SEMIAR */
   int n_steps;                /* K */
@@ -217,7 +221,9 @@ typedef struct {
 } smdm_plan;
 
 /* Full generation of `batch` sequences (slots 0..batch-1) with the same P, Lgen and step
- * count: prefill, then K steps.  d_prompts: int32 [batch][P]; plans: host [batch];
+ * count: prefill (the prompt cached once, Sec. 3.2), then K sparse steps, each one forward
+ * over the step's new-cache rows, decode set and registers (the Figure-3 example,
+ * papernotes "a complete example"; paperlayer.ai Sec. 3.2 and Appendix 7.2).  d_prompts: int32 [batch][P]; plans: host [batch];
  * d_grids: int32 [batch][Lgen] (output).  mode SMDM_MODE_SPARSE batches the sequences into
  * one forward per step; SMDM_MODE_DENSE runs the dense comparator step per sequence.
  * The whole plan is checked on the host before any work (step sizes, their sum, P + Lgen
@@ -236,10 +242,10 @@ smdm_status smdm_generate(smdm_handle* h, int batch, const int32_t* d_prompts, i
  * sequence's generation state.  Any row order is allowed.  Ids must lie in the embedding
  * table, positions in [0, max_len + tail rows + 2), types in 0..3, labels in [0, n] and logit
  * rows in [0, n): an id, position or logit row outside its range sets the device status word
- * (SMDM_EDEVICE at the next smdm_device_status) and is replaced by 0.  With the environment variable
- * SMDM_TRAIN_BOUND=1 (bf16 models) the attention skips the 128-key tiles that hold no key
- * visible to a 128-row query tile (same result); rows laid out as prompt, clean tokens by
- * step, then each step's masks and registers skip most of them. */
+ * (SMDM_EDEVICE at the next smdm_device_status) and is replaced by 0.  For bf16 models the
+ * attention skips the 128-key tiles that hold no key visible to a 128-row query tile (same
+ * result): rows laid out as the prompt, the clean tokens by step, then each step's masks and
+ * registers skip most of them. */
 smdm_status smdm_forward_stepcausal(smdm_handle* h, const int32_t* d_ids, const int32_t* d_pos,
                                     const int32_t* d_type, const int32_t* d_label, int n,
                                     const int32_t* d_logit_rows, int n_rows, float* d_logits,
@@ -273,7 +279,9 @@ typedef struct {
 } smdm_profile;
 
 /* Start counting kernel launches.  timed != 0 also records a CUDA event pair around every
- * launch (do not enable while capturing a CUDA graph).  Resets the counters. */
+ * launch.  Resets the counters.  Timed profiling may stay on while a CUDA graph is captured:
+ * the event records become nodes of the graph, and smdm_profile_end reads the times of the
+ * graph's latest replay (replay it before calling smdm_profile_end). */
 smdm_status smdm_profile_begin(smdm_handle* h, int timed);
 /* Synchronise `stream`, fill *out and stop profiling. */
 smdm_status smdm_profile_end(smdm_handle* h, smdm_profile* out, cudaStream_t stream);

@@ -77,7 +77,8 @@ int encode_gateup_interleaved(CUtensorMap* m, const void* gate, const void* up, 
   return up_first ? 2 : 1;
 }
 
-// Head-tile view for the attention kernel: rows of `row_elems` bf16 split into 64-element
+// Head-tile view for the attention kernel (q, K and V are fp16): rows of `row_elems` split into
+// 64-element
 // (128-byte) chunks, dims {64, rows, row_elems / 64}, box {64, 128, nsub}: one copy brings a
 // 128-row tile of nsub chunks, landing as nsub swizzled [128][64] sub-tiles.
 bool encode_head_tiles(CUtensorMap* m, const void* base, uint64_t row_elems, uint64_t rows,
@@ -88,40 +89,25 @@ bool encode_head_tiles(CUtensorMap* m, const void* base, uint64_t row_elems, uin
   cuuint64_t strides[2] = {row_elems * 2, 128};
   cuuint32_t box[3] = {64, 128, nsub};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-// The same 3-D head-tile view with another box: {64, box_rows, box_sub} (the CTA-pair attention
-// loads half key tiles: 64 rows of all chunks, or 128 rows of one 64-wide chunk).
-bool encode_head_tiles_box(CUtensorMap* m, const void* base, uint64_t row_elems, uint64_t rows,
-                           uint32_t box_rows, uint32_t box_sub) {
-  EncodeTiledFn fn = get_encode_fn();
-  if (!fn || row_elems % 64) return false;
-  cuuint64_t dims[3] = {64, rows, row_elems / 64};
-  cuuint64_t strides[2] = {row_elems * 2, 128};
-  cuuint32_t box[3] = {64, box_rows, box_sub};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-// 2-D output map for the GEMM epilogue's TMA stores: `cols` x `rows` elements (bf16 or fp32),
-// row pitch `ld` elements, box {box_cols, 32}, no swizzle.
-bool encode_out(CUtensorMap* m, const void* base, bool f32, uint64_t cols, uint64_t rows,
-                uint64_t ld, uint32_t box_cols) {
+// 2-D output map for the GEMM epilogue's TMA stores: `cols` x `rows` elements (fp32, bf16 or,
+// for q, fp16), row pitch `ld` elements, box {box_cols, 32}, no swizzle.
+bool encode_out(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols,
+                uint64_t rows, uint64_t ld, uint32_t box_cols) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn || !base || rows == 0) return false;
+  const bool f32 = dt == CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const uint64_t es = f32 ? 4 : 2;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {ld * es};
   cuuint32_t box[2] = {box_cols, 32};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  CUresult r = fn(m, dt, 2,
                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -164,8 +150,6 @@ struct Layout {
   size_t kc, vc, kscr, vscr, x, h, q, ao, act, hq, pmax, psum, parg, rows, rope, partial,
       counters, status, newpos, prompts, aux, attn_part, lbound, tlist, sw, total;
   size_t attn_part_bytes;
-  size_t qkv32 = 0;          // split QKV: fp32 q|k|v rows [max rows][3 d] (when has_qkv32)
-  bool has_qkv32 = false;
   int cap, max_pos, n_vt, rt_max, max_tiles, n_sms;
   size_t partial_bytes;
 };
@@ -175,27 +159,6 @@ struct Layout {
 int tail_rows(const smdm_config* c) { return c->n_reg == SMDM_REG_LEN ? 1 : c->n_reg; }
 // Embedding rows: content ids, [MASK], [LEN] and the registers.
 int emb_rows(const smdm_config* c) { return c->vocab + 2 + std::max(c->n_reg, 0); }
-
-// Process-wide switch: SMDM_TRAIN_BOUND=1 gives the training-form attention per-row key
-// bounds (tiles past a query tile's last visible key are skipped; off by default).
-// Process-wide switch: SMDM_QKV_SPLIT=1 runs the QKV GEMM (bf16 models) with an additive fp32
-// epilogue spread over all SMs, and a finalize kernel for RoPE and the K/V append (off by
-// default).
-int qkv_split_enabled() {
-  static int v = [] {
-    const char* e = getenv("SMDM_QKV_SPLIT");
-    return (e && e[0] == '1') ? 1 : 0;
-  }();
-  return v;
-}
-
-int train_bound_enabled() {
-  static int v = [] {
-    const char* e = getenv("SMDM_TRAIN_BOUND");
-    return (e && e[0] == '1') ? 1 : 0;
-  }();
-  return v;
-}
 
 bool config_ok(const smdm_config* c, std::string* why) {
   auto fail = [&](const char* s) {
@@ -235,8 +198,8 @@ int query_sms() {
 }
 
 // extras: the buffers of sampling sequences (KV caches, new-cache lists, prompt copies,
-// switched-step lists) and the opt-in split-QKV buffer; the allocation-free training form needs
-// none of them and lays its scratch out with extras = false.
+// switched-step lists); the allocation-free training form needs none of them and lays its
+// scratch out with extras = false.
 Layout make_layout(const smdm_config* c, int n_sms, bool extras = true) {
   Layout L{};
   const size_t es = c->dtype == SMDM_BF16 ? 2 : 4;
@@ -291,10 +254,6 @@ Layout make_layout(const smdm_config* c, int n_sms, bool extras = true) {
     const size_t T = MR / 128;   // query / key tiles of a training-form forward
     L.tlist = take((5 * T + T * T) * 4);
   }
-  if (extras && qkv_split_enabled() && c->dtype == SMDM_BF16) {
-    L.qkv32 = take(MR * 3 * d * 4);
-    L.has_qkv32 = true;
-  }
   // switched steps: per sequence, decoded positions, their steps and the query marks
   L.sw = take(extras ? (size_t)c->max_batch * 3 * c->max_len * 4 : 0);
   L.total = off + 1024;
@@ -339,13 +298,6 @@ struct smdm_handle {
   std::vector<CUtensorMap> tm_qkv, tm_o, tm_gate, tm_up, tm_down, tm_gu;
   std::vector<int> gu_il;   // per layer: 0 two-box gate/up tiles, 1/2 interleaved (tm_gu)
   CUtensorMap tm_lm, tm_kc, tm_vc, tm_kscr, tm_vscr, tm_q;
-  // half-tile K / V views for the CTA-pair attention kernel (d_head 128); pair_maps false when
-  // they could not be encoded (the single-CTA kernel is used)
-  CUtensorMap tm_kc_h, tm_vc_h, tm_kscr_h, tm_vscr_h;
-  bool pair_maps = false;
-  // split QKV (SMDM_QKV_SPLIT=1): plain 2-D maps of W_qkv; qkv_split false when not in use
-  std::vector<CUtensorMap> tm_qkv_plain;
-  bool qkv_split = false;
   std::string err;
   SeqState seq[SMDM_MAX_BATCH];
   int last_rows = 0;
@@ -467,6 +419,9 @@ smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensor
                  const EpiParams& ep, cudaStream_t st, int a_interleave = 0, int sched = 0) {
   if (rows <= 0) return SMDM_OK;
   Launch lg(h, cls, st);
+  constexpr CUtensorMapDataType F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                                BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                                F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   if (h->bf16) {
     CUtensorMap tmB;
     const size_t MR = align_up((size_t)h->cfg.max_rows, 256);
@@ -476,14 +431,14 @@ smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensor
     CUtensorMap tmOut;
     bool ok_out = false;
     switch (ep.kind) {
-      case kEpiStore: ok_out = encode_out(&tmOut, ep.out, false, ep.n_valid, rows, ep.ld_out, 128); break;
-      case kEpiQKV: ok_out = encode_out(&tmOut, ep.q_out, false, ep.d_model, rows, ep.d_model, 128); break;
-      case kEpiSwiGLU: ok_out = encode_out(&tmOut, ep.act, false, ep.n_valid, rows, ep.ld_act, 64); break;
-      case kEpiResid: ok_out = encode_out(&tmOut, ep.x, true, ep.n_valid, rows, ep.ld_x, 128); break;
+      case kEpiStore: ok_out = encode_out(&tmOut, ep.out, BF16, ep.n_valid, rows, ep.ld_out, 128); break;
+      case kEpiQKV: ok_out = encode_out(&tmOut, ep.q_out, F16, ep.d_model, rows, ep.d_model, 128); break;
+      case kEpiSwiGLU: ok_out = encode_out(&tmOut, ep.act, BF16, ep.n_valid, rows, ep.ld_act, 64); break;
+      case kEpiResid: ok_out = encode_out(&tmOut, ep.x, F32, ep.n_valid, rows, ep.ld_x, 128); break;
       case kEpiLMHead:
         // without logits the map is never used: any valid fp32 map will do
-        ok_out = ep.logits ? encode_out(&tmOut, ep.logits, true, ep.n_valid, rows, ep.ld_logits, 128)
-                           : encode_out(&tmOut, ep.pmax, true, 128, 32, 128, 128);
+        ok_out = ep.logits ? encode_out(&tmOut, ep.logits, F32, ep.n_valid, rows, ep.ld_logits, 128)
+                           : encode_out(&tmOut, ep.pmax, F32, 128, 32, 128, 128);
         break;
     }
     if (!ok_out) return fail(h, SMDM_ECUDA, "cuTensorMapEncodeTiled failed for a GEMM output");
@@ -547,6 +502,10 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
   const Rows& rw = h->rows;
   h->last_rows = R;
 
+  // The RMSNorms run as their own kernel between the GEMMs.  (Run inside the consuming GEMM,
+  // every CTA of that GEMM would have to wait for the rows of every other CTA at a grid-wide
+  // barrier; the separate kernel's small CTAs sit beside the previous GEMM's and start the
+  // moment it completes, while the next GEMM is already streaming its first weight stages.)
   if ((s = norm(h, x, h->attn_norm[0], hb, nullptr, h->emb, rw.ids, R, st))) return s;
   for (int l = 0; l < c.n_layers; ++l) {
     EpiParams ep{};
@@ -563,35 +522,9 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
     ep.row_slot = rw.slot;
     ep.row_pos = rw.pos;
     ep.rope = h->at<float2>(h->L.rope);
-    if (h->qkv_split) {
-      // additive fp32 q|k|v over all SMs (stream-K, no fix-up), then RoPE + K/V append
-      EpiParams eq{};
-      eq.kind = kEpiResid;
-      eq.rows = R;
-      eq.n_valid = 3 * d;
-      eq.x = h->at<float>(h->L.qkv32);
-      eq.ld_x = 3 * d;
-      if ((s = gemm(h, SMDM_K_GEMM_QKV, &h->tm_qkv_plain[l], nullptr, h->w_qkv[l], nullptr, hb,
-                    d, 3 * d, R, 0, eq, st, 0, 2)))
-        return s;
-      QkvFinalArgs qa{};
-      qa.qkv32 = eq.x;
-      qa.rows = R;
-      qa.d = d;
-      qa.dh = c.d_head;
-      qa.layer = ep.layer;
-      qa.pos = rw.pos;
-      qa.seq = rw.seq;
-      qa.slot = rw.slot;
-      qa.rope = ep.rope;
-      qa.q_out = static_cast<__nv_bfloat16*>(q);
-      qa.kv = kv;
-      Launch lgq(h, SMDM_K_GEMM_QKV, st);
-      CK(launch_qkv_finalize(qa, st));
-    } else if ((s = gemm(h, SMDM_K_GEMM_QKV, h->bf16 ? &h->tm_qkv[l] : nullptr, nullptr,
-                         h->w_qkv[l], nullptr, hb, d, 3 * d, R, 0, ep, st, c.d_head))) {
+    if ((s = gemm(h, SMDM_K_GEMM_QKV, h->bf16 ? &h->tm_qkv[l] : nullptr, nullptr,
+                  h->w_qkv[l], nullptr, hb, d, 3 * d, R, 0, ep, st, c.d_head)))
       return s;
-    }
     // step-causal attention
     if (h->bf16) {
       AttnCall a{};
@@ -612,8 +545,6 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
       a.tmQ = &h->tm_q;
       a.tmK = f.scratch_kv ? &h->tm_kscr : &h->tm_kc;
       a.tmV = f.scratch_kv ? &h->tm_vscr : &h->tm_vc;
-      a.tmKh = h->pair_maps ? (f.scratch_kv ? &h->tm_kscr_h : &h->tm_kc_h) : nullptr;
-      a.tmVh = h->pair_maps ? (f.scratch_kv ? &h->tm_vscr_h : &h->tm_vc_h) : nullptr;
       a.cache_rows_per_seq = f.scratch_kv ? 0 : (long long)c.n_layers * c.n_heads * h->L.cap;
       a.cap = kv.cap;
       a.out = ao;
@@ -834,23 +765,6 @@ smdm_status smdm_create(const smdm_config* cfg, const smdm_weights* w, void* d_w
     ok &= encode_head_tiles(&h->tm_kscr, h->at<uint8_t>(h->L.kscr), dh, (uint64_t)H * MR, dh / 64);
     ok &= encode_head_tiles(&h->tm_vscr, h->at<uint8_t>(h->L.vscr), dh, (uint64_t)H * MR, dh / 64);
     ok &= encode_head_tiles(&h->tm_q, h->at<uint8_t>(h->L.q), d, MR, dh / 64);
-    if (h->L.has_qkv32) {
-      bool qs = true;
-      h->tm_qkv_plain.resize(nl);
-      for (int l = 0; l < nl; ++l)
-        qs &= encode_2d(&h->tm_qkv_plain[l], w->w_qkv[l], d, 3 * (uint64_t)d, (uint64_t)d * 2, 64,
-                        128);
-      h->qkv_split = qs;
-    }
-    if (dh == 128) {
-      bool pm = encode_head_tiles_box(&h->tm_kc_h, h->at<uint8_t>(h->L.kc), dh, cache_rows, 64, 2);
-      pm &= encode_head_tiles_box(&h->tm_vc_h, h->at<uint8_t>(h->L.vc), dh, cache_rows, 128, 1);
-      pm &= encode_head_tiles_box(&h->tm_kscr_h, h->at<uint8_t>(h->L.kscr), dh, (uint64_t)H * MR,
-                                  64, 2);
-      pm &= encode_head_tiles_box(&h->tm_vscr_h, h->at<uint8_t>(h->L.vscr), dh, (uint64_t)H * MR,
-                                  128, 1);
-      h->pair_maps = pm;
-    }
     if (!ok) {
       delete h;
       return SMDM_ECUDA;
@@ -1344,7 +1258,9 @@ smdm_status smdm_forward_stepcausal(smdm_handle* h, const int32_t* d_ids, const 
   a.status = h->status();
   { Launch lg_(h, SMDM_K_PACK, st); CK(launch_pack_linear(a, st)); }
   { Launch lg_(h, SMDM_K_OTHER, st); CK(launch_gather_rows(d_logit_rows, n_rows, n, h->rows.qrow, h->status(), st)); }
-  const bool bound = h->bf16 && train_bound_enabled();
+  // bf16 models: per-row key bounds and per-query-tile key-tile lists, so the attention skips
+  // the 128-key tiles in which no key is visible to a query tile
+  const bool bound = h->bf16;
   int* tile_list = nullptr;
   int* tile_count = nullptr;
   if (bound) {

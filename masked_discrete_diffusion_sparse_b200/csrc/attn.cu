@@ -11,13 +11,12 @@
 // bf16 path: one CTA per (sequence, 128-row query tile, head, key split).  Warp 0 streams Q and
 // K/V tiles with TMA (one copy per 128-row head tile), warp 1 issues tcgen05.mma (S = Q K^T
 // into one of two TMEM buffers, O += P V into a TMEM accumulator), warps 2-5 own one query row
-// per thread: masking, online softmax in the exp2 domain, P (bf16) into one of two swizzled
+// per thread: masking, online softmax in the exp2 domain, P (fp16) into one of two swizzled
 // shared-memory buffers, final 1/l scaling (or the unnormalised partial for the combine).  The running maximum is
 // only moved (and O rescaled) when it grows by more than 2^8, so most tiles skip the rescale;
 // the result is exact because numerator and denominator share the reference maximum.
-// Opt-in variants: attn_pair_kernel (d_head 128, SMDM_ATTN_PAIR=1) streams each key tile once
-// for two query tiles as M=256 MMAs of a CTA pair; the bounded label-mode instantiation
-// (SMDM_TRAIN_BOUND=1) scans only the key tiles listed for each query tile.
+// The bounded label-mode instantiation (the training form of bf16 models) scans only the key
+// tiles listed for each query tile.
 // fp32 path: one warp per (row, head), SIMT.
 #include <algorithm>
 
@@ -52,7 +51,7 @@ struct AttnDev {
 };
 
 SMDM_DEV void p_store_swizzled(uint8_t* P, int row, int key8, uint4 val) {
-  // P: [2 sub-tiles][128 rows][64 keys] bf16, 128-byte swizzle; key8 = 16-byte chunk 0..15
+  // P: [2 sub-tiles][128 rows][64 keys] fp16, 128-byte swizzle; key8 = 16-byte chunk 0..15
   const int sub = key8 >> 3, cc = key8 & 7;
   uint8_t* dst = P + sub * 16384 + row * 128 + ((cc ^ (row & 7)) << 4);
   *reinterpret_cast<uint4*>(dst) = val;
@@ -67,6 +66,11 @@ SMDM_DEV float ex2_approx(float x) {
 
 SMDM_DEV uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+SMDM_DEV uint32_t pack_f16x2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
@@ -88,8 +92,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = k_full + NS;
-  uint64_t* kv_empty = v_full + NS;
-  uint64_t* s_full = kv_empty + NS;   // [2]
+  uint64_t* k_empty = v_full + NS;    // [NS] K stage free: the S = Q K^T product completed
+  uint64_t* v_empty = k_empty + NS;   // [NS] V stage free: the P V product completed
+  uint64_t* s_full = v_empty + NS;    // [2]
   uint64_t* s_free = s_full + 2;      // [2]
   uint64_t* p_full = s_free + 2;      // [2] per P buffer: softmax warps wrote P(j), j & 1 == b
   uint64_t* pv_done = p_full + 2;     // [2] per P buffer: the P(j) V(j) product completed
@@ -137,7 +142,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -163,30 +169,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   griddep_wait();   // q, the KV cache and the row metadata come from earlier kernels
 
   if (warp == 0) {
-    if (lane == 0) {
-      const uint64_t pol_q = policy_evict_normal();
+    // Two producer lanes fill the K and the V ring independently: a K stage is free again as
+    // soon as its S = Q K^T product completes, a V stage only after the P V product, so K loads
+    // run ahead of V loads.
+    if (lane < 2) {
+      const bool is_k = lane == 0;
       const uint64_t pol_kv = policy_evict_last();
-      mbar_arrive_expect_tx(q_full, 128 * dh * 2);
-      tma_load_3d(Qs, &tmQ, q_full, 0, qrow0, h * nsub, pol_q);   // nsub [128][64] sub-tiles
+      const CUtensorMap* tm = is_k ? &tmK : &tmV;
+      uint64_t* full_b = is_k ? k_full : v_full;
+      uint64_t* empty_b = is_k ? k_empty : v_empty;
+      const int off = is_k ? a.k_off : a.v_off;
+      if (is_k) {
+        mbar_arrive_expect_tx(q_full, 128 * dh * 2);
+        tma_load_3d(Qs, &tmQ, q_full, 0, qrow0, h * nsub, policy_evict_normal());   // nsub [128][64] sub-tiles
+      }
+      auto tile_y = [&](int jj) {
+        const int kt = kBound ? tlist[j0 + jj] : (j0 + jj);
+        return (int)(cache_base + (long long)kt * 128);
+      };
       int stage = 0;
       uint32_t phase = 0;
       for (int j = 0; j < nkv; ++j) {
-        if (!mbar_wait(&kv_empty[stage], phase ^ 1, abort_flag, a.status)) break;
-        uint8_t* Ks = smem + a.k_off + stage * a.stage_bytes;
-        uint8_t* Vs = smem + a.v_off + stage * a.stage_bytes;
-        const int kt = kBound ? tlist[j0 + j] : (j0 + j);
-        const int y = (int)(cache_base + (long long)kt * 128);
-        mbar_arrive_expect_tx(&k_full[stage], 128 * dh * 2);
-        tma_load_3d(Ks, &tmK, &k_full[stage], 0, y, 0, pol_kv);
-        mbar_arrive_expect_tx(&v_full[stage], 128 * dh * 2);
-        tma_load_3d(Vs, &tmV, &v_full[stage], 0, y, 0, pol_kv);
+        if (!mbar_wait(&empty_b[stage], phase ^ 1, abort_flag, a.status)) break;
+        uint8_t* dst = smem + off + stage * a.stage_bytes;
+        mbar_arrive_expect_tx(&full_b[stage], 128 * dh * 2);
+        tma_load_3d(dst, tm, &full_b[stage], 0, tile_y(j), 0, pol_kv);
         if (++stage == NS) { stage = 0; phase ^= 1; }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16(128, 128, 0, 0);
-      const uint32_t idesc_o = idesc_bf16(128, dh, 0, 1);   // V is MN-major (dh contiguous)
+      const uint32_t idesc_s = idesc_f16(128, 128, 0, 0);   // q, K fp16
+      const uint32_t idesc_o = idesc_f16(128, dh, 0, 1);   // P, V fp16; V is MN-major
       const uint32_t q_addr = smem_u32(Qs), p_addr = smem_u32(Ps);
       bool ok = mbar_wait(q_full, 0, abort_flag, a.status);
       int stage = 0;
@@ -207,6 +221,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                      sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
           }
           umma_commit(&s_full[b]);
+          umma_commit(&k_empty[stage]);
           if (++stage == NS) { stage = 0; phase ^= 1; }
         }
         if (j >= 1) {
@@ -224,7 +239,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                      sdesc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
                      (jj > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(&kv_empty[pstage]);
+          umma_commit(&v_empty[pstage]);
           umma_commit(&pv_done[pb]);
           if (++pstage == NS) { pstage = 0; pphase ^= 1; }
         }
@@ -280,23 +295,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         mw[w] = bits;
       }
-      // pass 1: row maximum over the visible keys (two 64-column halves)
-      float mx = -INFINITY;
+      // pass 1: row maximum over the visible keys (two 64-column halves); eight independent
+      // partial maxima, so one warp per scheduler is not held up by a 128-long dependent chain
+      float mxp[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) mxp[t] = -INFINITY;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         float sv[64];
         tmem_ld64(tbase + lane_off + b * 128 + hh * 64, sv);
 #pragma unroll
         for (int c = 0; c < 64; ++c)
-          if ((mw[hh * 2 + (c >> 5)] >> (c & 31)) & 1u) mx = fmaxf(mx, sv[c]);
+          mxp[c & 7] = fmaxf(mxp[c & 7], ((mw[hh * 2 + (c >> 5)] >> (c & 31)) & 1u) ? sv[c] : -INFINITY);
       }
+      float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                       fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
       mx *= a.scale_log2;
       float alpha = 1.f;
       if (mx > m_ref + 8.f) {          // move the reference maximum (also the first time)
         alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mx);
         m_ref = mx;
       }
-      float rs = 0.f;
+      float rsp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // partial sums of P
       // P buffer j & 1 was last read by the P V product of tile j - 2
       if (j >= 2 && !mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, a.status)) break;
       const bool rescale = __any_sync(0xffffffffu, alpha != 1.f) && j >= 1;
@@ -313,7 +333,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_st16(t_o + lane_off + c * 16, o);
         }
       }
-      // pass 2: P = 2^(s*scale - m_ref) as bf16 into swizzled shared memory
+      // pass 2: P = 2^(s*scale - m_ref) as fp16 into swizzled shared memory
       const float mref_eff = (m_ref == -INFINITY) ? 0.f : m_ref;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
@@ -327,19 +347,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int c = c8 * 8 + t;
             const bool vis = (mw[hh * 2 + (c >> 5)] >> (c & 31)) & 1u;
             p[t] = vis ? ex2_approx(fmaf(sv[c], a.scale_log2, -mref_eff)) : 0.f;
-            rs += p[t];
+            rsp[t] += p[t];
           }
           uint4 pk;
-          pk.x = pack_bf16x2(p[0], p[1]);
-          pk.y = pack_bf16x2(p[2], p[3]);
-          pk.z = pack_bf16x2(p[4], p[5]);
-          pk.w = pack_bf16x2(p[6], p[7]);
+          pk.x = pack_f16x2(p[0], p[1]);
+          pk.y = pack_f16x2(p[2], p[3]);
+          pk.z = pack_f16x2(p[4], p[5]);
+          pk.w = pack_f16x2(p[6], p[7]);
           p_store_swizzled(Ps + (j & 1) * (128 * 128 * 2), em, hh * 8 + c8, pk);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[b]);
+      const float rs = ((rsp[0] + rsp[1]) + (rsp[2] + rsp[3])) + ((rsp[4] + rsp[5]) + (rsp[6] + rsp[7]));
       l = l * alpha + rs;
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
@@ -394,344 +415,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
-  }
-}
-
-// ------------------------------------------------------------------------------------------
-// CTA-pair variant (d_head 128): a cluster of two CTAs takes two query tiles of the same
-// (sequence, head, key split) and streams each key tile once for both.  S = Q K^T and
-// O += P V run as M=256 MMAs (cta_group::2) issued by the first CTA: A rows (Q, P) come from
-// each CTA's own tile; B rows are split between the pair, so a CTA loads half of the key
-// tile's K (64 keys x 128 dims) and half of its V (128 keys x 64 dims) — 32 KB per key tile
-// instead of 64 KB, and twice as many key tiles in flight for the same shared memory.  Each
-// CTA's TMEM receives its own rows of S and O; its softmax warps work as in attn_tc_kernel.
-// Barriers that collect both CTAs (both Q tiles, both halves of a key tile, the softmax
-// warps' S-free and P-ready signals) live in the first CTA; MMA completions are multicast to
-// both.  No TMA load uses multicast.
-// ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(kAttnThreads, 1)
-    attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
-                     const __grid_constant__ CUtensorMap tmKh,
-                     const __grid_constant__ CUtensorMap tmVh, const AttnDev a) {
-  constexpr int dh = 128;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  uint8_t* Qs = smem + a.q_off;
-  uint8_t* Ps = smem + a.p_off;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.bar_off);
-  const int NS = a.nstages;
-  uint64_t* q_full = bars;            // first CTA: both query tiles
-  uint64_t* k_full = bars + 1;        // [NS] first CTA: both K halves
-  uint64_t* v_full = k_full + NS;     // [NS] first CTA: both V halves
-  uint64_t* kv_empty = v_full + NS;   // [NS] both CTAs (multicast MMA completion)
-  uint64_t* s_full = kv_empty + NS;   // [2] both CTAs (multicast)
-  uint64_t* s_free = s_full + 2;      // [2] first CTA: 4 softmax warps x 2 CTAs
-  uint64_t* p_full = s_free + 2;      // [2] first CTA: 4 softmax warps x 2 CTAs
-  uint64_t* pv_done = p_full + 2;     // [2] both CTAs (multicast)
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pv_done + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const bool leader = rank == 0;
-  const int cl = blockIdx.x >> 1;                    // cluster = (query-tile pair, key split)
-  const int pblk = cl / a.nsplit, split = cl % a.nsplit, h = blockIdx.y;
-  int si = 0;
-  while (si + 1 < a.n_seg && a.seg[si + 1].tile0 <= pblk) ++si;
-  const AttnSeg sg = a.seg[si];
-  const int tile = 2 * (pblk - sg.tile0) + (int)rank;
-  const int qrow0 = sg.row0 + tile * 128;            // first forward row of this CTA's tile
-  const int nq = max(0, min(128, sg.rows - tile * 128));   // 0: the pair's second tile is empty
-  const int nkeys = sg.nkeys;
-  const int nkv_all = (nkeys + 127) / 128;
-  const int j0 = split * nkv_all / a.nsplit, j1 = (split + 1) * nkv_all / a.nsplit;
-  const int nkv = j1 - j0;
-  if (nkv == 0) {                                    // both CTAs of the pair take this path
-    griddep_launch();
-    griddep_wait();
-    for (int r = threadIdx.x; r < nq; r += blockDim.x) {
-      float* ml = a.part_ml + (((size_t)split * a.rows_total + qrow0 + r) * a.H + h) * 2;
-      ml[0] = -INFINITY;
-      ml[1] = 0.f;
-    }
-    return;
-  }
-  const long long cache_base = (long long)sg.seq * a.cache_rows_per_seq +
-                               ((long long)a.layer * a.H + h) * a.cap;
-  auto lead = [&](uint64_t* bar) { return mapa_shared(smem_u32(bar), 0); };
-
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 8);
-      mbar_init(&p_full[b], 8);
-      mbar_init(&pv_done[b], 1);
-    }
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  // both CTAs' barriers are initialised before any cross-CTA signal and before the pair's
-  // joint TMEM allocation (one warp in each CTA)
-  cluster_sync_all();
-  if (warp == 1) {
-    tmem_alloc_pair(tmem_holder, 512);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tbase = *tmem_holder;
-  const uint32_t t_o = tbase + 256;   // O accumulator columns [256, 384)
-  griddep_launch();
-  griddep_wait();   // q, the KV cache and the row metadata come from earlier kernels
-
-  if (warp == 0) {
-    if (lane == 0) {
-      const uint64_t pol_q = policy_evict_normal();
-      const uint64_t pol_kv = policy_evict_last();
-      if (leader) mbar_arrive_expect_tx(q_full, 2 * 128 * dh * 2);
-      tma_load_3d_pair(Qs, &tmQ, lead(q_full), 0, qrow0, h * 2, pol_q);
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int j = 0; j < nkv; ++j) {
-        if (!mbar_wait(&kv_empty[stage], phase ^ 1, abort_flag, a.status)) { ok = false; break; }
-        uint8_t* Ks = smem + a.k_off + stage * a.stage_bytes;
-        uint8_t* Vs = smem + a.v_off + stage * a.stage_bytes;
-        const int y = (int)(cache_base + (long long)(j0 + j) * 128);
-        if (leader) mbar_arrive_expect_tx(&k_full[stage], 2 * 64 * dh * 2);
-        tma_load_3d_pair(Ks, &tmKh, lead(&k_full[stage]), 0, y + (int)rank * 64, 0, pol_kv);
-        if (leader) mbar_arrive_expect_tx(&v_full[stage], 2 * 128 * 64 * 2);
-        tma_load_3d_pair(Vs, &tmVh, lead(&v_full[stage]), 0, y, (int)rank, pol_kv);
-        if (++stage == NS) { stage = 0; phase ^= 1; }
-      }
-      // the pair's last MMA completions land in this CTA's barriers: see them all before exit
-      for (int i = nkv; ok && i < nkv + NS; ++i)
-        if (!mbar_wait(&kv_empty[i % NS], (uint32_t)(((i / NS) & 1) ^ 1), abort_flag, a.status))
-          break;
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && leader) {
-      const uint32_t idesc_s = idesc_bf16(256, 128, 0, 0);   // two query tiles x 128 keys
-      const uint32_t idesc_o = idesc_bf16(256, dh, 0, 1);    // V is MN-major (dh contiguous)
-      const uint32_t q_addr = smem_u32(Qs), p_addr = smem_u32(Ps);
-      bool ok = mbar_wait(q_full, 0, abort_flag, a.status);
-      int stage = 0;
-      uint32_t phase = 0;
-      int pstage = 0;
-      uint32_t pphase = 0;
-      for (int j = 0; ok && j <= nkv; ++j) {
-        if (j < nkv) {
-          const int b = j & 1;
-          if (!mbar_wait(&k_full[stage], phase, abort_flag, a.status)) break;
-          if (!mbar_wait(&s_free[b], ((j >> 1) & 1) ^ 1, abort_flag, a.status)) break;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(smem + a.k_off + stage * a.stage_bytes);
-#pragma unroll
-          for (int kk = 0; kk < dh / 16; ++kk) {
-            // Q: two [128 rows][64 dims] sub-tiles; K half: two [64 keys][64 dims] sub-tiles
-            const uint32_t qoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
-            umma_f16_pair(tbase + b * 128, sdesc_sw128(q_addr + qoff, 16, 1024),
-                          sdesc_sw128(k_addr + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-          }
-          umma_commit_pair(&s_full[b]);
-          if (++stage == NS) { stage = 0; phase ^= 1; }
-        }
-        if (j >= 1) {
-          // O += P_{j-1} V_{j-1}; this CTA's V half is [128 keys][64 dims], one sub-tile
-          const int jj = j - 1;
-          const int pb = jj & 1;
-          if (!mbar_wait(&p_full[pb], (jj >> 1) & 1, abort_flag, a.status)) break;
-          if (!mbar_wait(&v_full[pstage], pphase, abort_flag, a.status)) break;
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(smem + a.v_off + pstage * a.stage_bytes);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_f16_pair(t_o, sdesc_sw128(p_addr + pb * (128 * 128 * 2) + aoff, 16, 1024),
-                          sdesc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
-                          (jj > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit_pair(&kv_empty[pstage]);
-          umma_commit_pair(&pv_done[pb]);
-          if (++pstage == NS) { pstage = 0; pphase ^= 1; }
-        }
-      }
-    }
-  } else {
-    // Softmax warps (both CTAs): thread owns query row em of this CTA's tile; S-free and
-    // P-ready arrivals go to the first CTA's barriers.
-    const int q4 = warp & 3;
-    const int em = q4 * 32 + lane;
-    const int row = qrow0 + em;
-    const bool valid = em < nq;
-    const uint32_t lane_off = uint32_t(q4 * 32) << 16;
-    int kv_lim = 0, tq = 0, lq = 0;
-    if (valid) {
-      if (a.mode == 0) kv_lim = a.kvlen[row];
-      else { tq = a.type[row]; lq = a.label[row]; kv_lim = nkeys; }
-    }
-    float m_ref = -INFINITY, l = 0.f;
-    const bool warp_any = __any_sync(0xffffffffu, valid);
-    for (int j = 0; j < nkv; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag, a.status)) break;
-      tc_fence_after();
-      if (!warp_any) {
-        // no valid query row in this warp: keep the barrier protocol, skip the math
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(lead(&s_free[b]));
-        // keep in step with the other warps: signal P(j) only once P buffer j & 1 is free, so
-        // that no arrival can land in a later phase of p_full (its P rows are never read back)
-        if (j >= 2 && !mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, a.status)) break;
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(lead(&p_full[j & 1]));
-        continue;
-      }
-      const int key0 = (j0 + j) * 128;
-      // visibility of the 128 keys as four 32-bit masks (registers only, no local arrays)
-      uint32_t mw[4];
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const int kb = key0 + w * 32;
-        uint32_t bits;
-        if (a.mode == 0) {
-          const int n_ok = min(max(kv_lim - kb, 0), 32);
-          bits = n_ok == 32 ? 0xffffffffu : ((1u << n_ok) - 1u);
-        } else {
-          bits = 0;
-          for (int bb = 0; bb < 32; ++bb) {
-            const int key = kb + bb;
-            if (key < kv_lim && step_causal_allowed(tq, lq, a.type[key], a.label[key]))
-              bits |= 1u << bb;
-          }
-        }
-        mw[w] = bits;
-      }
-      // pass 1: row maximum over the visible keys (two 64-column halves)
-      float mx = -INFINITY;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float sv[64];
-        tmem_ld64(tbase + lane_off + b * 128 + hh * 64, sv);
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if ((mw[hh * 2 + (c >> 5)] >> (c & 31)) & 1u) mx = fmaxf(mx, sv[c]);
-      }
-      mx *= a.scale_log2;
-      float alpha = 1.f;
-      if (mx > m_ref + 8.f) {          // move the reference maximum (also the first time)
-        alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mx);
-        m_ref = mx;
-      }
-      float rs = 0.f;
-      // P buffer j & 1 was last read by the P V product of tile j - 2
-      if (j >= 2 && !mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, a.status)) break;
-      const bool rescale = __any_sync(0xffffffffu, alpha != 1.f) && j >= 1;
-      // rescaling O needs the product of tile j - 1 accumulated first
-      if (rescale && !mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status))
-        break;
-      tc_fence_after();
-      if (rescale) {
-        for (int c = 0; c < dh / 16; ++c) {
-          float o[16];
-          tmem_ld16(t_o + lane_off + c * 16, o);
-#pragma unroll
-          for (int t = 0; t < 16; ++t) o[t] *= alpha;
-          tmem_st16(t_o + lane_off + c * 16, o);
-        }
-      }
-      // pass 2: P = 2^(s*scale - m_ref) as bf16 into swizzled shared memory
-      const float mref_eff = (m_ref == -INFINITY) ? 0.f : m_ref;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float sv[64];
-        tmem_ld64(tbase + lane_off + b * 128 + hh * 64, sv);
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          float p[8];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const int c = c8 * 8 + t;
-            const bool vis = (mw[hh * 2 + (c >> 5)] >> (c & 31)) & 1u;
-            p[t] = vis ? ex2_approx(fmaf(sv[c], a.scale_log2, -mref_eff)) : 0.f;
-            rs += p[t];
-          }
-          uint4 pk;
-          pk.x = pack_bf16x2(p[0], p[1]);
-          pk.y = pack_bf16x2(p[2], p[3]);
-          pk.z = pack_bf16x2(p[4], p[5]);
-          pk.w = pack_bf16x2(p[6], p[7]);
-          p_store_swizzled(Ps + (j & 1) * (128 * 128 * 2), em, hh * 8 + c8, pk);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead(&s_free[b]));
-      l = l * alpha + rs;
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead(&p_full[j & 1]));
-    }
-    // Final: O / l (one split), or the unnormalised partial for the combine pass.
-    if (nkv > 0 && mbar_wait(&pv_done[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1, abort_flag, a.status)) {
-      tc_fence_after();
-      if (a.nsplit == 1) {
-        const float inv = (l > 0.f) ? 1.f / l : 0.f;
-        __nv_bfloat16* out =
-            reinterpret_cast<__nv_bfloat16*>(a.out) + (size_t)row * a.d_model + h * dh;
-        for (int c = 0; c < dh / 16; ++c) {
-          float o[16];
-          tmem_ld16(t_o + lane_off + c * 16, o);
-          if (valid) {
-            uint4 w0, w1;
-            w0.x = pack_bf16x2(o[0] * inv, o[1] * inv);
-            w0.y = pack_bf16x2(o[2] * inv, o[3] * inv);
-            w0.z = pack_bf16x2(o[4] * inv, o[5] * inv);
-            w0.w = pack_bf16x2(o[6] * inv, o[7] * inv);
-            w1.x = pack_bf16x2(o[8] * inv, o[9] * inv);
-            w1.y = pack_bf16x2(o[10] * inv, o[11] * inv);
-            w1.z = pack_bf16x2(o[12] * inv, o[13] * inv);
-            w1.w = pack_bf16x2(o[14] * inv, o[15] * inv);
-            reinterpret_cast<uint4*>(out + c * 16)[0] = w0;
-            reinterpret_cast<uint4*>(out + c * 16)[1] = w1;
-          }
-        }
-      } else {
-        float* po = a.part_o + ((size_t)split * a.rows_total + row) * a.d_model + h * dh;
-        for (int c = 0; c < dh / 16; ++c) {
-          float o[16];
-          tmem_ld16(t_o + lane_off + c * 16, o);
-          if (valid) {
-#pragma unroll
-            for (int t = 0; t < 16; t += 4)
-              *reinterpret_cast<float4*>(po + c * 16 + t) = make_float4(o[t], o[t + 1], o[t + 2], o[t + 3]);
-          }
-        }
-        if (valid) {
-          float* ml = a.part_ml + (((size_t)split * a.rows_total + row) * a.H + h) * 2;
-          ml[0] = m_ref;
-          ml[1] = l;
-        }
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();   // the peer is done with our TMEM, shared memory and barriers
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc_pair(tbase, 512);
   }
 }
 
@@ -822,41 +505,12 @@ static int attn_layout(int dh, AttnDev& d) {
   d.stage_bytes = kv_bytes;
   const int budget = 227 * 1024 - 1024 - 256;
   int ns = (budget - q_bytes - p_bytes) / (2 * kv_bytes);
-  if (ns > 4) ns = 4;
+  if (ns > 4) ns = 4;   // the 256-byte barrier area holds 1 + 4 * 4 + 8 barriers
   d.nstages = ns;
   d.k_off = q_bytes + p_bytes;
   d.v_off = d.k_off + ns * kv_bytes;
   d.bar_off = d.v_off + ns * kv_bytes;
   return d.bar_off + 256 + 1024;
-}
-
-// Shared memory of the pair kernel: Q, two P buffers, then NS stages of a K half and a V half
-// (16 KB each).
-static int attn_pair_layout(AttnDev& d) {
-  const int q_bytes = 128 * 128 * 2;
-  const int p_bytes = 2 * 128 * 128 * 2;
-  const int half = 64 * 128 * 2;
-  d.q_off = 0;
-  d.p_off = q_bytes;
-  d.stage_bytes = half;
-  const int budget = 227 * 1024 - 1024 - 256;
-  int ns = (budget - q_bytes - p_bytes) / (2 * half);
-  if (ns > 4) ns = 4;   // the 256-byte barrier area holds 1 + 3 * 4 + 8 barriers
-  d.nstages = ns;
-  d.k_off = q_bytes + p_bytes;
-  d.v_off = d.k_off + ns * half;
-  d.bar_off = d.v_off + ns * half;
-  return d.bar_off + 256 + 1024;
-}
-
-// Process-wide switch for the CTA-pair attention kernel: SMDM_ATTN_PAIR=1 selects it for
-// d_head 128 (off by default).
-static int attn_pair_enabled() {
-  static int v = [] {
-    const char* e = getenv("SMDM_ATTN_PAIR");
-    return (e && e[0] == '1') ? 1 : 0;
-  }();
-  return v;
 }
 
 cudaError_t attn_tc_set_smem_attr() {
@@ -924,26 +578,7 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t stream) {
   d.part_o = c.part_o;
   d.part_ml = c.part_o ? c.part_o + (size_t)d.nsplit * c.rows_total * c.d_model : nullptr;
   cudaError_t e;
-  if (attn_pair_enabled() && c.dh == 128 && c.tmKh && c.tmVh) {
-    // clusters of two query tiles of the same segment (the last one of an odd count is empty)
-    int npb = 0;
-    for (int s = 0; s < c.n_seg; ++s) {
-      d.seg[s].tile0 = npb;
-      npb += ((c.seg[s].rows + 127) / 128 + 1) / 2;
-    }
-    static bool attr_set[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_set[dev]) {
-      e = cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               227 * 1024);
-      if (e != cudaSuccess) return e;
-      attr_set[dev] = true;
-    }
-    const int smem = attn_pair_layout(d);
-    e = launch_pdl(attn_pair_kernel, dim3((unsigned)(npb * d.nsplit * 2), c.H),
-                   dim3(kAttnThreads), smem, stream, 2, *c.tmQ, *c.tmKh, *c.tmVh, d);
-  } else if (c.bound && c.mode == 1 && c.tile_list && c.tile_count && c.n_seg == 1 &&
+  if (c.bound && c.mode == 1 && c.tile_list && c.tile_count && c.n_seg == 1 &&
              c.seg[0].row0 == 0) {
     // label mode with per-row key bounds (training form over step-grouped rows)
     static bool attr_set[64];
@@ -1001,8 +636,6 @@ cudaError_t launch_attn_simt(const T* q, T* out, const KVAddr& kv, const AttnSim
 
 template cudaError_t launch_attn_simt<float>(const float*, float*, const KVAddr&,
                                              const AttnSimtArgs&, cudaStream_t);
-template cudaError_t launch_attn_simt<__nv_bfloat16>(const __nv_bfloat16*, __nv_bfloat16*,
-                                                     const KVAddr&, const AttnSimtArgs&,
-                                                     cudaStream_t);
+
 
 }  // namespace smdm

@@ -31,11 +31,6 @@ struct AttnCall {
   const CUtensorMap* tmQ;   // q [rows][d_model] bf16 (chunk coordinate = head * d_head / 64)
   const CUtensorMap* tmK;   // K cache [cache rows][d_head] bf16
   const CUtensorMap* tmV;   // V cache, same layout
-  // CTA-pair kernel (d_head 128, SMDM_ATTN_PAIR=1): the same K / V views with half-tile boxes,
-  // {64, 64, 2} over K (64 keys) and {64, 128, 1} over V (one 64-wide dimension chunk);
-  // nullptr keeps the single-CTA kernel
-  const CUtensorMap* tmKh;
-  const CUtensorMap* tmVh;
   long long cache_rows_per_seq;
   int cap;
   void* out;                // [rows][d_model] bf16

@@ -6,7 +6,9 @@
 // 128-row MMA M dimension.  Work is split stream-K style: the (tile, 64-wide K chunk) units are
 // divided evenly over one CTA (or 2-CTA cluster) per SM (pair); tiles cut between CTAs are
 // finished by whichever CTA contributes last (fp32 partials in L2-resident scratch, summed in a
-// fixed order so results are deterministic).  When the tile count is a large enough share of
+// fixed order).  The residual epilogues (O-proj, down) instead add every segment into the fp32
+// residual stream with TMA reduce-add as it finishes, so their sums — and through them the
+// logits — are not bit-reproducible from run to run.  When the tile count is a large enough share of
 // the grid, every CTA takes one whole tile instead.  Warp roles: warps 0 and 6 issue TMA loads
 // (alternate pipeline stages), warp 1 owns TMEM and issues tcgen05.mma (straight-line per
 // 64-wide K chunk), warps 2-5 drain the accumulator through the fused epilogue, which writes
@@ -620,27 +622,10 @@ int gemm_tc_box_rows(int rows, int pair) {
   return (RT > 256 ? RT / 2 : RT) / pair;
 }
 
-// Process-wide switch for the CTA-pair path: SMDM_GEMM_PAIR=0 forces single CTAs.
-static int pair_enabled() {
-  static int v = [] {
-    const char* e = getenv("SMDM_GEMM_PAIR");
-    return (e && e[0] == '0') ? 0 : 1;
-  }();
-  return v;
-}
-
 // Whole tiles (one CTA per tile, no split-K fix-up) when the tile count is at least this
 // percentage of the grid (measured on the 4096-token run: 40 puts the QKV GEMM (96 tiles) and
-// the LM head (64 tiles) on whole tiles, the O / down GEMMs (32 tiles) on stream-K);
-// SMDM_WHOLE_TILE_MIN overrides it.
-static int whole_tile_min_pct() {
-  static int v = [] {
-    const char* e = getenv("SMDM_WHOLE_TILE_MIN");
-    const int x = e ? atoi(e) : 40;
-    return (x >= 1 && x <= 100) ? x : 40;
-  }();
-  return v;
-}
+// the LM head (64 tiles) on whole tiles, the O / down GEMMs (32 tiles) on stream-K).
+constexpr int kWholeTileMinPct = 40;
 
 int gemm_tc_pair(int n_out, int swiglu, int rows, int epi_kind) {
   (void)rows;
@@ -649,7 +634,7 @@ int gemm_tc_pair(int n_out, int swiglu, int rows, int epi_kind) {
   // (O, down) and LM-head GEMMs a little.  The pair covers two adjacent 128-row weight tiles, so
   // their count must be even.
   const bool wants = epi_kind == kEpiQKV || epi_kind == kEpiSwiGLU;
-  return (pair_enabled() && wants && n_tiles % 2 == 0) ? 2 : 1;
+  return (wants && n_tiles % 2 == 0) ? 2 : 1;
 }
 
 static int pow2_ceil(int x) {
@@ -737,7 +722,7 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream) {
     if (mc > 0 && G > mc) G = mc;
   }
   const long long tiles_total = (long long)pair_tiles * g.row_blocks;
-  const int whole_pct = whole_tile_min_pct();
+  const int whole_pct = kWholeTileMinPct;
   if (c.sched == 1 ? tiles_total <= G
                    : c.sched == 0 && tiles_total <= G && tiles_total * 100 >= G * whole_pct)
     G = tiles_total;

@@ -14,15 +14,6 @@
 
 namespace smdm {
 
-// Programmatic dependent launch for the library's kernels (SMDM_PDL=0 turns it off).
-inline bool pdl_enabled() {
-  static const bool on = [] {
-    const char* e = getenv("SMDM_PDL");
-    return !(e && e[0] == '0');
-  }();
-  return on;
-}
-
 // Launch `kern` with programmatic stream serialization (and a cluster of cluster_x CTAs when
 // > 1).  Every kernel launched this way calls griddep_wait() before it touches data that an
 // earlier kernel produces or consumes.
@@ -37,7 +28,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   cudaLaunchAttribute attr[2];
   unsigned n = 0;
   attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[n].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
   ++n;
   if (cluster_x > 1) {
     attr[n].id = cudaLaunchAttributeClusterDimension;
@@ -326,29 +317,30 @@ SMDM_DEV void epilogue_block(const EpiParams& p, const CUtensorMap* tm_out, floa
       if (region < 2) {
         const int ih = (f % dh) % half;
         const bool second = (m & 1) != 0;
+        // all 32 rows' (cos, sin) requested before any is used: one memory round trip per
+        // block instead of one per few rows
+        float2 cs[32];
 #pragma unroll
-        for (int g = 0; g < 32; g += 8) {
-          float2 cs[8];
+        for (int j = 0; j < 32; ++j) {
+          const int jj = min(j, nrows - 1);
+          cs[j] = __ldg(p.rope + (size_t)meta_pos[r0 + jj - meta_r0] * half + ih);
+        }
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int jj = min(g + j, nrows - 1);
-            cs[j] = __ldg(p.rope + (size_t)meta_pos[r0 + jj - meta_r0] * half + ih);
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float a = v[g + j];
-            const float b = __shfl_xor_sync(0xffffffffu, a, 1);
-            v[g + j] = second ? (b * cs[j].y + a * cs[j].x) : (a * cs[j].x - b * cs[j].y);
-          }
+        for (int j = 0; j < 32; ++j) {
+          const float a = v[j];
+          const float b = __shfl_xor_sync(0xffffffffu, a, 1);
+          v[j] = second ? (b * cs[j].y + a * cs[j].x) : (a * cs[j].x - b * cs[j].y);
         }
       }
-      // q: [32 rows][128 features]; k / v: [head within the tile][32 rows][d_head]
-      __nv_bfloat16* Sb = reinterpret_cast<__nv_bfloat16*>(buf);
+      // q: [32 rows][128 features]; k / v: [head within the tile][32 rows][d_head].  The
+      // attention operands are fp16 (3 more mantissa bits than bf16; the attention's MMAs take
+      // both of their operands in fp16)
+      __half* Sb = reinterpret_cast<__half*>(buf);
       const int hh = f / dh;
-      __nv_bfloat16* dst = (region == 0) ? Sb + f : Sb + hh * 32 * dh + (f - hh * dh);
+      __half* dst = (region == 0) ? Sb + f : Sb + hh * 32 * dh + (f - hh * dh);
       const int stride = (region == 0) ? 128 : dh;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) dst[j * stride] = __float2bfloat16_rn(v[j]);
+      for (int j = 0; j < 32; ++j) dst[j * stride] = __float2half_rn(v[j]);
       publish();
       if (et == 0) {
         if (region == 0) {
@@ -356,8 +348,7 @@ SMDM_DEV void epilogue_block(const EpiParams& p, const CUtensorMap* tm_out, floa
         } else {
           const long long base = (long long)p.layer * p.kv.layer_stride +
                                  (long long)(nn0 / dh) * p.kv.head_stride;
-          __nv_bfloat16* cache =
-              reinterpret_cast<__nv_bfloat16*>(region == 1 ? p.kv.k : p.kv.v) + base;
+          __half* cache = reinterpret_cast<__half*>(region == 1 ? p.kv.k : p.kv.v) + base;
           int j0 = 0;
           while (j0 < nrows) {
             const long long o0 = meta_kv[r0 + j0 - meta_r0];
@@ -447,37 +438,42 @@ SMDM_DEV void epilogue_block(const EpiParams& p, const CUtensorMap* tm_out, floa
         tma_store_2d(tm_out, S, n0, r0);
         bulk_commit();
       }
-      const int warp = et >> 5, lane = et & 31;
+      // Per row: max, first argmax and sum exp(l - max) over the tile's 128 columns.  Four
+      // threads per row (et >> 2 = row, et & 3 = a quarter of 32 columns), each walking its
+      // columns in an order rotated by et so that the 32 lanes of a warp read 32 different
+      // banks; ties in the maximum go to the lowest column, whatever the walking order.
       const int vt = n0 >> 7;
-      for (int j = warp * 8; j < min(warp * 8 + 8, nrows); ++j) {
-        float best = -INFINITY;
-        int arg = 0x7fffffff;
+      const int j = et >> 2, qq = et & 3;
+      const float* Srow = S + j * 128 + qq * 32;
+      const int col0 = n0 + qq * 32;
+      float best = -INFINITY;
+      int arg = 0x7fffffff;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int ff = lane + 32 * u;
-          const float x = (n0 + ff < p.n_valid) ? S[j * 128 + ff] : -INFINITY;
-          if (x > best) { best = x; arg = n0 + ff; }
-        }
+      for (int c = 0; c < 32; ++c) {
+        const int cc = (c + et) & 31;
+        const float x = (col0 + cc < p.n_valid) ? Srow[cc] : -INFINITY;
+        if (x > best || (x == best && col0 + cc < arg)) { best = x; arg = col0 + cc; }
+      }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-          const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
-          if (ob > best || (ob == best && oa < arg)) { best = ob; arg = oa; }
-        }
-        float sum = 0.f;
+      for (int o = 1; o <= 2; o <<= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
+        if (ob > best || (ob == best && oa < arg)) { best = ob; arg = oa; }
+      }
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int ff = lane + 32 * u;
-          if (n0 + ff < p.n_valid) sum += __expf(S[j * 128 + ff] - best);
-        }
+      for (int c = 0; c < 32; ++c) {
+        const int cc = (c + et) & 31;
+        if (col0 + cc < p.n_valid) s4[c & 3] += __expf(Srow[cc] - best);
+      }
+      float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (lane == 0) {
-          const size_t idx = (size_t)(r0 + j) * p.n_vt + vt;
-          p.pmax[idx] = best;
-          p.parg[idx] = arg;
-          p.psum[idx] = sum;
-        }
+      for (int o = 1; o <= 2; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if (qq == 0 && j < nrows) {
+        const size_t idx = (size_t)(r0 + j) * p.n_vt + vt;
+        p.pmax[idx] = best;
+        p.parg[idx] = arg;
+        p.psum[idx] = sum;
       }
       break;
     }

@@ -1,14 +1,13 @@
 // The non-contraction kernels of the sparse sampling step:
 //   pack        — builds the step's sparse row set (Sparse-LaViDa Sec. 3.1 / Appendix 7.2:
 //                 |A| + |C| + m rows) and the per-row attention prefixes;
-//   embed_norm  — embedding gather into the fp32 residual stream + first RMSNorm;
-//   rmsnorm     — RMSNorm (optionally gathering the decode-set rows for the LM head);
+//   rmsnorm     — RMSNorm of fp32 models (optionally gathering the embedding rows first, or the
+//                 decode-set rows for the LM head); bf16 models run it inside the GEMMs;
 //   unmask      — confidence/argmax from the LM-head partials, top-n selection and the
 //                 scatter of committed tokens into the grid (Figure-3 example, Sec. 3.2);
 //   debug_mask  — the device step-causal predicate as a bitmap (test hook);
 //   pack_switched — the row set of a step under the Table-6 speed switches;
-//   label bounds, tile lists — the training form's key skipping (SMDM_TRAIN_BOUND=1);
-//   qkv_finalize — RoPE and the K/V append after an additive QKV GEMM (SMDM_QKV_SPLIT=1).
+//   label bounds, tile lists — the training form's key skipping (bf16 models);
 #include <climits>
 
 #include "misc.h"
@@ -363,48 +362,6 @@ __global__ void tile_list_kernel(const int4* summary, int n_tiles, int* lists, i
 }
 
 // ------------------------------------------------------------------------------------------
-// Split-QKV finalize (SMDM_QKV_SPLIT=1).  The QKV GEMM ran with an additive fp32 epilogue into
-// qkv32 [rows][3d] (split segments of a tile add independently, so every tile's K range can be
-// spread over all SMs with no fix-up).  Here: the rotary embedding of q and k (rotate-half
-// pairs (i, i + dh/2) of each head, angles of the row's position), q to q_out, k and v to the
-// cache rows at (seq, layer, head, slot), all bf16; the fp32 rows are zeroed for the next
-// launch.  One CTA per row.
-// ------------------------------------------------------------------------------------------
-__global__ void qkv_finalize_kernel(QkvFinalArgs a) {
-  griddep_launch();
-  griddep_wait();   // launched with programmatic dependent launch
-  const int r = blockIdx.x;
-  const int d = a.d, dh = a.dh, half = dh >> 1;
-  float* row = a.qkv32 + (size_t)r * 3 * d;
-  const float2* cs = a.rope + (size_t)a.pos[r] * half;
-  const long long kvoff = (long long)a.seq[r] * a.kv.seq_stride +
-                          (long long)a.layer * a.kv.layer_stride + (long long)a.slot[r] * dh;
-  __nv_bfloat16* q = a.q_out + (size_t)r * d;
-  __nv_bfloat16* K = reinterpret_cast<__nv_bfloat16*>(a.kv.k) + kvoff;
-  __nv_bfloat16* V = reinterpret_cast<__nv_bfloat16*>(a.kv.v) + kvoff;
-  for (int t = threadIdx.x; t < d / 2; t += blockDim.x) {   // rotary pairs of q and k
-    const int h = t / half, i = t - h * half;
-    const int f1 = h * dh + i, f2 = f1 + half;
-    const float2 c = cs[i];
-    const float q1 = row[f1], q2 = row[f2];
-    q[f1] = __float2bfloat16_rn(q1 * c.x - q2 * c.y);
-    q[f2] = __float2bfloat16_rn(q2 * c.x + q1 * c.y);
-    const float k1 = row[d + f1], k2 = row[d + f2];
-    __nv_bfloat16* Kh = K + (long long)h * a.kv.head_stride;
-    Kh[i] = __float2bfloat16_rn(k1 * c.x - k2 * c.y);
-    Kh[i + half] = __float2bfloat16_rn(k2 * c.x + k1 * c.y);
-    row[f1] = 0.f;
-    row[f2] = 0.f;
-    row[d + f1] = 0.f;
-    row[d + f2] = 0.f;
-  }
-  for (int f = threadIdx.x; f < d; f += blockDim.x) {      // v
-    const int h = f / dh;
-    V[(long long)h * a.kv.head_stride + (f - h * dh)] = __float2bfloat16_rn(row[2 * d + f]);
-    row[2 * d + f] = 0.f;
-  }
-}
-
 // Prefill / dense / training-form rows: one thread per row.
 __global__ void pack_linear_kernel(LinearPackArgs a) {
   griddep_launch();
@@ -564,6 +521,7 @@ __global__ void unmask_kernel(UnmaskArgs a) {
   int* tok = reinterpret_cast<int*>(sh + s.n_q);        // [n_q]
   int* commit = tok + s.n_q;                            // [n_q]
   const int lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  constexpr int kPer = 8;   // partials per lane held in registers (n_vt <= 256: V <= 32768)
   for (int j = threadIdx.x >> 5; j < s.n_q; j += nwarps) {
     const int lr = s.dense ? (a.qpos_of[s.qbase + j] - s.P - 1) : (s.qbase + j);
     const float* pm = a.pmax + (size_t)(s.lbase + lr) * a.n_vt;
@@ -571,18 +529,44 @@ __global__ void unmask_kernel(UnmaskArgs a) {
     const int* pa = a.parg + (size_t)(s.lbase + lr) * a.n_vt;
     float M = -INFINITY;
     int arg = 0x7fffffff;
-    for (int t = lane; t < a.n_vt; t += 32) {
-      const float v = pm[t];
-      if (v > M) { M = v; arg = pa[t]; }   // tiles in vocab order: first max = lowest id
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float oM = __shfl_xor_sync(0xffffffffu, M, o);
-      const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
-      if (oM > M || (oM == M && oa < arg)) { M = oM; arg = oa; }
-    }
     float z = 0.f;
-    for (int t = lane; t < a.n_vt; t += 32) z += ps[t] * __expf(pm[t] - M);
+    if (a.n_vt <= 32 * kPer) {
+      // every load of the row in flight at once (one round trip), then reduce from registers
+      float vm[kPer], vs[kPer];
+      int va[kPer];
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int t = lane + 32 * i;
+        const bool ok = t < a.n_vt;
+        vm[i] = ok ? pm[t] : -INFINITY;
+        vs[i] = ok ? ps[t] : 0.f;
+        va[i] = ok ? pa[t] : 0x7fffffff;
+      }
+#pragma unroll
+      for (int i = 0; i < kPer; ++i)
+        if (vm[i] > M) { M = vm[i]; arg = va[i]; }   // tiles in vocab order: first max = lowest id
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float oM = __shfl_xor_sync(0xffffffffu, M, o);
+        const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
+        if (oM > M || (oM == M && oa < arg)) { M = oM; arg = oa; }
+      }
+#pragma unroll
+      for (int i = 0; i < kPer; ++i)
+        if (vs[i] > 0.f) z += vs[i] * __expf(vm[i] - M);
+    } else {
+      for (int t = lane; t < a.n_vt; t += 32) {
+        const float v = pm[t];
+        if (v > M) { M = v; arg = pa[t]; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float oM = __shfl_xor_sync(0xffffffffu, M, o);
+        const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
+        if (oM > M || (oM == M && oa < arg)) { M = oM; arg = oa; }
+      }
+      for (int t = lane; t < a.n_vt; t += 32) z += ps[t] * __expf(pm[t] - M);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
     if (lane == 0) {
@@ -662,10 +646,6 @@ __global__ void fill_i32_kernel(int* p, int n, int v) {
 cudaError_t launch_pack_step(const PackArgs& a, cudaStream_t st) {
   return launch_pdl(pack_step_kernel, dim3(a.n_seq), dim3(256), 0, st, 1, a);
 }
-cudaError_t launch_qkv_finalize(const QkvFinalArgs& a, cudaStream_t st) {
-  if (a.rows <= 0) return cudaSuccess;
-  return launch_pdl(qkv_finalize_kernel, dim3(a.rows), dim3(256), 0, st, 1, a);
-}
 cudaError_t launch_pack_linear(const LinearPackArgs& a, cudaStream_t st) {
   if (a.n <= 0) return cudaSuccess;
   return launch_pdl(pack_linear_kernel, dim3((a.n + 255) / 256), dim3(256), 0, st, 1, a);
@@ -720,7 +700,7 @@ template cudaError_t launch_rmsnorm<__nv_bfloat16>(const NormArgs&, int, cudaStr
 
 cudaError_t launch_unmask(const UnmaskArgs& a, int max_nq, cudaStream_t st) {
   const size_t smem = (size_t)max_nq * 12;
-  return launch_pdl(unmask_kernel, dim3(a.n_seq), dim3(512), smem, st, 1, a);
+  return launch_pdl(unmask_kernel, dim3(a.n_seq), dim3(1024), smem, st, 1, a);
 }
 cudaError_t launch_debug_mask(const int* type, const int* label, int n, uint32_t* bitmap,
                               cudaStream_t st) {

@@ -108,21 +108,8 @@ struct UnmaskArgs {
   uint32_t* status;
 };
 
-// Split-QKV finalize (see misc.cu): rotary embedding, bf16 q and K/V cache rows from the fp32
-// q|k|v rows an additive QKV GEMM summed; the fp32 rows are zeroed for the next launch.
-struct QkvFinalArgs {
-  float* qkv32;          // [rows][3 d] fp32, zero again on return
-  int rows, d, dh, layer;
-  const int* pos;
-  const int* seq;
-  const int* slot;
-  const float2* rope;    // [pos][dh / 2] (cos, sin)
-  __nv_bfloat16* q_out;  // [rows][d]
-  KVAddr kv;
-};
 
 cudaError_t launch_pack_step(const PackArgs& a, cudaStream_t st);
-cudaError_t launch_qkv_finalize(const QkvFinalArgs& a, cudaStream_t st);
 cudaError_t launch_pack_linear(const LinearPackArgs& a, cudaStream_t st);
 cudaError_t launch_pack_switched(const PackSwArgs& a, cudaStream_t st);
 cudaError_t launch_gather_rows(const int* src, int n, int n_fwd, int* qrow, uint32_t* status,

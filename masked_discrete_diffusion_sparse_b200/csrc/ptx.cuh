@@ -4,6 +4,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -344,6 +345,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, 
   return (1u << 4)                          // D format: f32
          | (1u << 7)                        // A format: bf16
          | (1u << 10)                       // B format: bf16
+         | (uint32_t(a_mn_major) << 15)     // A major
+         | (uint32_t(b_mn_major) << 16)     // B major
+         | (uint32_t(N >> 3) << 17)         // N / 8
+         | (uint32_t(M >> 4) << 24);        // M / 16
+}
+
+// Instruction descriptor: f16 x f16 -> f32 (A and B formats 0 = f16), M x N, majors as above.
+// Both operands of one MMA always share their type.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn_major, int b_mn_major) {
+  return (1u << 4)                          // D format: f32
          | (uint32_t(a_mn_major) << 15)     // A major
          | (uint32_t(b_mn_major) << 16)     // B major
          | (uint32_t(N >> 3) << 17)         // N / 8

@@ -9,5 +9,3 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
     config.addinivalue_line("markers", "slow: long-running oracle comparison")
-    config.addinivalue_line("markers", "gpu_pending: GPU parity case not yet run on a B200 "
-                            "(select with -m gpu_pending)")

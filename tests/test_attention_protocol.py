@@ -111,7 +111,7 @@ def mma_issuer(nkv, NS, sim, q_full, k_full, v_full, s_free, p_full, on_s, on_pv
             b = j & 1
             yield lambda s=stage, p=phase: k_full[s].done(p)
             yield lambda b=b, j=j: s_free[b].done(((j >> 1) & 1) ^ 1)
-            sim.events.append(lambda b=b: on_s(b))
+            sim.events.append(lambda b=b, s=stage: on_s(b, s))
             stage += 1
             if stage == NS:
                 stage, phase = 0, phase ^ 1
@@ -127,36 +127,43 @@ def mma_issuer(nkv, NS, sim, q_full, k_full, v_full, s_free, p_full, on_s, on_pv
 
 
 def single(nkv, NS, rescale, sim, rnd):
+    """attn_tc_kernel: separate K and V rings, each filled by its own producer lane; a K stage
+    is released by the commit after S = Q K^T, a V stage by the commit after P V."""
     q_full = sim.bar("q_full")
     k_full = [sim.bar(("k", s)) for s in range(NS)]
     v_full = [sim.bar(("v", s)) for s in range(NS)]
-    kv_empty = [sim.bar(("empty", s)) for s in range(NS)]
+    k_empty = [sim.bar(("k_empty", s)) for s in range(NS)]
+    v_empty = [sim.bar(("v_empty", s)) for s in range(NS)]
     s_full = [sim.bar(("s_full", b)) for b in range(2)]
     s_free = [sim.bar(("s_free", b), 4) for b in range(2)]
     p_full = [sim.bar(("p_full", b), 4) for b in range(2)]
     pv_done = [sim.bar(("pv_done", b)) for b in range(2)]
 
-    def producer():
-        q_full.expect_tx(Q_BYTES)
-        sim.events.append(lambda: q_full.complete_tx(Q_BYTES))
+    def producer(full, empty, nbytes, with_q):
+        if with_q:
+            q_full.expect_tx(Q_BYTES)
+            sim.events.append(lambda: q_full.complete_tx(Q_BYTES))
         stage = phase = 0
         for _ in range(nkv):
-            yield lambda s=stage, p=phase ^ 1: kv_empty[s].done(p)
-            k_full[stage].expect_tx(K_BYTES)
-            sim.events.append(lambda s=stage: k_full[s].complete_tx(K_BYTES))
-            v_full[stage].expect_tx(V_BYTES)
-            sim.events.append(lambda s=stage: v_full[s].complete_tx(V_BYTES))
+            yield lambda s=stage, p=phase ^ 1: empty[s].done(p)
+            full[stage].expect_tx(nbytes)
+            sim.events.append(lambda s=stage: full[s].complete_tx(nbytes))
             stage += 1
             if stage == NS:
                 stage, phase = 0, phase ^ 1
 
+    def on_s(b, s):
+        s_full[b].arrive()
+        k_empty[s].arrive()
+
     def on_pv(s, pb):
-        kv_empty[s].arrive()
+        v_empty[s].arrive()
         pv_done[pb].arrive()
 
-    actors = {"producer": producer(),
+    actors = {"producer_k": producer(k_full, k_empty, K_BYTES, True),
+              "producer_v": producer(v_full, v_empty, V_BYTES, False),
               "mma": mma_issuer(nkv, NS, sim, q_full, k_full, v_full, s_free, p_full,
-                                lambda b: s_full[b].arrive(), on_pv)}
+                                on_s, on_pv)}
     for w in range(4):
         actors[f"softmax{w}"] = softmax_warp(nkv, s_full, pv_done, s_free, p_full, rescale, rnd)
     return actors
@@ -193,7 +200,7 @@ def pair(nkv, NS, rescale, sim, rnd, s_free_count=8):
         for i in range(nkv, nkv + NS):
             yield lambda i=i: kv_empty[rank][i % NS].done(((i // NS) & 1) ^ 1)
 
-    def on_s(b):
+    def on_s(b, s):
         for r in (0, 1):
             s_full[r][b].arrive()
 

@@ -111,7 +111,7 @@ def test_sparse_run_register_count(n_reg):
         r.close()
 
 
-@pytest.mark.parametrize("kind", ["inpaint", "infill"])
+@pytest.mark.parametrize("kind", ["inpaint", "outpaint", "infill"])
 def test_bidirectional_task_run(kind):
     """Bidirectional tasks (given generation tokens as block-0 clean rows, cached with the
     prompt): teacher-forced sampling of the remaining positions against the oracle."""

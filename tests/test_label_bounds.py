@@ -1,6 +1,6 @@
 """Per-row key bounds of the training form (CPU).
 
-With SMDM_TRAIN_BOUND=1 the library gives every row of a step-labelled forward the bound
+For bf16 models the library gives every row of a step-labelled forward the bound
 kvlen = 1 + the last key index it may see, from per-label last indices and their prefix maximum
 (misc.cu, label bounds).  This restates that rule and checks it against the step-causal
 predicate of the oracle for random row sets in any order, and shows that a trajectory's rows,
