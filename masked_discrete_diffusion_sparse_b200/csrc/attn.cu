@@ -11,8 +11,9 @@
 // bf16 path: one CTA per (sequence, 128-row query tile, head, key split).  Warp 0 streams Q and
 // K/V tiles with TMA (one copy per 128-row head tile), warp 1 issues tcgen05.mma (S = Q K^T
 // into one of two TMEM buffers, O += P V into a TMEM accumulator), warps 2-5 own one query row
-// per thread: masking, online softmax in the exp2 domain, P (fp16) into one of two swizzled
-// shared-memory buffers, final 1/l scaling (or the unnormalised partial for the combine).  The running maximum is
+// per thread: masking, online softmax in the exp2 domain, P (fp16) written into tensor memory
+// over the columns of the S buffer it came from (the P V product reads its A operand from
+// TMEM), final 1/l scaling (or the unnormalised partial for the combine).  The running maximum is
 // only moved (and O rescaled) when it grows by more than 2^8, so most tiles skip the rescale;
 // the result is exact because numerator and denominator share the reference maximum.
 // The bounded label-mode instantiation (the training form of bf16 models) scans only the key
@@ -38,7 +39,7 @@ struct AttnDev {
   int cap;
   float scale_log2;               // log2(e) / sqrt(dh)
   int nstages;
-  int q_off, k_off, v_off, p_off, bar_off, stage_bytes;
+  int q_off, k_off, v_off, bar_off, stage_bytes;
   void* out;                      // [rows][d_model] bf16
   uint32_t* status;
   int nsplit;                     // key splits per query tile
@@ -49,13 +50,6 @@ struct AttnDev {
   const int* tile_count;          // [query tile] listed key tiles
   int n_ktiles;
 };
-
-SMDM_DEV void p_store_swizzled(uint8_t* P, int row, int key8, uint4 val) {
-  // P: [2 sub-tiles][128 rows][64 keys] fp16, 128-byte swizzle; key8 = 16-byte chunk 0..15
-  const int sub = key8 >> 3, cc = key8 & 7;
-  uint8_t* dst = P + sub * 16384 + row * 128 + ((cc ^ (row & 7)) << 4);
-  *reinterpret_cast<uint4*>(dst) = val;
-}
 
 // 2^x with the hardware approximation (PTX ex2.approx.ftz.f32).
 SMDM_DEV float ex2_approx(float x) {
@@ -86,7 +80,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* Qs = smem + a.q_off;
-  uint8_t* Ps = smem + a.p_off;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.bar_off);
   const int NS = a.nstages;
   uint64_t* q_full = bars;
@@ -201,7 +194,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_s = idesc_f16(128, 128, 0, 0);   // q, K fp16
       const uint32_t idesc_o = idesc_f16(128, dh, 0, 1);   // P, V fp16; V is MN-major
-      const uint32_t q_addr = smem_u32(Qs), p_addr = smem_u32(Ps);
+      const uint32_t q_addr = smem_u32(Qs);
       bool ok = mbar_wait(q_full, 0, abort_flag, a.status);
       int stage = 0;
       uint32_t phase = 0;
@@ -225,20 +218,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (++stage == NS) { stage = 0; phase ^= 1; }
         }
         if (j >= 1) {
-          // O += P_{j-1} V_{j-1}
+          // O += P_{j-1} V_{j-1}, P from tensor memory: it occupies the first 64 columns of the
+          // S buffer of tile j-1 (two fp16 keys per column); S(j+1), the next write to that
+          // buffer, is issued after this product and the tensor core keeps issue order
           const int jj = j - 1;
-          const int pb = jj & 1;   // P buffer of tile jj; its k-th use has phase k & 1
+          const int pb = jj & 1;   // P / S buffer of tile jj; its k-th use has phase k & 1
           if (!mbar_wait(&p_full[pb], (jj >> 1) & 1, abort_flag, a.status)) break;
           if (!mbar_wait(&v_full[pstage], pphase, abort_flag, a.status)) break;
           tc_fence_after();
           const uint32_t v_addr = smem_u32(smem + a.v_off + pstage * a.stage_bytes);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_f16(t_o, sdesc_sw128(p_addr + pb * (128 * 128 * 2) + aoff, 16, 1024),
-                     sdesc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
-                     (jj > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < 8; ++kk)
+            umma_f16_ts(t_o, tbase + pb * 128 + kk * 8,
+                        sdesc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
+                        (jj > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&v_empty[pstage]);
           umma_commit(&pv_done[pb]);
           if (++pstage == NS) { pstage = 0; pphase ^= 1; }
@@ -333,39 +326,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_st16(t_o + lane_off + c * 16, o);
         }
       }
-      // pass 2: P = 2^(s*scale - m_ref) as fp16 into swizzled shared memory
+      // pass 2: P = 2^(s*scale - m_ref) in fp16, two keys per 32-bit column, written over the
+      // first 64 columns of this tile's S buffer (half hh -> columns 32 hh .. 32 hh + 31, after
+      // the S columns 64 hh .. 64 hh + 63 it replaces have been read)
       const float mref_eff = (m_ref == -INFINITY) ? 0.f : m_ref;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         float sv[64];
         tmem_ld64(tbase + lane_off + b * 128 + hh * 64, sv);
+        uint32_t pk[32];
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          float p[8];
+        for (int c2 = 0; c2 < 32; ++c2) {
+          float p2[2];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const int c = c8 * 8 + t;
+          for (int t = 0; t < 2; ++t) {
+            const int c = c2 * 2 + t;
             const bool vis = (mw[hh * 2 + (c >> 5)] >> (c & 31)) & 1u;
-            p[t] = vis ? ex2_approx(fmaf(sv[c], a.scale_log2, -mref_eff)) : 0.f;
-            rsp[t] += p[t];
+            p2[t] = vis ? ex2_approx(fmaf(sv[c], a.scale_log2, -mref_eff)) : 0.f;
+            rsp[(c2 & 3) * 2 + t] += p2[t];
           }
-          uint4 pk;
-          pk.x = pack_f16x2(p[0], p[1]);
-          pk.y = pack_f16x2(p[2], p[3]);
-          pk.z = pack_f16x2(p[4], p[5]);
-          pk.w = pack_f16x2(p[6], p[7]);
-          p_store_swizzled(Ps + (j & 1) * (128 * 128 * 2), em, hh * 8 + c8, pk);
+          pk[c2] = pack_f16x2(p2[0], p2[1]);
         }
+        tmem_st32(tbase + lane_off + b * 128 + hh * 32, pk);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[b]);
       const float rs = ((rsp[0] + rsp[1]) + (rsp[2] + rsp[3])) + ((rsp[4] + rsp[5]) + (rsp[6] + rsp[7]));
       l = l * alpha + rs;
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      // S(j) read and P(j) written (tcgen05.st completed): the S buffer may take S(j+2) once the
+      // P V product of this tile has been issued, which p_full orders
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[j & 1]);
+      if (lane == 0) {
+        mbar_arrive(&s_free[b]);
+        mbar_arrive(&p_full[j & 1]);
+      }
     }
     // Final: O / l (one split), or the unnormalised partial for the combine pass.
     if (nkv > 0 && mbar_wait(&pv_done[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1, abort_flag, a.status)) {
@@ -496,21 +489,20 @@ __global__ void attn_simt_kernel(const T* __restrict__ q, T* __restrict__ out, K
 // ------------------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------------------
+// Shared memory: the Q tile, then NS stages of K and NS stages of V (P lives in tensor memory).
 static int attn_layout(int dh, AttnDev& d) {
   const int q_bytes = 128 * dh * 2;
   const int kv_bytes = 128 * dh * 2;
-  const int p_bytes = 2 * 128 * 128 * 2;   // two P buffers (tile j uses buffer j & 1)
   d.q_off = 0;
-  d.p_off = q_bytes;
   d.stage_bytes = kv_bytes;
-  const int budget = 227 * 1024 - 1024 - 256;
-  int ns = (budget - q_bytes - p_bytes) / (2 * kv_bytes);
-  if (ns > 4) ns = 4;   // the 256-byte barrier area holds 1 + 4 * 4 + 8 barriers
+  const int budget = 227 * 1024 - 1024 - 512;
+  int ns = (budget - q_bytes) / (2 * kv_bytes);
+  if (ns > 6) ns = 6;   // the 512-byte barrier area holds 1 + 4 * 6 + 8 barriers
   d.nstages = ns;
-  d.k_off = q_bytes + p_bytes;
+  d.k_off = q_bytes;
   d.v_off = d.k_off + ns * kv_bytes;
   d.bar_off = d.v_off + ns * kv_bytes;
-  return d.bar_off + 256 + 1024;
+  return d.bar_off + 512 + 1024;
 }
 
 cudaError_t attn_tc_set_smem_attr() {
