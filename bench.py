@@ -39,6 +39,9 @@ import synth  # noqa: E402
 
 METRIC = "decoded tokens/s per full sparse-MDM sampling run"
 UNIT = "tokens/s"
+# bf16 models run their GEMMs and attention on fp16 operands (fp16 copies of the weights made at
+# handle creation, fp16 activations) with fp32 accumulation and an fp32 residual stream.
+COMPUTE_DTYPE = "f16"
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -533,7 +536,7 @@ def run_training_form(args, wl):
                       "unit": "rows/s", "n_gpus": 1, "steps": args.steps,
                       "warmup": max(3, args.warmup), "ms_per_step": ms,
                       "higher_is_better": True, "form": "training", "rows": n,
-                      "logit_rows": int(len(lrows)), "dtype": "bf16" if m.dtype == synth.BF16
+                      "logit_rows": int(len(lrows)), "dtype": COMPUTE_DTYPE if m.dtype == synth.BF16
                       else "f32", "data": "synthetic", "config": describe(wl)}), flush=True)
     model.close()
     return 0
@@ -633,7 +636,7 @@ def run_switched(args, wl):
     print(json.dumps({"metric": METRIC, "value": Lg / (ms / 1e3), "unit": UNIT, "n_gpus": 1,
                       "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
                       "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                      "dtype": "bf16" if m.dtype == synth.BF16 else "f32",
+                      "dtype": COMPUTE_DTYPE if m.dtype == synth.BF16 else "f32",
                       "data": "synthetic", "config": cfg_line}), flush=True)
     del graph
     model.close()
@@ -708,7 +711,7 @@ def run_task(args, wl):
     print(json.dumps({"metric": METRIC, "value": decoded / (ms / 1e3), "unit": UNIT,
                       "n_gpus": 1, "steps": args.steps, "warmup": max(3, args.warmup),
                       "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-                      "vs_baseline": None, "dtype": "bf16" if m.dtype == synth.BF16 else "f32",
+                      "vs_baseline": None, "dtype": COMPUTE_DTYPE if m.dtype == synth.BF16 else "f32",
                       "data": "synthetic", "config": cfg_line}), flush=True)
     del graph
     model.close()
@@ -937,7 +940,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if m.dtype == synth.BF16 else "f32",
+        "scaling": "weak", "vs_baseline": None, "dtype": COMPUTE_DTYPE if m.dtype == synth.BF16 else "f32",
         "data": "synthetic (seeded N(0,0.02) weights drawn on device; seeded prompts/orders)",
         "config": {**describe(wl), "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                    "l2": "weights 1.69 GB >> 126 MB L2 stream from HBM every run (no flush)",
@@ -961,6 +964,7 @@ def main():
                           "peaks": {"hbm_gbs": hbm, "bf16_tflops_sustained": tfl_s}},
         "per_class_ms_per_run": {k: round(v, 4) for k, v in cls_ms.items()},
         "per_class_basis": prof_basis,
+        **({"per_class_graph_error": gprof["error"]} if gprof and "error" in gprof else {}),
         "per_class_roofline_ms_per_run": class_roofline_ms(wl, plans, hbm, tfl_s),
         "per_step_ms": ms / wl.n_steps,
         "dense": dense,

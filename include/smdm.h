@@ -71,7 +71,14 @@ enum { SMDM_PLAN_ORDER = 0, SMDM_PLAN_SEMIAR = 1 };
  * position ids, SwiGLU MLP, untied LM head).
  * bf16 models need d_model % 128 == 0, d_head in {64, 128}, d_ffn % 64 == 0 and vocab % 4 == 0
  * (logit rows are written with 16-byte-aligned bulk copies; logit buffers passed to the
- * library must be 16-byte aligned). */
+ * library must be 16-byte aligned).
+ * Arithmetic of bf16 models: the weights are given in bf16; smdm_create keeps an fp16 copy of
+ * every weight matrix in the workspace, and the GEMMs and the attention multiply fp16 operands
+ * (weights, normalised rows, q/K/V, P, attention and SwiGLU outputs) with fp32 accumulation,
+ * around an fp32 residual stream, fp32 RMSNorm statistics, fp32 softmax and fp32 logits.  fp16
+ * keeps three more mantissa bits than bf16 at the same width and MMA rate; its range ends at
+ * 65504, so a model whose weights or activations go beyond it is not served in this mode (a
+ * weight beyond it fails smdm_create with SMDM_EINVAL). */
 typedef struct {
   int n_layers, d_model, n_heads, d_head, d_ffn;
   int vocab;         /* content vocabulary V */
@@ -107,14 +114,16 @@ typedef struct {
 typedef struct smdm_handle smdm_handle;
 
 /* Bytes of device workspace the handle needs (KV caches for max_batch sequences, activations,
- * RoPE table, reduction scratch).  Returns 0 for an invalid config. */
+ * RoPE table, reduction scratch and, for bf16 models, the fp16 copies of the weight matrices).
+ * Returns 0 for an invalid config. */
 size_t smdm_workspace_bytes(const smdm_config* cfg);
 
 /* Create a handle.  d_workspace: caller-allocated device memory of >= smdm_workspace_bytes,
  * 256-byte aligned; it is initialised here (synchronously, on the legacy default stream).
  * Fails with SMDM_ENOMEM if `bytes` is too small, SMDM_ESHAPE for unsupported shapes,
  * SMDM_EINVAL for a null `out`, null weights or a misaligned workspace (checked on the host,
- * before any CUDA call), SMDM_ECUDA if a CUDA call fails.  *out is null after any failure.
+ * before any CUDA call) or for a bf16 weight beyond the fp16 range (found while making the fp16
+ * copies), SMDM_ECUDA if a CUDA call fails.  *out is null after any failure.
  * Every other call returns SMDM_EINVAL for a null handle; smdm_destroy(NULL) does nothing. */
 smdm_status smdm_create(const smdm_config* cfg, const smdm_weights* w, void* d_workspace,
                         size_t bytes, smdm_handle** out);
@@ -292,10 +301,12 @@ smdm_status smdm_profile_end(smdm_handle* h, smdm_profile* out, cudaStream_t str
  * Same computation and arguments as smdm_forward_stepcausal, but without a handle: the caller
  * passes the model config, the weights and the inputs/outputs, and every byte of scratch
  * (activations, KV rows, split-K partial sums and tile counters, LM-head statistics, RoPE
- * table) lives in one 16 MiB static device array inside the library, which every GPU that
+ * table and, for bf16 models, the fp16 copies of the weight matrices, remade on every call)
+ * lives in one 16 MiB static device array inside the library, which every GPU that
  * loads the library holds until the process exits.  It calls no cudaMalloc/cudaFree.
  *  - Size limit: the scratch this call needs (a one-sequence workspace for max(n, n_rows) rows
- *    with the config's max_len, split-K over 32 CTAs) must fit in 16 MiB; otherwise the call
+ *    with the config's max_len, split-K over 32 CTAs, the weight copies) must fit in 16 MiB;
+ *    otherwise the call
  *    returns SMDM_ESHAPE before launching anything.  A 2-layer d=256 model with a few hundred
  *    rows fits.
  *  - The first call on each device looks up the array's device address and sets kernel
@@ -307,8 +318,9 @@ smdm_status smdm_profile_end(smdm_handle* h, smdm_profile* out, cudaStream_t str
  *    and the launches were accepted, NOT that the logits are valid.  A device-side wait that
  *    timed out, or an id outside the embedding table or a position outside
  *    [0, max_len + tail rows + 2) (replaced by 0 on the device), leaves wrong logits and no
- *    error.  Check the inputs on the host before the call: ids and positions in those ranges,
- *    types in 0..3, labels in [0, n], logit rows in [0, n). */
+ *    error, and so does a bf16 weight beyond the fp16 range.  Check the inputs on the host
+ *    before the call: ids and positions in those ranges, types in 0..3, labels in [0, n],
+ *    logit rows in [0, n). */
 smdm_status smdm_forward_stepcausal_noalloc(const smdm_config* cfg, const smdm_weights* w,
                                             const int32_t* d_ids, const int32_t* d_pos,
                                             const int32_t* d_type, const int32_t* d_label, int n,

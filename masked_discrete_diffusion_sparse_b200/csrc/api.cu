@@ -37,7 +37,8 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows, 128-byte swizzle.
+// 2-D fp16 tensor map: `inner` contiguous elements per row, `outer` rows, 128-byte swizzle (the
+// GEMMs' operands: the fp16 weight copies and the fp16 activations).
 bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
   EncodeTiledFn fn = get_encode_fn();
@@ -46,7 +47,7 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -69,7 +70,7 @@ int encode_gateup_interleaved(CUtensorMap* m, const void* gate, const void* up, 
   cuuint64_t strides[2] = {delta, d * 2};
   cuuint32_t box[3] = {64, 2, 64};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                   const_cast<void*>(up_first ? up : gate), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -130,14 +131,14 @@ bool encode_qkv_interleaved(CUtensorMap* m, const void* w, uint64_t d, int d_hea
     cuuint64_t dims[4] = {d, 2, 64, tiles};
     cuuint64_t strides[3] = {64 * rb, rb, 128 * rb};
     cuuint32_t box[4] = {64, 2, 64, 1};
-    r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(w), dims, strides, box, estr,
+    r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(w), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   } else {
     cuuint64_t dims[5] = {d, 2, 32, 2, tiles};
     cuuint64_t strides[4] = {32 * rb, rb, 64 * rb, 128 * rb};
     cuuint32_t box[5] = {64, 2, 32, 2, 1};
-    r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(w), dims, strides, box, estr,
+    r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 5, const_cast<void*>(w), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   }
@@ -147,6 +148,7 @@ bool encode_qkv_interleaved(CUtensorMap* m, const void* w, uint64_t d, int d_hea
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
+  size_t w16, w16_layer, w16_qkv, w16_o, w16_gu, w16_down, w16_lm;   // fp16 weight copies
   size_t kc, vc, kscr, vscr, x, h, q, ao, act, hq, pmax, psum, parg, rows, rope, partial,
       counters, status, newpos, prompts, aux, attn_part, lbound, tlist, sw, total;
   size_t attn_part_bytes;
@@ -215,6 +217,18 @@ Layout make_layout(const smdm_config* c, int n_sms, bool extras = true) {
     off = align_up(off + bytes, 1024);
     return o;
   };
+  // bf16 models: fp16 copies of every weight matrix, per layer [qkv 3d x d | o d x d |
+  // gate ffn x d | up ffn x d | down d x ffn], then the LM head [V][d]
+  if (c->dtype == SMDM_BF16) {
+    const size_t f = c->d_ffn;
+    L.w16_qkv = 0;
+    L.w16_o = 3 * d * d * 2;
+    L.w16_gu = L.w16_o + d * d * 2;
+    L.w16_down = L.w16_gu + 2 * f * d * 2;
+    L.w16_layer = align_up(L.w16_down + d * f * 2, 1024);
+    L.w16_lm = L.w16_layer * c->n_layers;
+    L.w16 = take(L.w16_lm + (size_t)c->vocab * d * 2);
+  }
   const size_t cache_elems = extras ? (size_t)c->max_batch * c->n_layers * H * L.cap * dh : 0;
   L.kc = take(cache_elems * es);
   L.vc = take(cache_elems * es);
@@ -347,13 +361,21 @@ struct Launch {
       }
       p.cls.resize(p.used + 1);
       p.cls[p.used] = cls;
-      cudaEventRecord(p.ev[p.used * 2], st);
+      record(p.ev[p.used * 2]);
     }
+  }
+  // Under stream capture a plain record only marks a point for cross-stream waits; the
+  // external flag turns it into an event-record node whose time the replay fills in.
+  void record(cudaEvent_t e) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(st, &cs);
+    if (cs == cudaStreamCaptureStatusActive) cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+    else cudaEventRecord(e, st);
   }
   ~Launch() {
     Profiler& p = h->prof;
     if (p.on && p.timed) {
-      cudaEventRecord(p.ev[p.used * 2 + 1], st);
+      record(p.ev[p.used * 2 + 1]);
       p.used++;
     }
   }
@@ -420,7 +442,6 @@ smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensor
   if (rows <= 0) return SMDM_OK;
   Launch lg(h, cls, st);
   constexpr CUtensorMapDataType F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                                BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                                 F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   if (h->bf16) {
     CUtensorMap tmB;
@@ -431,9 +452,9 @@ smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensor
     CUtensorMap tmOut;
     bool ok_out = false;
     switch (ep.kind) {
-      case kEpiStore: ok_out = encode_out(&tmOut, ep.out, BF16, ep.n_valid, rows, ep.ld_out, 128); break;
+      case kEpiStore: ok_out = encode_out(&tmOut, ep.out, F16, ep.n_valid, rows, ep.ld_out, 128); break;
       case kEpiQKV: ok_out = encode_out(&tmOut, ep.q_out, F16, ep.d_model, rows, ep.d_model, 128); break;
-      case kEpiSwiGLU: ok_out = encode_out(&tmOut, ep.act, BF16, ep.n_valid, rows, ep.ld_act, 64); break;
+      case kEpiSwiGLU: ok_out = encode_out(&tmOut, ep.act, F16, ep.n_valid, rows, ep.ld_act, 64); break;
       case kEpiResid: ok_out = encode_out(&tmOut, ep.x, F32, ep.n_valid, rows, ep.ld_x, 128); break;
       case kEpiLMHead:
         // without logits the map is never used: any valid fp32 map will do
@@ -483,8 +504,8 @@ smdm_status norm(smdm_handle* h, float* x, const void* gain, void* out, const in
   a.d = h->cfg.d_model;
   a.eps = h->cfg.rms_eps;
   Launch lg(h, SMDM_K_NORM, st);
-  if (h->bf16) CK(launch_rmsnorm<__nv_bfloat16>(a, rows, st));
-  else CK(launch_rmsnorm<float>(a, rows, st));
+  if (h->bf16) CK((launch_rmsnorm<__nv_bfloat16, __half>(a, rows, st)));
+  else CK((launch_rmsnorm<float, float>(a, rows, st)));
   return SMDM_OK;
 }
 
@@ -624,6 +645,53 @@ smdm_status forward(smdm_handle* h, const FwdSpec& f, cudaStream_t st) {
   return SMDM_OK;
 }
 
+// bf16 models compute in fp16 (fp32 accumulation): every weight matrix is re-encoded once into
+// an fp16 copy in the workspace (exact for magnitudes in [2^-14, 65504]; smaller ones round at
+// 2^-24 absolute; a larger one sets kStatusRange), and the GEMMs' tensor maps point at the
+// copies.  fp16 carries three more mantissa bits than bf16 at the same bytes and the same MMA
+// rate, so the activations that feed the GEMMs (normalised rows, attention output, SwiGLU
+// output) keep them too.  Asynchronous on `st`.
+bool prepare_weights16(smdm_handle* h, const smdm_weights* w, cudaStream_t st) {
+  const smdm_config& c = h->cfg;
+  const size_t d = c.d_model, f = c.d_ffn;
+  const int nl = c.n_layers, dh = c.d_head;
+  uint8_t* base = h->at<uint8_t>(h->L.w16);
+  auto conv = [&](const void* src, uint8_t* dst, size_t n) {
+    return launch_convert_bf16_f16(static_cast<const __nv_bfloat16*>(src),
+                                   reinterpret_cast<__half*>(dst), n, h->status(), st) ==
+           cudaSuccess;
+  };
+  bool ok = true;
+  h->tm_qkv.resize(nl);
+  h->tm_o.resize(nl);
+  h->tm_gate.resize(nl);
+  h->tm_up.resize(nl);
+  h->tm_gu.resize(nl);
+  h->gu_il.assign(nl, 0);
+  h->tm_down.resize(nl);
+  for (int l = 0; l < nl; ++l) {
+    uint8_t* lb = base + (size_t)l * h->L.w16_layer;
+    uint8_t* qkv = lb + h->L.w16_qkv;
+    uint8_t* o = lb + h->L.w16_o;
+    uint8_t* gate = lb + h->L.w16_gu;
+    uint8_t* up = gate + f * d * 2;
+    uint8_t* down = lb + h->L.w16_down;
+    ok &= conv(w->w_qkv[l], qkv, 3 * d * d) && conv(w->w_o[l], o, d * d) &&
+          conv(w->w_gate[l], gate, f * d) && conv(w->w_up[l], up, f * d) &&
+          conv(w->w_down[l], down, d * f);
+    ok &= encode_qkv_interleaved(&h->tm_qkv[l], qkv, d, dh);
+    ok &= encode_2d(&h->tm_o[l], o, d, d, d * 2, 64, 128);
+    ok &= encode_2d(&h->tm_gate[l], gate, d, f, d * 2, 64, 64);
+    ok &= encode_2d(&h->tm_up[l], up, d, f, d * 2, 64, 64);
+    h->gu_il[l] = encode_gateup_interleaved(&h->tm_gu[l], gate, up, d, f);
+    ok &= encode_2d(&h->tm_down[l], down, f, d, f * 2, 64, 128);
+  }
+  uint8_t* lm = base + h->L.w16_lm;
+  ok &= conv(w->lm_head, lm, (size_t)c.vocab * d);
+  ok &= encode_2d(&h->tm_lm, lm, d, c.vocab, d * 2, 64, 128);
+  return ok;
+}
+
 smdm_status check_seq(smdm_handle* h, int seq) {
   if (seq < 0 || seq >= h->cfg.max_batch)
     return fail(h, SMDM_EINVAL, "sequence slot %d out of range [0, %d)", seq, h->cfg.max_batch);
@@ -740,24 +808,8 @@ smdm_status smdm_create(const smdm_config* cfg, const smdm_weights* w, void* d_w
     if (e != cudaSuccess) return cuda_fail(e);
   }
   if (h->bf16) {
-    const int d = cfg->d_model, f = cfg->d_ffn, H = cfg->n_heads, dh = cfg->d_head;
-    bool ok = true;
-    h->tm_qkv.resize(nl);
-    h->tm_o.resize(nl);
-    h->tm_gate.resize(nl);
-    h->tm_up.resize(nl);
-    h->tm_gu.resize(nl);
-    h->gu_il.assign(nl, 0);
-    h->tm_down.resize(nl);
-    for (int l = 0; l < nl; ++l) {
-      ok &= encode_qkv_interleaved(&h->tm_qkv[l], w->w_qkv[l], d, dh);
-      ok &= encode_2d(&h->tm_o[l], w->w_o[l], d, d, (uint64_t)d * 2, 64, 128);
-      ok &= encode_2d(&h->tm_gate[l], w->w_gate[l], d, f, (uint64_t)d * 2, 64, 64);
-      ok &= encode_2d(&h->tm_up[l], w->w_up[l], d, f, (uint64_t)d * 2, 64, 64);
-      h->gu_il[l] = encode_gateup_interleaved(&h->tm_gu[l], w->w_gate[l], w->w_up[l], d, f);
-      ok &= encode_2d(&h->tm_down[l], w->w_down[l], f, d, (uint64_t)f * 2, 64, 128);
-    }
-    ok &= encode_2d(&h->tm_lm, w->lm_head, d, cfg->vocab, (uint64_t)d * 2, 64, 128);
+    const int d = cfg->d_model, H = cfg->n_heads, dh = cfg->d_head;
+    bool ok = prepare_weights16(h, w, 0);
     const size_t MR = align_up((size_t)cfg->max_rows, 256);
     const uint64_t cache_rows = (uint64_t)cfg->max_batch * nl * H * h->L.cap;
     ok &= encode_head_tiles(&h->tm_kc, h->at<uint8_t>(h->L.kc), dh, cache_rows, dh / 64);
@@ -776,6 +828,15 @@ smdm_status smdm_create(const smdm_config* cfg, const smdm_weights* w, void* d_w
   }
   e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e);
+  if (h->bf16) {   // a weight beyond the fp16 range (set by the conversion)
+    uint32_t bits = 0;
+    e = cudaMemcpy(&bits, h->status(), 4, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (bits & kStatusRange) {
+      delete h;
+      return SMDM_EINVAL;
+    }
+  }
   *out = h;
   return SMDM_OK;
 }
@@ -1460,24 +1521,8 @@ extern "C" smdm_status smdm_forward_stepcausal_noalloc(
     if (cudaGetLastError() != cudaSuccess) return SMDM_ECUDA;
   }
   if (h->bf16) {
-    const int d = vc.d_model, f = vc.d_ffn, H = vc.n_heads, dh = vc.d_head;
-    bool ok = true;
-    h->tm_qkv.resize(nl);
-    h->tm_o.resize(nl);
-    h->tm_gate.resize(nl);
-    h->tm_up.resize(nl);
-    h->tm_gu.resize(nl);
-    h->gu_il.assign(nl, 0);
-    h->tm_down.resize(nl);
-    for (int l = 0; l < nl; ++l) {
-      ok &= encode_qkv_interleaved(&h->tm_qkv[l], w->w_qkv[l], d, dh);
-      ok &= encode_2d(&h->tm_o[l], w->w_o[l], d, d, (uint64_t)d * 2, 64, 128);
-      ok &= encode_2d(&h->tm_gate[l], w->w_gate[l], d, f, (uint64_t)d * 2, 64, 64);
-      ok &= encode_2d(&h->tm_up[l], w->w_up[l], d, f, (uint64_t)d * 2, 64, 64);
-      h->gu_il[l] = encode_gateup_interleaved(&h->tm_gu[l], w->w_gate[l], w->w_up[l], d, f);
-      ok &= encode_2d(&h->tm_down[l], w->w_down[l], f, d, (uint64_t)f * 2, 64, 128);
-    }
-    ok &= encode_2d(&h->tm_lm, w->lm_head, d, vc.vocab, (uint64_t)d * 2, 64, 128);
+    const int d = vc.d_model, H = vc.n_heads, dh = vc.d_head;
+    bool ok = prepare_weights16(h, w, st);
     const size_t MR = align_up((size_t)vc.max_rows, 256);
     ok &= encode_head_tiles(&h->tm_kscr, h->at<uint8_t>(L.kscr), dh, (uint64_t)H * MR, dh / 64);
     ok &= encode_head_tiles(&h->tm_vscr, h->at<uint8_t>(L.vscr), dh, (uint64_t)H * MR, dh / 64);

@@ -8,7 +8,7 @@
 //   label mode — the training-form rule evaluated per (query, key) from row types and step
 //     labels; keys are the rows of the same forward.
 //
-// bf16 path: one CTA per (sequence, 128-row query tile, head, key split).  Warp 0 streams Q and
+// bf16 models (fp16 operands): one CTA per (sequence, 128-row query tile, head, key split).  Warp 0 streams Q and
 // K/V tiles with TMA (one copy per 128-row head tile), warp 1 issues tcgen05.mma (S = Q K^T
 // into one of two TMEM buffers, O += P V into a TMEM accumulator), warps 2-5 own one query row
 // per thread: masking, online softmax in the exp2 domain, P (fp16) written into tensor memory
@@ -40,7 +40,7 @@ struct AttnDev {
   float scale_log2;               // log2(e) / sqrt(dh)
   int nstages;
   int q_off, k_off, v_off, bar_off, stage_bytes;
-  void* out;                      // [rows][d_model] bf16
+  void* out;                      // [rows][d_model] fp16
   uint32_t* status;
   int nsplit;                     // key splits per query tile
   int rows_total;
@@ -56,11 +56,6 @@ SMDM_DEV float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-SMDM_DEV uint32_t pack_bf16x2(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 SMDM_DEV uint32_t pack_f16x2(float a, float b) {
@@ -365,21 +360,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_after();
       if (a.nsplit == 1) {
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
-        __nv_bfloat16* out =
-            reinterpret_cast<__nv_bfloat16*>(a.out) + (size_t)row * a.d_model + h * dh;
+        __half* out = reinterpret_cast<__half*>(a.out) + (size_t)row * a.d_model + h * dh;
         for (int c = 0; c < dh / 16; ++c) {
           float o[16];
           tmem_ld16(t_o + lane_off + c * 16, o);
           if (valid) {
             uint4 w0, w1;
-            w0.x = pack_bf16x2(o[0] * inv, o[1] * inv);
-            w0.y = pack_bf16x2(o[2] * inv, o[3] * inv);
-            w0.z = pack_bf16x2(o[4] * inv, o[5] * inv);
-            w0.w = pack_bf16x2(o[6] * inv, o[7] * inv);
-            w1.x = pack_bf16x2(o[8] * inv, o[9] * inv);
-            w1.y = pack_bf16x2(o[10] * inv, o[11] * inv);
-            w1.z = pack_bf16x2(o[12] * inv, o[13] * inv);
-            w1.w = pack_bf16x2(o[14] * inv, o[15] * inv);
+            w0.x = pack_f16x2(o[0] * inv, o[1] * inv);
+            w0.y = pack_f16x2(o[2] * inv, o[3] * inv);
+            w0.z = pack_f16x2(o[4] * inv, o[5] * inv);
+            w0.w = pack_f16x2(o[6] * inv, o[7] * inv);
+            w1.x = pack_f16x2(o[8] * inv, o[9] * inv);
+            w1.y = pack_f16x2(o[10] * inv, o[11] * inv);
+            w1.z = pack_f16x2(o[12] * inv, o[13] * inv);
+            w1.w = pack_f16x2(o[14] * inv, o[15] * inv);
             reinterpret_cast<uint4*>(out + c * 16)[0] = w0;
             reinterpret_cast<uint4*>(out + c * 16)[1] = w1;
           }
@@ -415,7 +409,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // (row, head).
 __global__ void attn_combine_kernel(const float* __restrict__ part_o,
                                     const float* __restrict__ part_ml, int nsplit, int rows,
-                                    int H, int dh, int d_model, __nv_bfloat16* __restrict__ out) {
+                                    int H, int dh, int d_model, __half* __restrict__ out) {
   griddep_launch();
   griddep_wait();
   const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -439,7 +433,7 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o,
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
   for (int t = 0; t < per; ++t)
-    out[(size_t)row * d_model + h * dh + lane * per + t] = __float2bfloat16_rn(acc[t] * inv);
+    out[(size_t)row * d_model + h * dh + lane * per + t] = __float2half_rn(acc[t] * inv);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -612,7 +606,7 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t stream) {
   const long long warps = (long long)c.rows_total * c.H;
   return launch_pdl(attn_combine_kernel, dim3((unsigned)((warps * 32 + 255) / 256)), dim3(256), 0,
                     stream, 1, (const float*)d.part_o, (const float*)d.part_ml, d.nsplit,
-                    c.rows_total, c.H, c.dh, c.d_model, reinterpret_cast<__nv_bfloat16*>(c.out));
+                    c.rows_total, c.H, c.dh, c.d_model, reinterpret_cast<__half*>(c.out));
 }
 
 template <typename T>

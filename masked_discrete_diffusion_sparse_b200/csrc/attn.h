@@ -28,12 +28,12 @@ struct AttnCall {
   const int* label;
   // 3-D head-tile maps {64, rows, row elements / 64}, box {64, 128, d_head / 64} (one copy per
   // 128-row tile):
-  const CUtensorMap* tmQ;   // q [rows][d_model] bf16 (chunk coordinate = head * d_head / 64)
-  const CUtensorMap* tmK;   // K cache [cache rows][d_head] bf16
+  const CUtensorMap* tmQ;   // q [rows][d_model] fp16 (chunk coordinate = head * d_head / 64)
+  const CUtensorMap* tmK;   // K cache [cache rows][d_head] fp16
   const CUtensorMap* tmV;   // V cache, same layout
   long long cache_rows_per_seq;
   int cap;
-  void* out;                // [rows][d_model] bf16
+  void* out;                // [rows][d_model] fp16
   uint32_t* status;
   // split-KV: partial results of `nsplit` key ranges, merged by a combine kernel
   float* part_o;            // [nsplit][rows][d_model] fp32 (unnormalised)

@@ -1,6 +1,7 @@
 // Weight-streaming GEMMs of the transformer step: Y[r][n] = sum_k X[r][k] * W[n][k].
 //
-// bf16 path (tcgen05): "swap-AB" tiles — the weight tile (128 output features x 64 of K) is
+// bf16 models (tcgen05, fp16 operands: the weights' fp16 copies and fp16 activations, fp32
+// accumulation): "swap-AB" tiles — the weight tile (128 output features x 64 of K) is
 // the MMA's A operand and the activation rows (up to 512 of them) are its N dimension, so the
 // per-step row count of a sparse step (|A| + |C| + registers, usually < 300) never pads the
 // 128-row MMA M dimension.  Work is split stream-K style: the (tile, 64-wide K chunk) units are
@@ -21,7 +22,7 @@
 namespace smdm {
 
 constexpr int kGemmThreads = 224;   // 7 warps: 2 producers, MMA, 4 epilogue
-constexpr int kATileBytes = 128 * 128;   // 128 rows x 64 bf16
+constexpr int kATileBytes = 128 * 128;   // 128 rows x 64 fp16
 constexpr int kRing = 16;                // max landing slots (16 KB each) for split-K partials
 
 struct SmemLayout {
@@ -257,7 +258,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
-      const uint32_t idesc = idesc_bf16(128 * kPair, part_rows, 0, 0);
+      const uint32_t idesc = idesc_f16(128 * kPair, part_rows, 0, 0);   // fp16 x fp16 -> fp32
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -644,10 +645,10 @@ static int pow2_ceil(int x) {
 }
 
 cudaError_t gemm_tc_set_smem_attr() {
-  const void* fns[4] = {(const void*)gemm_tc_kernel<__nv_bfloat16, 1, 1>,
-                        (const void*)gemm_tc_kernel<__nv_bfloat16, 1, 2>,
-                        (const void*)gemm_tc_kernel<__nv_bfloat16, 2, 1>,
-                        (const void*)gemm_tc_kernel<__nv_bfloat16, 2, 2>};
+  const void* fns[4] = {(const void*)gemm_tc_kernel<__half, 1, 1>,
+                        (const void*)gemm_tc_kernel<__half, 1, 2>,
+                        (const void*)gemm_tc_kernel<__half, 2, 1>,
+                        (const void*)gemm_tc_kernel<__half, 2, 2>};
   for (const void* f : fns) {
     const cudaError_t e =
         cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
@@ -674,7 +675,7 @@ static int max_pair_clusters(int smem_bytes) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<__nv_bfloat16, 2, 1>, &cfg) !=
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<__half, 2, 1>, &cfg) !=
         cudaSuccess) {
       cudaGetLastError();
       n = -1;
@@ -739,16 +740,16 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream) {
   const bool two_parts = g.RT > 256;
   if (pair == 1) {
     if (two_parts)
-      return launch_pdl(gemm_tc_kernel<__nv_bfloat16, 1, 2>, dim3((unsigned)G), dim3(kGemmThreads),
+      return launch_pdl(gemm_tc_kernel<__half, 1, 2>, dim3((unsigned)G), dim3(kGemmThreads),
                         L.total, stream, 1, *c.tmA, tA2, *c.tmB, *c.tmOut, g, c.epi);
-    return launch_pdl(gemm_tc_kernel<__nv_bfloat16, 1, 1>, dim3((unsigned)G), dim3(kGemmThreads),
+    return launch_pdl(gemm_tc_kernel<__half, 1, 1>, dim3((unsigned)G), dim3(kGemmThreads),
                       L.total, stream, 1, *c.tmA, tA2, *c.tmB, *c.tmOut, g, c.epi);
   }
   if (two_parts)
-    return launch_pdl(gemm_tc_kernel<__nv_bfloat16, 2, 2>, dim3((unsigned)(G * 2)),
+    return launch_pdl(gemm_tc_kernel<__half, 2, 2>, dim3((unsigned)(G * 2)),
                       dim3(kGemmThreads), L.total, stream, 2, *c.tmA, tA2, *c.tmB, *c.tmOut, g,
                       c.epi);
-  return launch_pdl(gemm_tc_kernel<__nv_bfloat16, 2, 1>, dim3((unsigned)(G * 2)),
+  return launch_pdl(gemm_tc_kernel<__half, 2, 1>, dim3((unsigned)(G * 2)),
                     dim3(kGemmThreads), L.total, stream, 2, *c.tmA, tA2, *c.tmB, *c.tmOut, g,
                     c.epi);
 }

@@ -126,13 +126,6 @@ struct EpiParams {
 // silu(g) = g * sigmoid(g) with the fast division (a full-precision division takes a slow
 // software path)
 SMDM_DEV float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
-// silu for bf16 outputs: sigmoid(g) = (1 + tanh(g / 2)) / 2 with the hardware tanh
-// approximation (one special-function op instead of two; its error is far below bf16 rounding)
-SMDM_DEV float silu_bf16out(float g) {
-  float t;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * g));
-  return g * fmaf(0.5f, t, 0.5f);
-}
 
 // Apply the epilogue to a staged tile S[16][128] (S[j][m] = accumulator for activation row
 // r0 + j and output feature n0 + m; for SwiGLU m < 64 are gate rows f0 + m and m >= 64 the up
@@ -365,9 +358,9 @@ SMDM_DEV void epilogue_block(const EpiParams& p, const CUtensorMap* tm_out, floa
       break;
     }
     case kEpiStore: {
-      __nv_bfloat16* Sb = reinterpret_cast<__nv_bfloat16*>(buf);
+      __half* Sb = reinterpret_cast<__half*>(buf);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) Sb[j * 128 + m] = __float2bfloat16_rn(v[j]);
+      for (int j = 0; j < 32; ++j) Sb[j * 128 + m] = __float2half_rn(v[j]);
       publish();
       if (et == 0) {
         tma_store_2d(tm_out, Sb, n0, r0);
@@ -390,7 +383,7 @@ SMDM_DEV void epilogue_block(const EpiParams& p, const CUtensorMap* tm_out, floa
       if (p.swiglu_il) {
         // the partner lane m ^ 1 holds the other half of the pair; lane parity picks the rows
         // (even lanes even rows) so that the work splits evenly, with no shared-memory exchange
-        __nv_bfloat16* Ob = reinterpret_cast<__nv_bfloat16*>(buf);   // [32][64] bf16
+        __half* Ob = reinterpret_cast<__half*>(buf);   // [32][64] fp16
         const int i = m >> 1, h = m & 1;
         const bool mine_is_gate = (h == (p.swiglu_up_first ? 1 : 0));
 #pragma unroll
@@ -401,7 +394,7 @@ SMDM_DEV void epilogue_block(const EpiParams& p, const CUtensorMap* tm_out, floa
           const float other = h ? o1 : o0;
           const float gate = mine_is_gate ? mine : other;
           const float up = mine_is_gate ? other : mine;
-          Ob[(j + h) * 64 + i] = __float2bfloat16_rn(silu_bf16out(gate) * up);
+          Ob[(j + h) * 64 + i] = __float2half_rn(silu_f(gate) * up);
         }
         publish();
         if (et == 0) {
@@ -412,7 +405,7 @@ SMDM_DEV void epilogue_block(const EpiParams& p, const CUtensorMap* tm_out, floa
       }
       // lanes 0..63: gate rows f0 + m; lanes 64..127: up rows f0 + m - 64 (f0 = n0 / 2)
       float* U = reinterpret_cast<float*>(buf);                               // [32][64] fp32
-      __nv_bfloat16* Ob = reinterpret_cast<__nv_bfloat16*>(buf + 32 * 64 * 4);  // [32][64] bf16
+      __half* Ob = reinterpret_cast<__half*>(buf + 32 * 64 * 4);  // [32][64] fp16
       if (m >= 64) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) U[j * 64 + (m - 64)] = v[j];
@@ -420,7 +413,7 @@ SMDM_DEV void epilogue_block(const EpiParams& p, const CUtensorMap* tm_out, floa
       named_bar_sync(1, 128);
       if (m < 64) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) Ob[j * 64 + m] = __float2bfloat16_rn(silu_bf16out(v[j]) * U[j * 64 + m]);
+        for (int j = 0; j < 32; ++j) Ob[j * 64 + m] = __float2half_rn(silu_f(v[j]) * U[j * 64 + m]);
       }
       publish();
       if (et == 0) {

@@ -461,8 +461,19 @@ template <> struct Vec4<__nv_bfloat16> {
   }
 };
 
-// One CTA of 256 threads per row; the row stays in registers (d <= 8192, d % 4 == 0).
-template <typename T>
+template <> struct Vec4<__half> {
+  static SMDM_DEV void store(__half* p, float4 v) {
+    __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+  }
+};
+
+// One CTA of 256 threads per row; the row stays in registers (d <= 8192, d % 4 == 0).  T: gain
+// and embedding dtype; OutT: output dtype.
+template <typename T, typename OutT>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(NormArgs a) {
   griddep_launch();
   griddep_wait();   // launched with programmatic dependent launch
@@ -497,13 +508,13 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(NormArgs a) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) tot += red[i];
   const float rstd = rsqrtf(tot / (float)a.d + a.eps);
-  T* out = reinterpret_cast<T*>(a.out) + (size_t)r * a.d;
+  OutT* out = reinterpret_cast<OutT*>(a.out) + (size_t)r * a.d;
 #pragma unroll
   for (int t = 0; t < kMaxV; ++t) {
     const int i4 = threadIdx.x + t * 256;
     if (i4 < d4) {
       const float4 gg = Vec4<T>::load(g + 4 * i4);
-      Vec4<T>::store(out + 4 * i4, make_float4(v[t].x * rstd * gg.x, v[t].y * rstd * gg.y,
+      Vec4<OutT>::store(out + 4 * i4, make_float4(v[t].x * rstd * gg.x, v[t].y * rstd * gg.y,
                                                v[t].z * rstd * gg.z, v[t].w * rstd * gg.w));
     }
   }
@@ -690,13 +701,49 @@ cudaError_t launch_gather_rows(const int* src, int n, int n_fwd, int* qrow, uint
   return launch_pdl(gather_rows_kernel, dim3((n + 255) / 256), dim3(256), 0, st, 1, src, n, n_fwd, qrow,
                     status);
 }
-template <typename T>
+template <typename T, typename OutT>
 cudaError_t launch_rmsnorm(const NormArgs& a, int rows, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  return launch_pdl(rmsnorm_kernel<T>, dim3(rows), dim3(256), 0, st, 1, a);
+  return launch_pdl(rmsnorm_kernel<T, OutT>, dim3(rows), dim3(256), 0, st, 1, a);
 }
-template cudaError_t launch_rmsnorm<float>(const NormArgs&, int, cudaStream_t);
-template cudaError_t launch_rmsnorm<__nv_bfloat16>(const NormArgs&, int, cudaStream_t);
+template cudaError_t launch_rmsnorm<float, float>(const NormArgs&, int, cudaStream_t);
+template cudaError_t launch_rmsnorm<__nv_bfloat16, __half>(const NormArgs&, int, cudaStream_t);
+
+// bf16 -> fp16, 8 elements per thread when the pointers allow 16-byte accesses
+__global__ void convert_bf16_f16_kernel(const __nv_bfloat16* __restrict__ src,
+                                        __half* __restrict__ dst, size_t n, uint32_t* status) {
+  const size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (i >= n) return;
+  bool over = false;
+  if (i + 8 <= n && ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15) == 0) {
+    const uint4 u = *reinterpret_cast<const uint4*>(src + i);
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+    uint4 o;
+    __half2* h = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(b[k]);
+      over |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
+      h[k] = __floats2half2_rn(f.x, f.y);
+    }
+    *reinterpret_cast<uint4*>(dst + i) = o;
+  } else {
+    for (size_t j = i; j < n && j < i + 8; ++j) {
+      const float f = __bfloat162float(src[j]);
+      over |= fabsf(f) > 65504.f;
+      dst[j] = __float2half_rn(f);
+    }
+  }
+  if (over) atomicOr(status, kStatusRange);
+}
+
+cudaError_t launch_convert_bf16_f16(const __nv_bfloat16* src, __half* dst, size_t n,
+                                    uint32_t* status, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const size_t threads = (n + 7) / 8;
+  convert_bf16_f16_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(src, dst, n, status);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_unmask(const UnmaskArgs& a, int max_nq, cudaStream_t st) {
   const size_t smem = (size_t)max_nq * 12;

@@ -112,6 +112,9 @@ struct UnmaskArgs {
 cudaError_t launch_pack_step(const PackArgs& a, cudaStream_t st);
 cudaError_t launch_pack_linear(const LinearPackArgs& a, cudaStream_t st);
 cudaError_t launch_pack_switched(const PackSwArgs& a, cudaStream_t st);
+// fp16 copy of a bf16 tensor of n elements (kStatusRange in *status for a value beyond 65504).
+cudaError_t launch_convert_bf16_f16(const __nv_bfloat16* src, __half* dst, size_t n,
+                                    uint32_t* status, cudaStream_t st);
 cudaError_t launch_gather_rows(const int* src, int n, int n_fwd, int* qrow, uint32_t* status,
                                cudaStream_t st);
 // Training form: per-row key bounds of the step-causal rule into kvlen (see misc.cu);
@@ -122,7 +125,8 @@ cudaError_t launch_label_bounds(const int* type, const int* label, int n, int* s
 // misc.cu).  scratch: 5 * T + T * T ints, T = ceil(n / 128); returns the list and count arrays.
 cudaError_t launch_tile_lists(const int* type, const int* label, int n, int* scratch,
                               int** lists, int** counts, cudaStream_t st);
-template <typename T>
+// T: the gain / embedding dtype (bf16 or fp32); OutT: the output dtype (fp16 for bf16 models).
+template <typename T, typename OutT>
 cudaError_t launch_rmsnorm(const NormArgs& a, int rows, cudaStream_t st);
 cudaError_t launch_unmask(const UnmaskArgs& a, int max_nq, cudaStream_t st);
 cudaError_t launch_debug_mask(const int* type, const int* label, int n, uint32_t* bitmap,

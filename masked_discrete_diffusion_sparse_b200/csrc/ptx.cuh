@@ -16,6 +16,7 @@ namespace smdm {
 enum : uint32_t {
   kStatusTimeout = 1u << 0,   // a bounded wait gave up
   kStatusBounds = 1u << 1,    // an index failed a device-side bounds check
+  kStatusRange = 1u << 2,     // a bf16 weight lies beyond the fp16 range
 };
 
 SMDM_DEV uint32_t smem_u32(const void* p) {
