@@ -25,7 +25,7 @@
 
 namespace smdm {
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 320;   // warp 0 loads, warp 1 MMA, warps 2-9 two softmax groups
 
 struct AttnDev {
   int mode;        // 0 prefix, 1 label
@@ -67,6 +67,12 @@ SMDM_DEV uint32_t pack_f16x2(float a, float b) {
 // straight-line code (control flow between tcgen05.mma instructions stalls the issue).
 // kBound (label mode, training form from row 0): kvlen[row] bounds the keys a row may see, and
 // a query tile scans only the key tiles listed for it (tile_list / tile_count).
+//
+// Two softmax groups take the key tiles in turn (group g: tiles g, g + 2, ...), each with its
+// own S/P buffer (tensor-memory columns [128 g, 128 g + 128)), its own O accumulator (columns
+// 256 + g DH ...) and its own running maximum and sum, so that one group's exponentials overlap
+// the other's and the tensor core's work.  At the end the two partial results of every row are
+// merged exactly as two key splits are: O = 2^(m0 - M) O0 + 2^(m1 - M) O1 over the same sum.
 template <int DH, bool kBound = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -82,10 +88,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* v_full = k_full + NS;
   uint64_t* k_empty = v_full + NS;    // [NS] K stage free: the S = Q K^T product completed
   uint64_t* v_empty = k_empty + NS;   // [NS] V stage free: the P V product completed
-  uint64_t* s_full = v_empty + NS;    // [2]
-  uint64_t* s_free = s_full + 2;      // [2]
-  uint64_t* p_full = s_free + 2;      // [2] per P buffer: softmax warps wrote P(j), j & 1 == b
-  uint64_t* pv_done = p_full + 2;     // [2] per P buffer: the P(j) V(j) product completed
+  uint64_t* s_full = v_empty + NS;    // [2] per group: S of its current tile is in its buffer
+  uint64_t* s_free = s_full + 2;      // [2] per group: S read (the buffer may take the next S
+                                      //     once the group's P V product has been issued)
+  uint64_t* p_full = s_free + 2;      // [2] per group: P of its current tile written
+  uint64_t* pv_done = p_full + 2;     // [2] per group: the P V product of its tile completed
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pv_done + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -136,8 +143,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
       mbar_init(&s_free[b], 4);
-    }
-    for (int b = 0; b < 2; ++b) {
       mbar_init(&p_full[b], 4);
       mbar_init(&pv_done[b], 1);
     }
@@ -152,7 +157,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
-  const uint32_t t_o = tbase + 256;   // O accumulator columns [256, 256 + dh)
+  const uint32_t t_o0 = tbase + 256;   // O accumulator of group g: columns [256 + g dh, ...)
   griddep_launch();
   griddep_wait();   // q, the KV cache and the row metadata come from earlier kernels
 
@@ -197,6 +202,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint32_t pphase = 0;
       for (int j = 0; ok && j <= nkv; ++j) {
         if (j < nkv) {
+          // S(j) into the buffer of group j & 1, once that group has read S(j - 2)
           const int b = j & 1;
           if (!mbar_wait(&k_full[stage], phase, abort_flag, a.status)) break;
           if (!mbar_wait(&s_free[b], ((j >> 1) & 1) ^ 1, abort_flag, a.status)) break;
@@ -213,20 +219,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (++stage == NS) { stage = 0; phase ^= 1; }
         }
         if (j >= 1) {
-          // O += P_{j-1} V_{j-1}, P from tensor memory: it occupies the first 64 columns of the
-          // S buffer of tile j-1 (two fp16 keys per column); S(j+1), the next write to that
-          // buffer, is issued after this product and the tensor core keeps issue order
+          // O_g += P_{j-1} V_{j-1} (g = (j - 1) & 1), P from tensor memory: it occupies the
+          // first 64 columns of the group's S buffer (two fp16 keys per column); the next S
+          // written there is issued after this product and the tensor core keeps issue order
           const int jj = j - 1;
-          const int pb = jj & 1;   // P / S buffer of tile jj; its k-th use has phase k & 1
+          const int pb = jj & 1;
           if (!mbar_wait(&p_full[pb], (jj >> 1) & 1, abort_flag, a.status)) break;
           if (!mbar_wait(&v_full[pstage], pphase, abort_flag, a.status)) break;
           tc_fence_after();
           const uint32_t v_addr = smem_u32(smem + a.v_off + pstage * a.stage_bytes);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            umma_f16_ts(t_o, tbase + pb * 128 + kk * 8,
+            umma_f16_ts(t_o0 + pb * dh, tbase + pb * 128 + kk * 8,
                         sdesc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
-                        (jj > 0 || kk > 0) ? 1u : 0u);
+                        (jj >= 2 || kk > 0) ? 1u : 0u);
           umma_commit(&v_empty[pstage]);
           umma_commit(&pv_done[pb]);
           if (++pstage == NS) { pstage = 0; pphase ^= 1; }
@@ -234,12 +240,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
   } else {
-    // Softmax warps: thread owns query row em of the tile.
+    // Softmax groups: warps 2-5 (g = 0) and 6-9 (g = 1); a thread owns query row em of the tile
+    // (TMEM lane quarter = warp % 4).
+    const int g = (warp - 2) >> 2;
     const int q4 = warp & 3;
     const int em = q4 * 32 + lane;
     const int row = qrow0 + em;
     const bool valid = em < nq;
     const uint32_t lane_off = uint32_t(q4 * 32) << 16;
+    const uint32_t t_s = tbase + lane_off + g * 128;   // this group's S / P buffer
+    const uint32_t t_og = t_o0 + lane_off + g * dh;    // this group's O accumulator
     int kv_lim = 0, tq = 0, lq = 0;
     if (valid) {
       if (a.mode == 0) kv_lim = a.kvlen[row];
@@ -247,20 +257,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     float m_ref = -INFINITY, l = 0.f;
     const bool warp_any = __any_sync(0xffffffffu, valid);
-    for (int j = 0; j < nkv; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag, a.status)) break;
+    const int n_mine = (nkv - g + 1) >> 1;             // tiles g, g + 2, ... below nkv
+    for (int it = 0; it < n_mine; ++it) {
+      const int j = g + 2 * it;
+      if (!mbar_wait(&s_full[g], it & 1, abort_flag, a.status)) break;
       tc_fence_after();
       if (!warp_any) {
         // no valid query row in this warp: keep the barrier protocol, skip the math
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[b]);
-        // keep in step with the other warps: signal P(j) only once P buffer j & 1 is free, so
-        // that no arrival can land in a later phase of p_full (its P rows are never read back)
-        if (j >= 2 && !mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, a.status)) break;
+        if (lane == 0) mbar_arrive(&s_free[g]);
+        // signal P only once the P buffer is free (the group's previous product completed), so
+        // that no arrival can land in a later phase of p_full (these P rows are never read back)
+        if (it >= 1 && !mbar_wait(&pv_done[g], (it - 1) & 1, abort_flag, a.status)) break;
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[j & 1]);
+        if (lane == 0) mbar_arrive(&p_full[g]);
         continue;
       }
       const int key0 = (kBound ? tlist[j0 + j] : (j0 + j)) * 128;
@@ -281,20 +292,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               bits |= 1u << bb;
           }
         }
-        mw[w] = bits;
+        mw[w] = valid ? bits : 0xffffffffu;   // rows past the tile's end: results unused
       }
-      // pass 1: row maximum over the visible keys (two 64-column halves); eight independent
-      // partial maxima, so one warp per scheduler is not held up by a 128-long dependent chain
+      // Most tiles are visible to every row of the warp: then the per-key tests drop out of
+      // both passes (the softmax is bound by its instruction count, not by latency).
+      const bool full = __all_sync(0xffffffffu, (mw[0] & mw[1] & mw[2] & mw[3]) == 0xffffffffu);
+      // pass 1: row maximum over the visible keys (two 64-column halves) with eight
+      // independent partial maxima (no 128-long dependent chain)
       float mxp[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) mxp[t] = -INFINITY;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         float sv[64];
-        tmem_ld64(tbase + lane_off + b * 128 + hh * 64, sv);
+        tmem_ld64(t_s + hh * 64, sv);
+        if (full) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          mxp[c & 7] = fmaxf(mxp[c & 7], ((mw[hh * 2 + (c >> 5)] >> (c & 31)) & 1u) ? sv[c] : -INFINITY);
+          for (int c = 0; c < 64; ++c) mxp[c & 7] = fmaxf(mxp[c & 7], sv[c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            mxp[c & 7] = fmaxf(mxp[c & 7], ((mw[hh * 2 + (c >> 5)] >> (c & 31)) & 1u) ? sv[c] : -INFINITY);
+        }
       }
       float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
                        fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
@@ -304,96 +323,132 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mx);
         m_ref = mx;
       }
-      float rsp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // partial sums of P
-      // P buffer j & 1 was last read by the P V product of tile j - 2
-      if (j >= 2 && !mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, a.status)) break;
-      const bool rescale = __any_sync(0xffffffffu, alpha != 1.f) && j >= 1;
-      // rescaling O needs the product of tile j - 1 accumulated first
-      if (rescale && !mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status))
-        break;
+      // the P buffer (and O_g) were last used by the group's previous P V product
+      if (it >= 1 && !mbar_wait(&pv_done[g], (it - 1) & 1, abort_flag, a.status)) break;
       tc_fence_after();
-      if (rescale) {
+      if (__any_sync(0xffffffffu, alpha != 1.f) && it >= 1) {
         for (int c = 0; c < dh / 16; ++c) {
           float o[16];
-          tmem_ld16(t_o + lane_off + c * 16, o);
+          tmem_ld16(t_og + c * 16, o);
 #pragma unroll
           for (int t = 0; t < 16; ++t) o[t] *= alpha;
-          tmem_st16(t_o + lane_off + c * 16, o);
+          tmem_st16(t_og + c * 16, o);
         }
       }
-      // pass 2: P = 2^(s*scale - m_ref) in fp16, two keys per 32-bit column, written over the
-      // first 64 columns of this tile's S buffer (half hh -> columns 32 hh .. 32 hh + 31, after
-      // the S columns 64 hh .. 64 hh + 63 it replaces have been read)
+      // pass 2: P = 2^(s*scale - m_ref) in fp16, two keys per 32-bit column, over the first 64
+      // columns of the S buffer (half hh -> columns 32 hh .. 32 hh + 31, after the S columns
+      // 64 hh .. 64 hh + 63 it replaces have been read)
       const float mref_eff = (m_ref == -INFINITY) ? 0.f : m_ref;
+      float rsp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // partial sums of P
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         float sv[64];
-        tmem_ld64(tbase + lane_off + b * 128 + hh * 64, sv);
+        tmem_ld64(t_s + hh * 64, sv);
         uint32_t pk[32];
+        if (full) {
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
-          float p2[2];
+          for (int c2 = 0; c2 < 32; ++c2) {
+            float p2[2];
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const int c = c2 * 2 + t;
-            const bool vis = (mw[hh * 2 + (c >> 5)] >> (c & 31)) & 1u;
-            p2[t] = vis ? ex2_approx(fmaf(sv[c], a.scale_log2, -mref_eff)) : 0.f;
-            rsp[(c2 & 3) * 2 + t] += p2[t];
+            for (int t = 0; t < 2; ++t) {
+              p2[t] = ex2_approx(fmaf(sv[c2 * 2 + t], a.scale_log2, -mref_eff));
+              rsp[(c2 & 3) * 2 + t] += p2[t];
+            }
+            pk[c2] = pack_f16x2(p2[0], p2[1]);
           }
-          pk[c2] = pack_f16x2(p2[0], p2[1]);
+        } else {
+#pragma unroll
+          for (int c2 = 0; c2 < 32; ++c2) {
+            float p2[2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              const int c = c2 * 2 + t;
+              const bool vis = (mw[hh * 2 + (c >> 5)] >> (c & 31)) & 1u;
+              p2[t] = vis ? ex2_approx(fmaf(sv[c], a.scale_log2, -mref_eff)) : 0.f;
+              rsp[(c2 & 3) * 2 + t] += p2[t];
+            }
+            pk[c2] = pack_f16x2(p2[0], p2[1]);
+          }
         }
-        tmem_st32(tbase + lane_off + b * 128 + hh * 32, pk);
+        tmem_st32_nowait(t_s + hh * 32, pk);
       }
+      tmem_wait_st();
       const float rs = ((rsp[0] + rsp[1]) + (rsp[2] + rsp[3])) + ((rsp[4] + rsp[5]) + (rsp[6] + rsp[7]));
       l = l * alpha + rs;
-      // S(j) read and P(j) written (tcgen05.st completed): the S buffer may take S(j+2) once the
-      // P V product of this tile has been issued, which p_full orders
+      // S read and P written (tcgen05.st completed)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&s_free[b]);
-        mbar_arrive(&p_full[j & 1]);
+        mbar_arrive(&s_free[g]);
+        mbar_arrive(&p_full[g]);
       }
     }
-    // Final: O / l (one split), or the unnormalised partial for the combine pass.
-    if (nkv > 0 && mbar_wait(&pv_done[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1, abort_flag, a.status)) {
-      tc_fence_after();
-      if (a.nsplit == 1) {
-        const float inv = (l > 0.f) ? 1.f / l : 0.f;
-        __half* out = reinterpret_cast<__half*>(a.out) + (size_t)row * a.d_model + h * dh;
-        for (int c = 0; c < dh / 16; ++c) {
-          float o[16];
-          tmem_ld16(t_o + lane_off + c * 16, o);
-          if (valid) {
-            uint4 w0, w1;
-            w0.x = pack_f16x2(o[0] * inv, o[1] * inv);
-            w0.y = pack_f16x2(o[2] * inv, o[3] * inv);
-            w0.z = pack_f16x2(o[4] * inv, o[5] * inv);
-            w0.w = pack_f16x2(o[6] * inv, o[7] * inv);
-            w1.x = pack_f16x2(o[8] * inv, o[9] * inv);
-            w1.y = pack_f16x2(o[10] * inv, o[11] * inv);
-            w1.z = pack_f16x2(o[12] * inv, o[13] * inv);
-            w1.w = pack_f16x2(o[14] * inv, o[15] * inv);
-            reinterpret_cast<uint4*>(out + c * 16)[0] = w0;
-            reinterpret_cast<uint4*>(out + c * 16)[1] = w1;
-          }
-        }
-      } else {
-        float* po = a.part_o + ((size_t)split * a.rows_total + row) * a.d_model + h * dh;
-        for (int c = 0; c < dh / 16; ++c) {
-          float o[16];
-          tmem_ld16(t_o + lane_off + c * 16, o);
-          if (valid) {
+    // The group's last product; after the barrier below every product of the CTA has completed
+    // (the group holding the final tile waited for it, and a commit covers all earlier MMAs),
+    // so the Q tile's shared memory is free for the exchange of (m, l).
+    if (n_mine > 0) mbar_wait(&pv_done[g], (n_mine - 1) & 1, abort_flag, a.status);
+    named_bar_sync(1, 256);
+    tc_fence_after();
+    float* xch = reinterpret_cast<float*>(Qs);   // [group][row][m, l]
+    xch[(g * 128 + em) * 2 + 0] = m_ref;
+    xch[(g * 128 + em) * 2 + 1] = l;
+    named_bar_sync(2, 256);
+    const float m_x = xch[((g ^ 1) * 128 + em) * 2 + 0];
+    const float l_x = xch[((g ^ 1) * 128 + em) * 2 + 1];
+    const float m0 = g ? m_x : m_ref, l0 = g ? l_x : l;
+    const float m1 = g ? m_ref : m_x, l1 = g ? l : l_x;
+    const float M = fmaxf(m0, m1);
+    const float a0 = (M == -INFINITY || m0 == -INFINITY) ? 0.f : ex2_approx(m0 - M);
+    const float a1 = (M == -INFINITY || m1 == -INFINITY) ? 0.f : ex2_approx(m1 - M);
+    const float L = a0 * l0 + a1 * l1;
+    // a group without tiles never wrote its accumulator: leave it out (its a is 0)
+    const bool use1 = nkv >= 2;
+    // group g writes the head-dim columns [g dh/2, (g + 1) dh/2) of the merged row
+    constexpr int half = dh / 2;
+    const uint32_t t_c0 = t_o0 + lane_off + g * half;
+    if (a.nsplit == 1) {
+      const float inv = (L > 0.f) ? 1.f / L : 0.f;
+      const float f0 = a0 * inv, f1 = a1 * inv;
+      __half* out = reinterpret_cast<__half*>(a.out) + (size_t)row * a.d_model + h * dh + g * half;
+      for (int c = 0; c < half / 16; ++c) {
+        float o[16], o1[16];
+        tmem_ld16(t_c0 + c * 16, o);
+        if (use1) tmem_ld16(t_c0 + dh + c * 16, o1);
+        else {
 #pragma unroll
-            for (int t = 0; t < 16; t += 4)
-              *reinterpret_cast<float4*>(po + c * 16 + t) = make_float4(o[t], o[t + 1], o[t + 2], o[t + 3]);
-          }
+          for (int t = 0; t < 16; ++t) o1[t] = 0.f;
         }
         if (valid) {
-          float* ml = a.part_ml + (((size_t)split * a.rows_total + row) * a.H + h) * 2;
-          ml[0] = m_ref;
-          ml[1] = l;
+          uint32_t w[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            w[t] = pack_f16x2(o[2 * t] * f0 + o1[2 * t] * f1, o[2 * t + 1] * f0 + o1[2 * t + 1] * f1);
+          reinterpret_cast<uint4*>(out + c * 16)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          reinterpret_cast<uint4*>(out + c * 16)[1] = make_uint4(w[4], w[5], w[6], w[7]);
         }
+      }
+    } else {
+      float* po = a.part_o + ((size_t)split * a.rows_total + row) * a.d_model + h * dh + g * half;
+      for (int c = 0; c < half / 16; ++c) {
+        float o[16], o1[16];
+        tmem_ld16(t_c0 + c * 16, o);
+        if (use1) tmem_ld16(t_c0 + dh + c * 16, o1);
+        else {
+#pragma unroll
+          for (int t = 0; t < 16; ++t) o1[t] = 0.f;
+        }
+        if (valid) {
+#pragma unroll
+          for (int t = 0; t < 16; t += 4)
+            *reinterpret_cast<float4*>(po + c * 16 + t) =
+                make_float4(o[t] * a0 + o1[t] * a1, o[t + 1] * a0 + o1[t + 1] * a1,
+                            o[t + 2] * a0 + o1[t + 2] * a1, o[t + 3] * a0 + o1[t + 3] * a1);
+        }
+      }
+      if (valid && g == 0) {
+        float* ml = a.part_ml + (((size_t)split * a.rows_total + row) * a.H + h) * 2;
+        ml[0] = M;
+        ml[1] = L;
       }
     }
   }

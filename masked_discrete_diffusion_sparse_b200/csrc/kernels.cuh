@@ -289,8 +289,8 @@ SMDM_DEV int qkv_lane_feature(int m, int d_head) {
 // callers alternate two, and since et == 0 waits for its earlier copies to finish reading
 // shared memory before the block's barrier, a buffer is free again two blocks later.  All 128
 // epilogue threads call this (et = 0..127); et == 0 issues the copies.  tm_out: the call's
-// output tensor map (bf16 out / q / act boxes of 32 rows, fp32 x / logits boxes of 32 rows);
-// K/V cache rows of QKV tiles go out as 1-D bulk copies, one per run of consecutive slots.
+// output tensor map (fp16 out / q / act boxes of 32 rows, fp32 x / logits boxes of 32 rows);
+// K/V cache rows of QKV tiles go out as 16-byte stores of all epilogue threads.
 // Output rows at or beyond the map's row count are clipped by the TMA unit.
 template <typename T>
 SMDM_DEV void epilogue_block(const EpiParams& p, const CUtensorMap* tm_out, float* v, uint8_t* buf,
@@ -335,25 +335,29 @@ SMDM_DEV void epilogue_block(const EpiParams& p, const CUtensorMap* tm_out, floa
 #pragma unroll
       for (int j = 0; j < 32; ++j) dst[j * stride] = __float2half_rn(v[j]);
       publish();
-      if (et == 0) {
-        if (region == 0) {
+      if (region == 0) {
+        if (et == 0) {
           tma_store_2d(tm_out, Sb, nn0, r0);
-        } else {
-          const long long base = (long long)p.layer * p.kv.layer_stride +
-                                 (long long)(nn0 / dh) * p.kv.head_stride;
-          __half* cache = reinterpret_cast<__half*>(region == 1 ? p.kv.k : p.kv.v) + base;
-          int j0 = 0;
-          while (j0 < nrows) {
-            const long long o0 = meta_kv[r0 + j0 - meta_r0];
-            int j1 = j0 + 1;
-            while (j1 < nrows && meta_kv[r0 + j1 - meta_r0] == o0 + (long long)(j1 - j0) * dh) ++j1;
-            for (int h = 0; h < 128 / dh; ++h)
-              bulk_store(cache + (long long)h * p.kv.head_stride + o0, Sb + (h * 32 + j0) * dh,
-                         (uint32_t)((j1 - j0) * dh * 2));
-            j0 = j1;
-          }
+          bulk_commit();
         }
-        bulk_commit();
+      } else {
+        // K / V rows go to their cache slots, which follow the positions (scattered at a
+        // sampling step): 16-byte stores by all 128 threads, two rows per warp instruction.
+        // (One bulk copy per row issued by a single thread serialised the block.)  The staging
+        // buffer is read synchronously here, so it is free again two blocks later as well.
+        const long long base = (long long)p.layer * p.kv.layer_stride +
+                               (long long)(nn0 / dh) * p.kv.head_stride;
+        __half* cache = reinterpret_cast<__half*>(region == 1 ? p.kv.k : p.kv.v) + base;
+        const int cpr = dh / 8;                  // 16-byte chunks per row of one head
+        const int per_head = nrows * cpr;
+        const int total = (128 / dh) * per_head;
+        for (int i = et; i < total; i += 128) {
+          const int hh2 = i / per_head, rem = i - hh2 * per_head;
+          const int rr = rem / cpr, c = rem - rr * cpr;
+          const long long o0 = meta_kv[r0 + rr - meta_r0];
+          const uint4 v4 = *reinterpret_cast<const uint4*>(Sb + (hh2 * 32 + rr) * dh + c * 8);
+          *reinterpret_cast<uint4*>(cache + (long long)hh2 * p.kv.head_stride + o0 + c * 8) = v4;
+        }
       }
       break;
     }
