@@ -438,31 +438,42 @@ SMDM_DEV void epilogue_block(const EpiParams& p, const CUtensorMap* tm_out, floa
       // Per row: max, first argmax and sum exp(l - max) over the tile's 128 columns.  Four
       // threads per row (et >> 2 = row, et & 3 = a quarter of 32 columns), each walking its
       // columns in an order rotated by et so that the 32 lanes of a warp read 32 different
-      // banks; ties in the maximum go to the lowest column, whatever the walking order.
+      // banks.  Three passes (the row maximum, the lowest column holding it, the sum), each a
+      // short loop of four independent chains: compact code, no 32-long dependent chain.
       const int vt = n0 >> 7;
       const int j = et >> 2, qq = et & 3;
       const float* Srow = S + j * 128 + qq * 32;
       const int col0 = n0 + qq * 32;
-      float best = -INFINITY;
-      int arg = 0x7fffffff;
+      const int nv = min(32, max(0, p.n_valid - col0));   // valid columns of this quarter
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+      for (int c0 = 0; c0 < 32; c0 += 8) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const int cc = (c + et) & 31;
-        const float x = (col0 + cc < p.n_valid) ? Srow[cc] : -INFINITY;
-        if (x > best || (x == best && col0 + cc < arg)) { best = x; arg = col0 + cc; }
+        for (int i = 0; i < 8; ++i) {
+          const int cc = (c0 + i + et) & 31;
+          if (cc < nv) m4[i & 3] = fmaxf(m4[i & 3], Srow[cc]);
+        }
       }
+      float best = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
 #pragma unroll
-      for (int o = 1; o <= 2; o <<= 1) {
-        const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
-        if (ob > best || (ob == best && oa < arg)) { best = ob; arg = oa; }
-      }
+      for (int o = 1; o <= 2; o <<= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
+      int a4[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int c0 = 0; c0 < 32; c0 += 8) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const int cc = (c + et) & 31;
-        if (col0 + cc < p.n_valid) s4[c & 3] += __expf(Srow[cc] - best);
+        for (int i = 0; i < 8; ++i) {
+          const int cc = (c0 + i + et) & 31;
+          if (cc < nv) {
+            const float x = Srow[cc];
+            if (x == best) a4[i & 3] = min(a4[i & 3], col0 + cc);
+            s4[i & 3] += __expf(x - best);
+          }
+        }
       }
+      int arg = min(min(a4[0], a4[1]), min(a4[2], a4[3]));
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) arg = min(arg, __shfl_xor_sync(0xffffffffu, arg, o));
       float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
 #pragma unroll
       for (int o = 1; o <= 2; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
