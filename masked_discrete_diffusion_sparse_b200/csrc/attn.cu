@@ -200,43 +200,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint32_t phase = 0;
       int pstage = 0;
       uint32_t pphase = 0;
-      for (int j = 0; ok && j <= nkv; ++j) {
-        if (j < nkv) {
-          // S(j) into the buffer of group j & 1, once that group has read S(j - 2)
-          const int b = j & 1;
-          if (!mbar_wait(&k_full[stage], phase, abort_flag, a.status)) break;
-          if (!mbar_wait(&s_free[b], ((j >> 1) & 1) ^ 1, abort_flag, a.status)) break;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(smem + a.k_off + stage * a.stage_bytes);
+      // S(j) = Q K(j)^T into the buffer of group j & 1, once that group has read S(j - 2)
+      auto issue_s = [&](int j) -> bool {
+        const int b = j & 1;
+        if (!mbar_wait(&k_full[stage], phase, abort_flag, a.status)) return false;
+        if (!mbar_wait(&s_free[b], ((j >> 1) & 1) ^ 1, abort_flag, a.status)) return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + a.k_off + stage * a.stage_bytes);
 #pragma unroll
-          for (int kk = 0; kk < dh / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_f16(tbase + b * 128, sdesc_sw128(q_addr + off, 16, 1024),
-                     sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&s_full[b]);
-          umma_commit(&k_empty[stage]);
-          if (++stage == NS) { stage = 0; phase ^= 1; }
+        for (int kk = 0; kk < dh / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_f16(tbase + b * 128, sdesc_sw128(q_addr + off, 16, 1024),
+                   sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
-        if (j >= 1) {
-          // O_g += P_{j-1} V_{j-1} (g = (j - 1) & 1), P from tensor memory: it occupies the
-          // first 64 columns of the group's S buffer (two fp16 keys per column); the next S
-          // written there is issued after this product and the tensor core keeps issue order
-          const int jj = j - 1;
-          const int pb = jj & 1;
-          if (!mbar_wait(&p_full[pb], (jj >> 1) & 1, abort_flag, a.status)) break;
-          if (!mbar_wait(&v_full[pstage], pphase, abort_flag, a.status)) break;
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(smem + a.v_off + pstage * a.stage_bytes);
+        umma_commit(&s_full[b]);
+        umma_commit(&k_empty[stage]);
+        if (++stage == NS) { stage = 0; phase ^= 1; }
+        return true;
+      };
+      // Issue order follows the order in which the groups finish their tiles: after group g
+      // publishes P(j), its product O_g += P(j) V(j) and then its next score tile S(j + 2).
+      // (Issuing S(j) before P(j - 1) V(j - 1) made each group wait for the other's softmax,
+      // so the two never overlapped.)
+      if (ok) ok = issue_s(0);
+      if (ok && nkv > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < nkv; ++j) {
+        // O_g += P_j V_j (g = j & 1), P from tensor memory: it occupies the first 64 columns of
+        // the group's S buffer (two fp16 keys per column); the next S written there is issued
+        // after this product and the tensor core keeps issue order
+        const int pb = j & 1;
+        if (!mbar_wait(&p_full[pb], (j >> 1) & 1, abort_flag, a.status)) break;
+        if (!mbar_wait(&v_full[pstage], pphase, abort_flag, a.status)) break;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(smem + a.v_off + pstage * a.stage_bytes);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_f16_ts(t_o0 + pb * dh, tbase + pb * 128 + kk * 8,
-                        sdesc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
-                        (jj >= 2 || kk > 0) ? 1u : 0u);
-          umma_commit(&v_empty[pstage]);
-          umma_commit(&pv_done[pb]);
-          if (++pstage == NS) { pstage = 0; pphase ^= 1; }
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          umma_f16_ts(t_o0 + pb * dh, tbase + pb * 128 + kk * 8,
+                      sdesc_sw128(v_addr + kk * 2048, 16384, 1024), idesc_o,
+                      (j >= 2 || kk > 0) ? 1u : 0u);
+        umma_commit(&v_empty[pstage]);
+        umma_commit(&pv_done[pb]);
+        if (++pstage == NS) { pstage = 0; pphase ^= 1; }
+        if (j + 2 < nkv && !issue_s(j + 2)) break;
       }
     }
   } else {

@@ -87,33 +87,39 @@ def run(actors, sim, seed):
 
 
 def mma_issuer(nkv, NS, sim, q_full, k_full, v_full, s_free, p_full, on_s, on_pv, st):
-    """S(j) = Q K(j)^T into buffer j & 1 once K(j) landed and that buffer is free; then
-    O_{(j-1)&1} += P(j-1) V(j-1) once P(j-1) and V(j-1) are there.  on_s / on_pv deliver the
-    commits' arrivals."""
+    """S(0) and S(1), then per tile j in order: O_{j&1} += P(j) V(j) once P(j) and V(j) are
+    there, then S(j + 2) into buffer j & 1 once K(j + 2) landed and the buffer is free.
+    on_s / on_pv deliver the commits' arrivals."""
     yield lambda: q_full.done(0)
-    stage = phase = pstage = pphase = 0
-    for j in range(nkv + 1):
-        if j < nkv:
-            b = j & 1
-            yield lambda s=stage, p=phase: k_full[s].done(p)
-            yield lambda b=b, j=j: s_free[b].done(((j >> 1) & 1) ^ 1)
-            # the buffer's previous tile (j - 2) was read and its P V product issued before
-            assert j < 2 or (st["reads"][j - 2] == 4 and (j - 2) in st["pv_issued"])
-            sim.events.append(lambda b=b, s=stage, j=j: on_s(j, b, s))
-            stage += 1
-            if stage == NS:
-                stage, phase = 0, phase ^ 1
-        if j >= 1:
-            jj = j - 1
-            pb = jj & 1
-            yield lambda pb=pb, jj=jj: p_full[pb].done((jj >> 1) & 1)
-            assert st["writes"][jj] == 4, "P V issued before all of P(j) was written"
-            yield lambda s=pstage, p=pphase: v_full[s].done(p)
-            st["pv_issued"].add(jj)
-            sim.events.append(lambda s=pstage, pb=pb, jj=jj: on_pv(jj, s, pb))
-            pstage += 1
-            if pstage == NS:
-                pstage, pphase = 0, pphase ^ 1
+    ring = {"stage": 0, "phase": 0}
+
+    def issue_s(j):
+        b = j & 1
+        yield lambda s=ring["stage"], p=ring["phase"]: k_full[s].done(p)
+        yield lambda b=b, j=j: s_free[b].done(((j >> 1) & 1) ^ 1)
+        # the buffer's previous tile (j - 2) was read and its P V product issued before
+        assert j < 2 or (st["reads"][j - 2] == 4 and (j - 2) in st["pv_issued"])
+        sim.events.append(lambda b=b, s=ring["stage"], j=j: on_s(j, b, s))
+        ring["stage"] += 1
+        if ring["stage"] == NS:
+            ring["stage"], ring["phase"] = 0, ring["phase"] ^ 1
+
+    yield from issue_s(0)
+    if nkv > 1:
+        yield from issue_s(1)
+    pstage = pphase = 0
+    for j in range(nkv):
+        pb = j & 1
+        yield lambda pb=pb, j=j: p_full[pb].done((j >> 1) & 1)
+        assert st["writes"][j] == 4, "P V issued before all of P(j) was written"
+        yield lambda s=pstage, p=pphase: v_full[s].done(p)
+        st["pv_issued"].add(j)
+        sim.events.append(lambda s=pstage, pb=pb, j=j: on_pv(j, s, pb))
+        pstage += 1
+        if pstage == NS:
+            pstage, pphase = 0, pphase ^ 1
+        if j + 2 < nkv:
+            yield from issue_s(j + 2)
 
 
 def softmax_warp(g, nkv, s_full, pv_done, s_free, p_full, st, final_wait=True):
