@@ -179,3 +179,21 @@ def test_oracle_sample_states_have_the_run_shapes():
         # doubling every sampled time halves the extrapolated rate
         assert abs(s.extrapolate({c: 2 * v for c, v in secs.items()})
                    - 2 * s.extrapolate(secs)) < 1e-9 * s.extrapolate(secs) + 1e-12
+
+
+def test_oracle_sample_components_time_repeatedly_on_unchanged_states():
+    """The single-threaded and the all-cores samples, and the reference arm's rotation, time the
+    same step several times: each call must start from the same state (the step appends to its
+    cache), so the cache length seen by a step is the same on every call."""
+    b = _bench()
+    wl = synth.WORKLOADS["tiny-f32-cos"]
+    s = b.OracleSample(wl)
+    s.run(1)
+    s.run(2)
+    k = s.steps[-1]
+    st0, _ = s._states[k]
+    ctx0 = st0.ctx
+    for _ in range(3):
+        s.time_component(f"step {k}", 1)
+        st = s._states[k][0]
+        assert st.ctx == ctx0 and all(len(kc) == ctx0 for kc in st.k_cache + st.v_cache)
