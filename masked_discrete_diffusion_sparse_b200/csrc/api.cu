@@ -252,7 +252,7 @@ Layout make_layout(const smdm_config* c, int n_sms, bool extras = true) {
   int max_nt = 3 * c->d_model / 128 + 1;
   max_nt = std::max(max_nt, c->d_ffn / 64 + 1);
   max_nt = std::max(max_nt, (c->vocab + 127) / 128);
-  const int rb = c->max_rows > 512 ? (c->max_rows + 255) / 256 : 1;
+  const int rb = c->max_rows > 512 ? (c->max_rows + 255) / 256 : 2;   // (2: the split LM head)
   L.max_tiles = max_nt * rb;
   L.counters = take((size_t)L.max_tiles * 4);
   L.status = take(256);
@@ -447,7 +447,8 @@ smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensor
     CUtensorMap tmB;
     const size_t MR = align_up((size_t)h->cfg.max_rows, 256);
     const int pair = gemm_tc_pair(n_out, swiglu, rows, ep.kind);
-    if (!encode_2d(&tmB, X, K, MR, (uint64_t)K * 2, 64, gemm_tc_box_rows(rows, pair)))
+    const int mrb = gemm_tc_min_row_blocks(n_out, rows, ep.kind, h->L.n_sms);
+    if (!encode_2d(&tmB, X, K, MR, (uint64_t)K * 2, 64, gemm_tc_box_rows(rows, pair, mrb)))
       return fail(h, SMDM_ECUDA, "cuTensorMapEncodeTiled failed for an activation operand");
     CUtensorMap tmOut;
     bool ok_out = false;
@@ -477,6 +478,7 @@ smdm_status gemm(smdm_handle* h, int cls, const CUtensorMap* tmA, const CUtensor
     c.swiglu_il = swiglu && ep.swiglu_il;
     c.a_interleave = a_interleave;
     c.sched = sched;
+    c.min_row_blocks = mrb;
     c.num_ctas = h->L.n_sms;
     c.partial = h->at<float>(h->L.partial);
     c.partial_bytes = h->L.partial_bytes;

@@ -610,7 +610,11 @@ __global__ void __launch_bounds__(128)
 // Host side
 // ------------------------------------------------------------------------------------------
 
-int gemm_tc_row_tile(int rows) {
+int gemm_tc_row_tile(int rows, int min_blocks) {
+  if (min_blocks > 1) {   // at least min_blocks blocks of a multiple of 32 rows
+    const int rt = ((rows + min_blocks - 1) / min_blocks + 31) & ~31;
+    return rt > 256 ? 256 : rt;
+  }
   // One row block of up to 512 rows keeps every weight tile streamed exactly once.
   const int R16 = (rows + 15) & ~15;
   if (R16 <= 256) return R16;
@@ -618,9 +622,17 @@ int gemm_tc_row_tile(int rows) {
   return 256;
 }
 
-int gemm_tc_box_rows(int rows, int pair) {
-  const int RT = gemm_tc_row_tile(rows);
+int gemm_tc_box_rows(int rows, int pair, int min_blocks) {
+  const int RT = gemm_tc_row_tile(rows, min_blocks);
   return (RT > 256 ? RT / 2 : RT) / pair;
+}
+
+int gemm_tc_min_row_blocks(int n_out, int rows, int epi_kind, int sms) {
+  // The LM head's whole tiles (V / 128, 64 for V = 8192) leave most SMs idle while each CTA
+  // runs the row-statistics epilogue over every decode row; two row blocks put twice the CTAs
+  // on it, each with half the epilogue (the weight tile is then read twice, from L2).
+  const int n_tiles = (n_out + 127) / 128;
+  return (epi_kind == kEpiLMHead && rows >= 64 && 2 * n_tiles <= sms) ? 2 : 1;
 }
 
 // Whole tiles (one CTA per tile, no split-K fix-up) when the tile count is at least this
@@ -692,7 +704,7 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream) {
   g.swiglu = c.swiglu;
   g.a_mode = c.swiglu ? (c.swiglu_il ? 4 : 1) : c.a_interleave == 128 ? 2 : c.a_interleave == 64 ? 3 : 0;
   g.n_tiles = c.swiglu ? (c.n_out + 63) / 64 : (c.n_out + 127) / 128;
-  g.RT = gemm_tc_row_tile(c.rows);
+  g.RT = gemm_tc_row_tile(c.rows, c.min_row_blocks);
   g.row_blocks = (c.rows + g.RT - 1) / g.RT;
   g.rows = c.rows;
   g.row0 = c.row0;

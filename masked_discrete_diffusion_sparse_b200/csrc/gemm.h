@@ -5,14 +5,14 @@
 namespace smdm {
 
 struct GemmCall {
-  const CUtensorMap* tmA;   // weights [n_out][K] bf16, box {64, 128} (SwiGLU: gate, box {64, 64})
+  const CUtensorMap* tmA;   // weights [n_out][K] fp16, box {64, 128} (SwiGLU: gate, box {64, 64})
   const CUtensorMap* tmA2;  // SwiGLU: up weights, box {64, 64} (split layout)
                             // interleaved layout: tmA = 3-D map {d, 2 (gate/up), ffn}, box
                             // {64, 2, 64}: A-tile row 2i / 2i+1 = gate / up row f0 + i
-  const CUtensorMap* tmB;   // activations [*][K] bf16, box {64, gemm_tc_box_rows(rows, pair)}
+  const CUtensorMap* tmB;   // activations [*][K] fp16, box {64, gemm_tc_box_rows(rows, pair, mrb)}
   const CUtensorMap* tmOut; // epilogue output, rows = `rows` (no swizzle), box {w, 32}:
-                            //   store: out bf16 [rows][n_out], w 128;  QKV: q bf16 [rows][d], w 128;
-                            //   SwiGLU: act bf16 [rows][ffn], w 64;  residual: x fp32 [rows][d],
+                            //   store: out fp16 [rows][n_out], w 128;  QKV: q fp16 [rows][d], w 128;
+                            //   SwiGLU: act fp16 [rows][ffn], w 64;  residual: x fp32 [rows][d],
                             //   w 128 (reduce-add);  LM head: logits fp32 [rows][V], w 128 (or any
                             //   valid map when no logits are written)
   int K;
@@ -27,8 +27,9 @@ struct GemmCall {
                             // activation rows per CTA); gemm_tc_pair() picks it
   int max_stages;           // 0 = as many as fit
   int producers;            // TMA-issuing threads, 1 or 2 (0 = default)
-  int sched;                // 0: whole tiles per CTA when the tile count is 60-100% of the grid,
+  int sched;                // 0: whole tiles per CTA when the tile count is 40-100% of the grid,
                             // else stream-K; 1: whole tiles whenever they fit; 2: stream-K
+  int min_row_blocks;       // gemm_tc_min_row_blocks(); the B map's box must match
   float* partial;           // split-K scratch: [num_ctas][2][128][row_tile rounded to 32] fp32
   size_t partial_bytes;
   unsigned* counters;       // [max_tiles], zero-initialised; restored to zero by the kernel
@@ -37,8 +38,13 @@ struct GemmCall {
   EpiParams epi;
 };
 
-int gemm_tc_row_tile(int rows);
-int gemm_tc_box_rows(int rows, int pair);
+// Activation rows per row block; min_blocks > 1 splits the rows into at least that many
+// blocks (multiples of 32 rows).
+int gemm_tc_row_tile(int rows, int min_blocks = 1);
+int gemm_tc_box_rows(int rows, int pair, int min_blocks = 1);
+// Row blocks to ask for: 2 for an LM head whose tiles would occupy at most half of the SMs
+// (its epilogue, not its weights, sets its time there), else 1.
+int gemm_tc_min_row_blocks(int n_out, int rows, int epi_kind, int sms);
 // CTA-pair mode (2) or single-CTA mode (1) for a bf16 GEMM of this shape.
 int gemm_tc_pair(int n_out, int swiglu, int rows, int epi_kind);
 cudaError_t gemm_tc_set_smem_attr();
