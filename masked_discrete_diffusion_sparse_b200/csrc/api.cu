@@ -96,8 +96,8 @@ bool encode_head_tiles(CUtensorMap* m, const void* base, uint64_t row_elems, uin
   return r == CUDA_SUCCESS;
 }
 
-// 2-D output map for the GEMM epilogue's TMA stores: `cols` x `rows` elements (fp32, bf16 or,
-// for q, fp16), row pitch `ld` elements, box {box_cols, 32}, no swizzle.
+// 2-D output map for the GEMM epilogue's TMA stores: `cols` x `rows` elements (fp32 or fp16),
+// row pitch `ld` elements, box {box_cols, 32}, no swizzle.
 bool encode_out(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols,
                 uint64_t rows, uint64_t ld, uint32_t box_cols) {
   EncodeTiledFn fn = get_encode_fn();

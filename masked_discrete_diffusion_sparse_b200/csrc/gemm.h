@@ -45,7 +45,7 @@ int gemm_tc_box_rows(int rows, int pair, int min_blocks = 1);
 // Row blocks to ask for: 2 for an LM head whose tiles would occupy at most half of the SMs
 // (its epilogue, not its weights, sets its time there), else 1.
 int gemm_tc_min_row_blocks(int n_out, int rows, int epi_kind, int sms);
-// CTA-pair mode (2) or single-CTA mode (1) for a bf16 GEMM of this shape.
+// CTA-pair mode (2) or single-CTA mode (1) for a tensor-core GEMM of this shape.
 int gemm_tc_pair(int n_out, int swiglu, int rows, int epi_kind);
 cudaError_t gemm_tc_set_smem_attr();
 cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t stream);

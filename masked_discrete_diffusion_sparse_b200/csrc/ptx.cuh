@@ -322,7 +322,7 @@ SMDM_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 SMDM_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 SMDM_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, f32 accumulate (kind::f16).
+// D[tmem] (+)= A[smem] * B[smem]^T, fp16 inputs, f32 accumulate (kind::f16).
 SMDM_DEV void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                        uint32_t accumulate) {
   asm volatile(
@@ -333,7 +333,7 @@ SMDM_DEV void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T, f16/bf16 inputs, f32 accumulate: the A operand is read from
+// D[tmem] (+)= A[tmem] * B[smem]^T, fp16 inputs, f32 accumulate: the A operand is read from
 // tensor memory (K-major: lane = row of A, each 32-bit column holds two consecutive K elements,
 // the lower K index in the low half), 8 columns per K = 16 step.
 SMDM_DEV void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
@@ -354,19 +354,8 @@ SMDM_DEV void umma_commit(uint64_t* bar) {
       : "memory");
 }
 
-// Instruction descriptor: bf16 x bf16 -> f32, M x N, A/B major given (0 = K-major, 1 = MN-major).
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
-  return (1u << 4)                          // D format: f32
-         | (1u << 7)                        // A format: bf16
-         | (1u << 10)                       // B format: bf16
-         | (uint32_t(a_mn_major) << 15)     // A major
-         | (uint32_t(b_mn_major) << 16)     // B major
-         | (uint32_t(N >> 3) << 17)         // N / 8
-         | (uint32_t(M >> 4) << 24);        // M / 16
-}
-
-// Instruction descriptor: f16 x f16 -> f32 (A and B formats 0 = f16), M x N, majors as above.
-// Both operands of one MMA always share their type.
+// Instruction descriptor: f16 x f16 -> f32 (A and B formats 0 = f16), M x N, A/B major given
+// (0 = K-major, 1 = MN-major).  Both operands of one MMA always share their type.
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn_major, int b_mn_major) {
   return (1u << 4)                          // D format: f32
          | (uint32_t(a_mn_major) << 15)     // A major
@@ -376,7 +365,7 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn_major, i
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle.
-//   K-major operand: rows of 128 B (64 bf16 along K), 8-row atoms of 1024 B; SBO = 1024 B
+//   K-major operand: rows of 128 B (64 16-bit elements along K), 8-row atoms of 1024 B; SBO = 1024 B
 //   between 8-row groups; LBO unused (1).
 //   MN-major operand: 128 B runs along M/N, K rows of 128 B; SBO = 1024 B between 8-row groups
 //   along K; LBO = byte distance between 64-element chunks along M/N.
