@@ -584,10 +584,14 @@ int attn_tc_splits(const AttnCall& c) {
   double best_cost = 1e30;
   for (int s = 1; s <= 16; ++s) {
     if (s > 1 && (s * 2 > nkv || (size_t)s * per_split > c.part_bytes || !c.part_o)) break;
-    // one CTA per SM: cost ~ waves x (key tiles per split + fixed prologue/epilogue)
+    // one CTA per SM: cost ~ waves x (key tiles per split + a CTA's fixed cost) + the combine
+    // launch, in periods of one key tile (≈1.4 µs at the 4096-token workload's last step): a
+    // CTA's fixed cost (waiting for q, a first tile on a cold instruction cache, the merge and
+    // output) is ≈8 of them, and so is the combine (measured: 8 and 8 run the 4096-token
+    // workload 1.5 % faster than 2 and 0.5; 12 / 8, 8 / 16 and 10 / 12 within 0.5 % of it)
     const long long ctas = base * s;
     const double waves = (double)((ctas + sms - 1) / sms);
-    const double cost = waves * ((nkv + s - 1) / s + 2.0) + (s > 1 ? 0.5 : 0.0);
+    const double cost = waves * ((nkv + s - 1) / s + 8.0) + (s > 1 ? 8.0 : 0.0);
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best = s;
