@@ -13,7 +13,7 @@
 // the grid, every CTA takes one whole tile instead.  Warp roles: warps 0 and 6 issue TMA loads
 // (alternate pipeline stages), warp 1 owns TMEM and issues tcgen05.mma (straight-line per
 // 64-wide K chunk), warps 2-5 drain the accumulator through the fused epilogue, which writes
-// its 32-row blocks with TMA / bulk copies.
+// its 32-row blocks with TMA stores (K/V cache rows, scattered, with 16-byte stores).
 //
 // fp32 path (SIMT FFMA): the same tiles and epilogues for fp32 models, where a tf32 MMA would
 // not hold the 1e-4 tolerance.
